@@ -1,0 +1,170 @@
+/*
+ * pisa.h -- C ABI of the B200 (sm_100a) PISA block-sparse attention library.
+ *
+ * PISA ("Block Sparse Attention with Log-Linear Complexity") selects, for every
+ * query, K leaf blocks of C keys by walking a mean-pooled key pyramid from the
+ * root down, keeping the Top-K nodes at each level, and then runs causal softmax
+ * attention over the keys of the selected leaves. Citations below name the page
+ * "论文精读 · Block Sparse Attention with Log-Linear Complexity (PISA)"
+ * (qqtang-code.github.io) as "close reading", by section and equation.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * Layout.   Q, O: [B, Hq, N, d]; K, V: [B, Hkv, N, d]; all contiguous, row-major,
+ *           element type cfg->dtype (fp32 or bf16). pyr: fp32 [B, Hkv, R, d] with
+ *           R = pisa_pyramid_rows(cfg), levels 1..L concatenated (leaves first).
+ *           idx: int32 [B, Hkv, N, K]: per query position and KV head, the selected
+ *           leaf indices sorted ascending, padded with -1 when fewer than K leaves
+ *           are eligible. Leaf i covers tokens [i*C, min((i+1)*C, N)).
+ * Indices.  0-based. Node i of level l covers tokens [i*C*g^(l-1), ...).
+ * Heads.    G = Hq / Hkv query heads share one KV head; selection runs per
+ *           (token, KV head) with node scores summed over the G heads (close
+ *           reading §04 4.4, Eq.(11)); MHA is G = 1.
+ * Causal.   When cfg->causal, query t sees key j iff j <= t; nodes whose first
+ *           token is > t are not candidates; nodes containing t are always kept
+ *           and never ranked (close reading §5.3).
+ * Forced.   cfg->forced_mask bit0 = first leaf, bit1 = previous leaf, bit2 =
+ *           current leaf (implied when causal); their ancestor paths are kept
+ *           unranked and they count against K (close reading §5.3, Eq.(6)).
+ * Ties.     Equal scores rank the lower node index first.
+ * Memory.   The caller owns every buffer (device memory unless stated). The
+ *           library allocates nothing and keeps no state between calls.
+ * Streams.  `stream` is a cudaStream_t passed as void*; NULL is the legacy
+ *           default stream. Every call only enqueues work; it returns before
+ *           the GPU finishes, and the caller synchronises.
+ * Errors.   Calls return PISA_OK (0) or a negative PISA_E_* code. Arguments are
+ *           validated on the host before anything is enqueued; a call that
+ *           fails validation writes nothing. PISA_E_CUDA reports a launch error
+ *           (cudaGetLastError after the launch). No device-side assert or trap
+ *           is ever used.
+ * Limits.   GPU path: g = 2, d in {64, 128}, 1 <= K <= 16, 1 <= C <= 1024,
+ *           G in {1, 2, 4, 8, 16}, at most 32 pyramid levels, N < 2^31,
+ *           16-byte aligned tensor pointers.
+ */
+#ifndef PISA_H
+#define PISA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum pisa_dtype { PISA_DTYPE_F32 = 0, PISA_DTYPE_BF16 = 1 };
+
+enum pisa_status {
+    PISA_OK = 0,
+    PISA_E_INVALID = -1,      /* null pointer, bad size, inconsistent config */
+    PISA_E_UNSUPPORTED = -2,  /* valid for the method, outside the GPU limits */
+    PISA_E_CUDA = -3,         /* a CUDA launch or runtime call failed */
+    PISA_E_ALIGNMENT = -4     /* a tensor pointer is not 16-byte aligned */
+};
+
+/* Problem statement (close reading §02-§04: N, d, C, K, g, causal). */
+typedef struct pisa_cfg {
+    int32_t B;            /* batch (sequences) */
+    int32_t Hq;           /* query heads */
+    int32_t Hkv;          /* key/value heads; Hq % Hkv == 0 */
+    int32_t N;            /* tokens per sequence (decode calls: cache capacity) */
+    int32_t d;            /* head dimension */
+    int32_t C;            /* leaf block size g_0 (Eq.(3)) */
+    int32_t K;            /* blocks kept per level (Eq.(6)) */
+    int32_t g;            /* branching factor above the leaves (Eq.(3)); must be 2 */
+    int32_t causal;       /* 1: causal mask and causal eligibility; 0: none */
+    int32_t forced_mask;  /* bit0 first, bit1 previous, bit2 current leaf */
+    int32_t dtype;        /* enum pisa_dtype of Q, K, V, O and the decode caches */
+} pisa_cfg;
+
+/* ---- geometry (close reading §04 4.1, Eq.(3)) -------------------------------
+ * M_1 = ceil(N / C), M_{l+1} = ceil(M_l / g), L = first level with one node. */
+
+/* Number of pyramid levels L (0 when N == 0; negative status on a bad cfg). */
+int pisa_num_levels(const pisa_cfg *cfg);
+/* M_l, nodes of level l (1 <= l <= L); negative status on error. */
+int64_t pisa_level_nodes(const pisa_cfg *cfg, int level);
+/* Row offset of level l inside one (b, kv-head) pyramid; negative on error. */
+int64_t pisa_level_offset(const pisa_cfg *cfg, int level);
+/* R = sum_l M_l: fp32 rows of d elements per (b, kv-head) pyramid. The whole
+ * pyramid buffer holds B * Hkv * R * d floats. Negative status on error. */
+int64_t pisa_pyramid_rows(const pisa_cfg *cfg);
+
+/* ---- prefill path ------------------------------------------------------------ */
+
+/* Key pyramid (close reading §04 4.1, Eq.(3)-(4)): leaf summaries are the mean
+ * of the C raw keys of each leaf, every higher node the mean of its existing
+ * children summaries; all levels are written.
+ * K: [B, Hkv, N, d] (dtype); pyr: fp32 [B, Hkv, R, d] (written). */
+int pisa_build_pyramid(const pisa_cfg *cfg, const void *K, float *pyr, void *stream);
+
+/* Pyramid Top-K selection (close reading §04 4.2-4.4, Eq.(5)-(7), (11); §5.3).
+ * For every (b, kv-head, t): start from the root; at each level the candidates
+ * are the eligible children of the nodes kept one level up; when there are at
+ * most K of them all are kept, otherwise the forced ones plus the best-scoring
+ * others up to K, where a node's score is the LSE over its child summaries of
+ * q . kbar / sqrt(d) (raw keys at the leaves) summed over the G query heads.
+ * Q: [B, Hq, N, d]; K: [B, Hkv, N, d]; pyr from pisa_build_pyramid;
+ * idx: int32 [B, Hkv, N, K] (written). */
+int pisa_select(const pisa_cfg *cfg, const void *Q, const void *K, const float *pyr,
+                int32_t *idx, void *stream);
+
+/* Attention over the selected blocks (close reading §02, Eq.(2)): for query
+ * head h at position t, softmax(q . k_j / sqrt(d)) over the keys j of the leaves
+ * in idx[b, h / G, t, :] (j <= t when causal), applied to V. The score matrix
+ * is never stored. Q: [B, Hq, N, d]; K, V: [B, Hkv, N, d]; idx as written by
+ * pisa_select (entries < 0 are skipped); O: [B, Hq, N, d] (written, dtype). */
+int pisa_sparse_attn(const pisa_cfg *cfg, const void *Q, const void *K, const void *V,
+                     const int32_t *idx, void *O, void *stream);
+
+/* The whole prefill path, in order on one stream: pisa_build_pyramid, then
+ * pisa_select, then pisa_sparse_attn. pyr and idx are caller-owned outputs. */
+int pisa_forward(const pisa_cfg *cfg, const void *Q, const void *K, const void *V,
+                 float *pyr, int32_t *idx, void *O, void *stream);
+
+/* Flat block selection, the quadratic comparison (close reading §02, Eq.(1)):
+ * every eligible leaf is scored by q . kbar_i / sqrt(d) against its mean
+ * summary (summed over the G heads), with the same forced/causal rules and
+ * ranking key as pisa_select. Reads only level 1 of pyr.
+ * Q: [B, Hq, N, d]; idx: int32 [B, Hkv, N, K] (written). */
+int pisa_bsa_select(const pisa_cfg *cfg, const void *Q, const float *pyr, int32_t *idx,
+                    void *stream);
+
+/* ---- decode path (close reading §5.1 last paragraph; §5.3 "decode cache") ----
+ * For decode calls cfg->N is the cache CAPACITY: Kc, Vc: [B, Hkv, N, d] and the
+ * pyramid is laid out for length N (pisa_pyramid_rows(cfg) rows per head).
+ * pos: int32 [B] device array, the position n of each sequence's new token
+ * (its cache length before the append). Rows with pos[b] outside [0, N) are
+ * left untouched by the append and produce idx = -1 and o = 0 in the step. */
+
+/* Pyramid of the first len[b] keys of each cached sequence (len: int32 [B]
+ * device array, values clamped to [0, N]), laid out for capacity N. */
+int pisa_build_pyramid_prefix(const pisa_cfg *cfg, const void *Kc, const int32_t *len,
+                              float *pyr, void *stream);
+
+/* Append one token per sequence: k_new, v_new [B, Hkv, d] are written to cache
+ * row pos[b]; the leaf holding pos[b] and each of its ancestors is recomputed
+ * as the mean of what exists at length pos[b] + 1 (O(C + L) work per head). */
+int pisa_pyramid_append(const pisa_cfg *cfg, void *Kc, void *Vc, float *pyr,
+                        const void *k_new, const void *v_new, const int32_t *pos,
+                        void *stream);
+
+/* One fused decode step (close reading §5.1: a single-stage kernel per query
+ * that walks the levels, scores the leaves and attends): for each sequence b
+ * and KV head, select K leaves for the query q_new[b] at t = pos[b] against
+ * the first pos[b] + 1 cached keys, then attend over them.
+ * q_new: [B, Hq, d]; idx: int32 [B, Hkv, K] (written); o: [B, Hq, d] (written). */
+int pisa_decode(const pisa_cfg *cfg, const void *q_new, const void *Kc, const void *Vc,
+                const float *pyr, const int32_t *pos, int32_t *idx, void *o, void *stream);
+
+/* ---- misc --------------------------------------------------------------------- */
+
+/* Static English text for a status code (never NULL). */
+const char *pisa_status_string(int status);
+/* Library version string, e.g. "pisa-b200 0.1.0 sm_100a". */
+const char *pisa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PISA_H */
