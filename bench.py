@@ -1,0 +1,558 @@
+#!/usr/bin/env python
+"""Prefill benchmark of the PISA path (pyramid pooling -> pyramid Top-K
+selection -> sparse attention) on B200, one process per GPU.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl pisa|reference]
+                    [--workload mha8_n256k] [--no-decode] [--no-cpu-baseline]
+
+A step is one pisa_forward over the whole workload (B*N tokens, all heads)
+with inputs resident in HBM. Rank 0 prints one JSON line. Under torchrun
+every rank runs its own seeded copy of the workload (weak scaling, no
+data-path collective); the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+FP32_LANES_PER_SM = 128
+SM_COUNT = 148
+
+
+def peaks():
+    """Measured peaks (driver-written) or the recipe's fallback."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "sm_max_mhz": d.get("sm_max_mhz", 1965.0),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0,
+            "source": "fallback"}
+
+
+def fp32_fma_peak_tflops(sm_mhz: float) -> float:
+    """CUDA-core fp32 FMA peak: SMs x 128 lanes x 2 FLOP x clock."""
+    return SM_COUNT * FP32_LANES_PER_SM * 2 * sm_mhz * 1e6 / 1e12
+
+
+# ---------------------------------------------------------------- work model ----
+
+def walk_counts(N: int, C: int, K: int, forced_mask: int):
+    """Per query position t (causal): dots scored at internal levels, raw keys
+    scored at the leaves, and keys attended. Exact for the causal walk: only
+    WHICH non-forced nodes survive depends on the data; how many candidates each
+    level has depends on t alone (non-forced survivors are wholly in the past
+    and have both children; forced paths are fixed by t)."""
+    t = np.arange(N, dtype=np.int64)
+    c = t // C
+    M1 = -(-N // C)
+    L = 1
+    m = M1
+    while m > 1:
+        m = -(-m // 2)
+        L += 1
+    n = np.ones(N, np.int64)            # candidates at the current level
+    internal = np.zeros(N, np.int64)
+    leafkeys = np.zeros(N, np.int64)
+    attended = np.zeros(N, np.int64)
+    for lvl in range(L, 0, -1):
+        s = lvl - 1
+        cur = c >> s
+        fs = [cur]
+        if forced_mask & 1:
+            fs.append(np.where(cur != 0, 0, -1))
+        if forced_mask & 2:
+            prev = np.where(c >= 1, (c - 1) >> s, -1)
+            prev = np.where((prev == cur) | ((forced_mask & 1) & (prev == 0)), -1, prev)
+            fs.append(prev)
+        nf = sum((f >= 0).astype(np.int64) for f in fs)
+        kept = np.minimum(n, K)
+        scored = np.where((n > K) & (K - nf > 0), n - nf, 0)
+        if lvl >= 2:
+            internal += scored * 2
+            span_child = C << (lvl - 2)
+            nxt = 2 * (kept - nf)
+            for f in fs:
+                ok = f >= 0
+                right_ok = (2 * f + 1) * span_child <= t
+                nxt += np.where(ok, 1 + right_ok.astype(np.int64), 0)
+            n = nxt
+        else:
+            leafkeys += scored * C
+            att = (kept - nf) * C + (t - c * C + 1)
+            for f in fs[1:]:
+                att += np.where(f >= 0, C, 0)
+            attended += att
+    return internal, leafkeys, attended
+
+
+def algorithmic(w, N: int):
+    """Per-launch algorithmic FLOPs and compulsory bytes of one prefill step."""
+    internal, leafkeys, attended = walk_counts(N, w.C, w.K, w.forced_mask)
+    G = w.Hq // w.Hkv
+    units = w.B * w.Hkv
+    e = 2 if w.dtype == "bf16" else 4
+    d = w.d
+    from hierarchical_block_sparse_b200.workloads import Workload  # noqa: F401
+    M1 = -(-N // w.C)
+    rows = 0
+    m = M1
+    while True:
+        rows += m
+        if m == 1:
+            break
+        m = -(-m // 2)
+    q_b = w.B * w.Hq * N * d * e
+    k_b = w.B * w.Hkv * N * d * e
+    pyr_b = w.B * w.Hkv * rows * d * 4
+    idx_b = w.B * w.Hkv * N * w.K * 4
+    return {
+        "select_flops": float(units * G * (internal.sum() + leafkeys.sum()) * 2 * d),
+        "attn_flops": float(units * G * attended.sum() * 4 * d),
+        "select_dots_per_query": float((internal.sum() + leafkeys.sum()) / N),
+        "attended_keys_per_query": float(attended.sum() / N),
+        "pool_bytes": float(k_b + pyr_b),
+        "select_bytes": float(q_b + k_b + pyr_b + idx_b),
+        "attn_bytes": float(q_b + 2 * k_b + idx_b + q_b),
+        "prefill_bytes": float(q_b + 2 * k_b + q_b + pyr_b + idx_b),
+        "selection_bytes": float(q_b + k_b + pyr_b + idx_b),
+    }
+
+
+def source_sha(files):
+    h = hashlib.sha256()
+    for f in files:
+        h.update(open(os.path.join(ROOT, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+KERNEL_SOURCES = {
+    "pool": ["hierarchical_block_sparse_b200/csrc/pool.cu", "hierarchical_block_sparse_b200/csrc/pisa_device.cuh"],
+    "select": ["hierarchical_block_sparse_b200/csrc/select.cu", "hierarchical_block_sparse_b200/csrc/pisa_walk.cuh",
+               "hierarchical_block_sparse_b200/csrc/pisa_device.cuh"],
+    "attn": ["hierarchical_block_sparse_b200/csrc/attn.cu", "hierarchical_block_sparse_b200/csrc/pisa_attn.cuh",
+             "hierarchical_block_sparse_b200/csrc/pisa_walk.cuh", "hierarchical_block_sparse_b200/csrc/pisa_device.cuh"],
+}
+
+
+def measured_traffic(kernel: str, workload: str):
+    """dram read+write bytes per launch from profiles/ncu_traffic.json, if the
+    kernel's sources are unchanged since the counters were taken."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        d = json.load(open(p)).get(kernel)
+    except Exception:
+        return None
+    if not d or d.get("workload") != workload or d.get("source_sha") != source_sha(KERNEL_SOURCES[kernel]):
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+# ------------------------------------------------------------------- clocks ----
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+             "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+             "clocks_event_reasons.sw_power_cap")
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.dev), f"--query-gpu={q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.t.join(timeout=2)
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": float(max(mx)), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------ cpu baseline ----
+
+def oracle_prefill_sample(w, Q, K, V, rows_per_head: int, rng_seed: int = 0):
+    """Time the oracle (fp64, OpenMP) on: the full pyramid of every KV head and
+    selection + attention for `rows_per_head` sampled query rows of every head.
+    Returns (seconds_pyramid, seconds_rows, rows_per_head)."""
+    from oracle import oracle
+    N = Q.shape[2]
+    G = w.Hq // w.Hkv
+    rng = np.random.default_rng(rng_seed)
+    rows = np.sort(rng.choice(N, size=min(rows_per_head, N), replace=False)).astype(np.int64)
+    tt = __import__("torch").as_tensor(rows)
+    Kf = [[oracle.to_f64(K[b, h]) for h in range(w.Hkv)] for b in range(w.B)]
+    Vf = [[oracle.to_f64(V[b, h]) for h in range(w.Hkv)] for b in range(w.B)]
+    Qf = [[oracle.to_f64(Q[b, h * G:(h + 1) * G][:, tt]).transpose(1, 0, 2).copy() for h in range(w.Hkv)]
+          for b in range(w.B)]
+    t0 = time.perf_counter()
+    P = [[oracle.build_pyramid(Kf[b][h], w.C) for h in range(w.Hkv)] for b in range(w.B)]
+    t1 = time.perf_counter()
+    for b in range(w.B):
+        for h in range(w.Hkv):
+            idx, _ = oracle.select_rows(Qf[b][h], rows, Kf[b][h], P[b][h], C=w.C, K=w.K, causal=w.causal,
+                                        forced_mask=w.forced_mask)
+            for j in range(G):
+                oracle.attn_rows(Qf[b][h][:, j], rows, Kf[b][h], Vf[b][h], idx, C=w.C, causal=w.causal)
+    t2 = time.perf_counter()
+    return t1 - t0, t2 - t1, len(rows)
+
+
+def oracle_tokens_per_s(w, N, t_pyr, t_rows, nrows):
+    """Extrapolate a sample to the whole workload: pyramid once + N rows."""
+    per_row = t_rows / nrows
+    total = t_pyr + N * per_row
+    return w.B * N / total, total
+
+
+def size_oracle_sample(w, Q, K, V, target_s: float):
+    t_pyr, t_rows, n = oracle_prefill_sample(w, Q, K, V, 256)
+    per_row = t_rows / n
+    budget = max(target_s - t_pyr, 0.5)
+    return int(min(max(8, budget / max(per_row, 1e-6)), Q.shape[2]))
+
+
+# -------------------------------------------------------------------- main ----
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="pisa", choices=["pisa", "reference"])
+    ap.add_argument("--workload", default="mha8_n256k")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-bsa", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        print("warning: --warmup raised to 3", file=sys.stderr)
+        args.warmup = 3
+
+    import torch
+    from hierarchical_block_sparse_b200 import pisa
+    from hierarchical_block_sparse_b200.workloads import WORKLOADS, make_inputs
+
+    w = WORKLOADS[args.workload]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    config = {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d, "C": w.C, "K": w.K,
+              "g": w.g, "causal": w.causal, "forced_mask": w.forced_mask,
+              "l2": "inputs larger than L2 (Q, K, V, O exceed 126 MB)",
+              "parallelism": f"replicas{world}" if world > 1 else "single"}
+    metric = "prefill tokens/s"
+    unit = "tokens/s"
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        return reference_arm(args, w, config, metric, unit)
+
+    if not torch.cuda.is_available():
+        raise RuntimeError("bench.py needs a CUDA device")
+    pisa.load()
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+
+    Q, K, V, meta = make_inputs(w, seed=w.seed + rank)
+    Qd, Kd, Vd = Q.to(dev), K.to(dev), V.to(dev)
+    cfg = pisa.cfg_for(Qd, Kd, C=w.C, K_=w.K, causal=w.causal, forced_mask=w.forced_mask)
+    pyr, idx, O = pisa.alloc_outputs(cfg, dev, Qd.dtype)
+    stream = torch.cuda.current_stream()
+    launches_per_step = 3 + (1 if pisa.pisa_num_levels(cfg) >= 6 else 0)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        pisa.pisa_build_pyramid(cfg, Kd, pyr)
+        if ev is not None:
+            ev[1].record(stream)
+        pisa.pisa_select(cfg, Qd, Kd, pyr, idx)
+        if ev is not None:
+            ev[2].record(stream)
+        pisa.pisa_sparse_attn(cfg, Qd, Kd, Vd, idx, O)
+        if ev is not None:
+            ev[3].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    with ClockSampler(dev.index) as clk:
+        for s in range(args.steps):
+            step(evs[s])
+        torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    total_ms = evs[0][0].elapsed_time(evs[-1][3])
+    pool_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
+    sel_ms = float(np.mean([e[1].elapsed_time(e[2]) for e in evs]))
+    attn_ms = float(np.mean([e[2].elapsed_time(e[3]) for e in evs]))
+    if dist:
+        tt = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        total_ms = float(tt.item())
+    ms_per_step = total_ms / args.steps
+    tokens = w.B * w.N * world
+    value = tokens / (ms_per_step / 1e3)
+
+    alg = algorithmic(w, w.N)
+    pk = peaks()
+    clocks = clk.summary()
+    fma_peak = fp32_fma_peak_tflops(pk["sm_max_mhz"])
+    times = {"pool": pool_ms, "select": sel_ms, "attn": attn_ms}
+    dom = max(times, key=times.get)
+    if dom == "pool":
+        achieved = alg["pool_bytes"] / (pool_ms / 1e3) / 1e9
+        roof = {"kernel": "pool_leaves_kernel+pool_top_kernel", "bound": "hbm", "achieved": achieved,
+                "peak": pk["hbm_gbs"], "unit": "GB/s"}
+    else:
+        flops = alg["select_flops"] if dom == "select" else alg["attn_flops"]
+        achieved = flops / (times[dom] / 1e3) / 1e12
+        roof = {"kernel": "select_kernel" if dom == "select" else "attn_kernel", "bound": "alu",
+                "achieved": achieved, "peak": fma_peak, "unit": "TFLOP/s",
+                "peak_note": "fp32 FMA: 148 SMs x 128 lanes x 2 FLOP x max SM clock"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = measured_traffic(dom, w.name)
+    roof["algorithmic_per_launch"] = alg["pool_bytes"] if dom == "pool" else (
+        alg["select_flops"] if dom == "select" else alg["attn_flops"])
+    roof["launch_ms"] = times[dom]
+
+    sel_total = pool_ms + sel_ms
+    hbm = pk["hbm_gbs"] * 1e9
+    out = {
+        "metric": metric, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic (seeded i.i.d. N(0,1))",
+        "config": config,
+        "selection_ms": sel_total, "pool_ms": pool_ms, "select_ms": sel_ms, "attn_ms": attn_ms,
+        "hbm_roofline_frac": {"prefill": alg["prefill_bytes"] / (ms_per_step / 1e3) / hbm,
+                              "selection": alg["selection_bytes"] / (sel_total / 1e3) / hbm,
+                              "pool": alg["pool_bytes"] / (pool_ms / 1e3) / hbm},
+        "work": {"select_dots_per_query": alg["select_dots_per_query"],
+                 "attended_keys_per_query": alg["attended_keys_per_query"],
+                 "select_tflop": alg["select_flops"] / 1e12, "attn_tflop": alg["attn_flops"] / 1e12},
+        "roofline": roof,
+        "peaks_source": pk["source"],
+        "clocks": clocks,
+        "gpu_launches": launches_per_step * args.steps,
+    }
+
+    # ---- end to end through the public API: pinned host -> device -> host ----
+    Qh, Kh, Vh = Q.pin_memory(), K.pin_memory(), V.pin_memory()
+    Oh = torch.empty(O.shape, dtype=O.dtype, pin_memory=True)
+    Ih = torch.empty(idx.shape, dtype=idx.dtype, pin_memory=True)
+
+    def e2e_step():
+        Qd.copy_(Qh, non_blocking=True)
+        Kd.copy_(Kh, non_blocking=True)
+        Vd.copy_(Vh, non_blocking=True)
+        pisa.pisa_forward(cfg, Qd, Kd, Vd, pyr, idx, O)
+        Oh.copy_(O, non_blocking=True)
+        Ih.copy_(idx, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n_e2e = max(3, min(args.steps, 5))
+    e0.record(stream)
+    for _ in range(n_e2e):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / n_e2e
+    if dist:
+        tt = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_ms = float(tt.item())
+    out["e2e"] = {"value": tokens / (e2e_ms / 1e3), "unit": unit,
+                  "h2d_bytes_per_step": int(Qh.nbytes + Kh.nbytes + Vh.nbytes),
+                  "d2h_bytes_per_step": int(Oh.nbytes + Ih.nbytes), "ms_per_step": e2e_ms}
+    del Qh, Kh, Vh, Oh, Ih
+
+    # ---- flat BSA selection, the quadratic comparison ----
+    if not args.no_bsa:
+        bidx = torch.empty_like(idx)
+        pisa.pisa_build_pyramid(cfg, Kd, pyr)
+        pisa.pisa_bsa_select(cfg, Qd, pyr, bidx)
+        torch.cuda.synchronize()
+        b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        b0.record(stream)
+        pisa.pisa_build_pyramid(cfg, Kd, pyr)
+        pisa.pisa_bsa_select(cfg, Qd, pyr, bidx)
+        b1.record(stream)
+        torch.cuda.synchronize()
+        out["bsa_selection_ms"] = b0.elapsed_time(b1)
+        out["pisa_vs_bsa_selection_speedup"] = out["bsa_selection_ms"] / sel_total
+        del bidx
+
+    # ---- decode: 64 sequences, one new token each, against 256K-key caches ----
+    if not args.no_decode and w.decode_batch:
+        out["decode"] = bench_decode(w, dev, stream)
+
+    del Qd, Kd, Vd, pyr, idx, O
+    torch.cuda.empty_cache()
+
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        n = size_oracle_sample(w, Q, K, V, args.cpu_seconds)
+        t_pyr, t_rows, nr = oracle_prefill_sample(w, Q, K, V, n, rng_seed=1)
+        from oracle import oracle
+        v, total = oracle_tokens_per_s(w, w.N, t_pyr, t_rows, nr)
+        out["cpu_baseline"] = {"value": v, "unit": unit, "cores": oracle.threads(), "kind": "oracle",
+                               "sample": f"full fp64 pyramid of all {w.B * w.Hkv} KV heads ({t_pyr:.2f} s) + "
+                                         f"selection and attention for {nr} random query rows of every head "
+                                         f"({t_rows:.2f} s), extrapolated to all {w.N} rows"}
+    if rank == 0:
+        print(json.dumps(out))
+    return 0
+
+
+def bench_decode(w, dev, stream, steps: int = 8):
+    import torch
+    from hierarchical_block_sparse_b200 import pisa
+    from hierarchical_block_sparse_b200.workloads import decode_cache, decode_step_inputs
+    prefix = w.N
+    cap = prefix + 64
+    B = w.decode_batch
+    Kc, Vc, _, _ = decode_cache(w, cap, prefix, dev)
+    cfg = pisa.make_cfg(B=B, Hq=w.Hq, Hkv=w.Hkv, N=cap, d=w.d, C=w.C, K=w.K, causal=True,
+                        forced_mask=w.forced_mask, dtype=Kc.dtype)
+    pyr = torch.empty((B, w.Hkv, pisa.pisa_pyramid_rows(cfg), w.d), dtype=torch.float32, device=dev)
+    pos = torch.full((B,), prefix, dtype=torch.int32, device=dev)
+    pisa.pisa_build_pyramid_prefix(cfg, Kc, pos, pyr)
+    ins = [tuple(x.to(dev) for x in decode_step_inputs(w, s)) for s in range(steps + 3)]
+    idx = torch.empty((B, w.Hkv, w.K), dtype=torch.int32, device=dev)
+    o = torch.empty((B, w.Hq, w.d), dtype=Kc.dtype, device=dev)
+    for s in range(3):
+        q, k, v = ins[s]
+        pisa.pisa_pyramid_append(cfg, Kc, Vc, pyr, k, v, pos)
+        pisa.pisa_decode(cfg, q, Kc, Vc, pyr, pos, idx, o)
+        pos += 1
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    for s in range(steps):
+        q, k, v = ins[3 + s]
+        ev[s][0].record(stream)
+        pisa.pisa_pyramid_append(cfg, Kc, Vc, pyr, k, v, pos)
+        ev[s][1].record(stream)
+        pisa.pisa_decode(cfg, q, Kc, Vc, pyr, pos, idx, o)
+        ev[s][2].record(stream)
+        pos += 1
+    torch.cuda.synchronize()
+    app = float(np.mean([e[0].elapsed_time(e[1]) for e in ev])) * 1e3
+    dec = float(np.mean([e[1].elapsed_time(e[2]) for e in ev])) * 1e3
+    # gathered bytes per step (per sequence and KV head): the scored internal
+    # children summaries, the scored leaves' raw keys and the attended K and V rows
+    internal, leafkeys, attended = walk_counts(prefix + 8, w.C, w.K, w.forced_mask)
+    tlast = prefix + 4
+    G = w.Hq // w.Hkv
+    e = 2 if w.dtype == "bf16" else 4
+    per_unit = internal[tlast] * w.d * 4 + leafkeys[tlast] * w.d * e + 2 * attended[tlast] * w.d * e + \
+        (G * 2 * w.d * e)
+    step_bytes = per_unit * B * w.Hkv
+    us = app + dec
+    pk = peaks()
+    del Kc, Vc, pyr
+    return {"batch": B, "cache_keys": prefix, "us_per_step": us, "append_us": app, "decode_kernel_us": dec,
+            "tokens_per_s": B / (us / 1e6), "gathered_bytes_per_step": int(step_bytes),
+            "hbm_roofline_frac": step_bytes / (dec / 1e6) / (pk["hbm_gbs"] * 1e9)}
+
+
+def reference_arm(args, w, config, metric, unit):
+    """The oracle (fp64 CPU, the reference computation of this method), timed on
+    the host cores on a bounded sample of the same workload per step."""
+    from hierarchical_block_sparse_b200.workloads import make_inputs
+    from oracle import oracle
+    Q, K, V, _ = make_inputs(w)
+    n = size_oracle_sample(w, Q, K, V, 4.0)
+    for _ in range(args.warmup):
+        oracle_prefill_sample(w, Q, K, V, max(8, n // 8), rng_seed=99)
+    vals, secs = [], []
+    for s in range(args.steps):
+        t_pyr, t_rows, nr = oracle_prefill_sample(w, Q, K, V, n, rng_seed=s)
+        v, _ = oracle_tokens_per_s(w, w.N, t_pyr, t_rows, nr)
+        vals.append(v)
+        secs.append(t_pyr + t_rows)
+    value = float(np.mean(vals))
+    sample = (f"per step: full fp64 pyramid of all {w.B * w.Hkv} KV heads + selection and attention for {n} "
+              f"random query rows of every head, extrapolated to all {w.N} rows")
+    out = {"metric": metric, "value": value, "unit": unit, "n_gpus": args.gpus, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": float(np.mean(secs)) * 1e3, "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded i.i.d. N(0,1))",
+           "config": config, "impl": "reference",
+           "cpu_baseline": {"value": value, "unit": unit, "cores": oracle.threads(), "kind": "oracle",
+                            "sample": sample},
+           "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out))
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,246 @@
+// api.cu -- the extern "C" boundary declared in include/pisa.h: argument
+// validation on the host, geometry, and dispatch to the kernel launchers.
+// Nothing is enqueued unless every check passes; no call allocates memory.
+#include <math.h>
+#include <stdint.h>
+
+#include "pisa.h"
+#include "pisa_internal.h"
+
+using namespace pisa;
+
+namespace {
+
+// checks that need no device: the problem statement itself
+int check_cfg(const pisa_cfg* c) {
+    if (!c) return PISA_E_INVALID;
+    if (c->B < 1 || c->Hq < 1 || c->Hkv < 1 || c->N < 0 || c->d < 1 || c->C < 1 || c->K < 1 || c->g < 2)
+        return PISA_E_INVALID;
+    if (c->Hq % c->Hkv != 0) return PISA_E_INVALID;
+    if (c->causal != 0 && c->causal != 1) return PISA_E_INVALID;
+    if (c->forced_mask < 0 || c->forced_mask > 7) return PISA_E_INVALID;
+    if (c->dtype != PISA_DTYPE_F32 && c->dtype != PISA_DTYPE_BF16) return PISA_E_INVALID;
+    const int forced = c->forced_mask | (c->causal ? 4 : 0);
+    const int nf = (forced & 1) + ((forced >> 1) & 1) + ((forced >> 2) & 1);
+    if (c->K < nf) return PISA_E_INVALID;  // forced leaves count against K (Eq.6)
+    return PISA_OK;
+}
+
+// limits of the GPU kernels
+int check_gpu(const pisa_cfg* c) {
+    int s = check_cfg(c);
+    if (s) return s;
+    if (c->g != 2) return PISA_E_UNSUPPORTED;
+    if (c->d != 64 && c->d != 128) return PISA_E_UNSUPPORTED;
+    if (c->K > 16) return PISA_E_UNSUPPORTED;
+    if (c->C > 1024) return PISA_E_UNSUPPORTED;
+    const int G = c->Hq / c->Hkv;
+    if (G != 1 && G != 2 && G != 4 && G != 8 && G != 16) return PISA_E_UNSUPPORTED;
+    Geom g;
+    if (make_geom(c->N, c->C, &g) < 0) return PISA_E_UNSUPPORTED;
+    return PISA_OK;
+}
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? PISA_OK : PISA_E_CUDA; }
+
+// generic geometry for any g >= 2 (host only)
+int geom_any(const pisa_cfg* c, int64_t* M, int64_t* off, int maxl) {
+    if (c->N == 0) return 0;
+    int L = 1;
+    M[1] = ((int64_t)c->N + c->C - 1) / c->C;
+    off[1] = 0;
+    while (M[L] > 1) {
+        if (L + 1 > maxl) return -1;
+        M[L + 1] = (M[L] + c->g - 1) / c->g;
+        off[L + 1] = off[L] + M[L];
+        ++L;
+    }
+    return L;
+}
+
+SelectParams select_params(const pisa_cfg* c, const Geom& g) {
+    SelectParams p;
+    p.B = c->B; p.Hq = c->Hq; p.Hkv = c->Hkv; p.N = c->N; p.C = c->C; p.K = c->K;
+    p.causal = c->causal; p.forced_mask = c->forced_mask;
+    p.qscale = (float)(1.4426950408889634 / sqrt((double)c->d));
+    p.geom = g;
+    return p;
+}
+
+PoolParams pool_params(const pisa_cfg* c, const Geom& g, const int32_t* len) {
+    PoolParams p;
+    p.B = c->B; p.Hkv = c->Hkv; p.N = c->N; p.C = c->C;
+    p.k_rows = c->N;
+    p.len = len;
+    p.geom = g;
+    return p;
+}
+
+DecodeParams decode_params(const pisa_cfg* c, const Geom& g) {
+    DecodeParams p;
+    p.B = c->B; p.Hq = c->Hq; p.Hkv = c->Hkv; p.N = c->N; p.C = c->C; p.K = c->K;
+    p.forced_mask = c->forced_mask;
+    p.qscale = (float)(1.4426950408889634 / sqrt((double)c->d));
+    p.geom = g;
+    return p;
+}
+
+}  // namespace
+
+extern "C" {
+
+int pisa_num_levels(const pisa_cfg* cfg) {
+    int s = check_cfg(cfg);
+    if (s) return s;
+    int64_t M[65], off[65];
+    int L = geom_any(cfg, M, off, 64);
+    return L < 0 ? PISA_E_UNSUPPORTED : L;
+}
+
+int64_t pisa_level_nodes(const pisa_cfg* cfg, int level) {
+    int s = check_cfg(cfg);
+    if (s) return s;
+    int64_t M[65], off[65];
+    int L = geom_any(cfg, M, off, 64);
+    if (L < 0) return PISA_E_UNSUPPORTED;
+    if (level < 1 || level > L) return PISA_E_INVALID;
+    return M[level];
+}
+
+int64_t pisa_level_offset(const pisa_cfg* cfg, int level) {
+    int s = check_cfg(cfg);
+    if (s) return s;
+    int64_t M[65], off[65];
+    int L = geom_any(cfg, M, off, 64);
+    if (L < 0) return PISA_E_UNSUPPORTED;
+    if (level < 1 || level > L) return PISA_E_INVALID;
+    return off[level];
+}
+
+int64_t pisa_pyramid_rows(const pisa_cfg* cfg) {
+    int s = check_cfg(cfg);
+    if (s) return s;
+    int64_t M[65], off[65];
+    int L = geom_any(cfg, M, off, 64);
+    if (L < 0) return PISA_E_UNSUPPORTED;
+    return L == 0 ? 0 : off[L] + M[L];
+}
+
+int pisa_build_pyramid(const pisa_cfg* cfg, const void* K, float* pyr, void* stream) {
+    int s = check_gpu(cfg);
+    if (s) return s;
+    if (cfg->N == 0) return PISA_OK;
+    if (!K || !pyr) return PISA_E_INVALID;
+    if (!aligned16(K) || !aligned16(pyr)) return PISA_E_ALIGNMENT;
+    Geom g;
+    make_geom(cfg->N, cfg->C, &g);
+    return cuda_status(launch_pool(cfg->dtype, cfg->d, K, pyr, pool_params(cfg, g, nullptr), (cudaStream_t)stream));
+}
+
+int pisa_select(const pisa_cfg* cfg, const void* Q, const void* K, const float* pyr, int32_t* idx, void* stream) {
+    int s = check_gpu(cfg);
+    if (s) return s;
+    if (cfg->N == 0) return PISA_OK;
+    if (!Q || !K || !pyr || !idx) return PISA_E_INVALID;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(pyr) || !aligned16(idx)) return PISA_E_ALIGNMENT;
+    Geom g;
+    make_geom(cfg->N, cfg->C, &g);
+    return cuda_status(launch_select(cfg->dtype, cfg->d, Q, K, pyr, idx, select_params(cfg, g), (cudaStream_t)stream));
+}
+
+int pisa_sparse_attn(const pisa_cfg* cfg, const void* Q, const void* K, const void* V, const int32_t* idx, void* O,
+                     void* stream) {
+    int s = check_gpu(cfg);
+    if (s) return s;
+    if (cfg->N == 0) return PISA_OK;
+    if (!Q || !K || !V || !idx || !O) return PISA_E_INVALID;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(idx) || !aligned16(O)) return PISA_E_ALIGNMENT;
+    AttnParams p;
+    p.B = cfg->B; p.Hq = cfg->Hq; p.Hkv = cfg->Hkv; p.N = cfg->N; p.C = cfg->C; p.K = cfg->K;
+    p.causal = cfg->causal;
+    p.qscale = (float)(1.4426950408889634 / sqrt((double)cfg->d));
+    return cuda_status(launch_attn(cfg->dtype, cfg->d, Q, K, V, idx, O, p, (cudaStream_t)stream));
+}
+
+int pisa_forward(const pisa_cfg* cfg, const void* Q, const void* K, const void* V, float* pyr, int32_t* idx, void* O,
+                 void* stream) {
+    int s = check_gpu(cfg);
+    if (s) return s;
+    if (cfg->N == 0) return PISA_OK;
+    if (!Q || !K || !V || !pyr || !idx || !O) return PISA_E_INVALID;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(pyr) || !aligned16(idx) || !aligned16(O))
+        return PISA_E_ALIGNMENT;
+    s = pisa_build_pyramid(cfg, K, pyr, stream);
+    if (s) return s;
+    s = pisa_select(cfg, Q, K, pyr, idx, stream);
+    if (s) return s;
+    return pisa_sparse_attn(cfg, Q, K, V, idx, O, stream);
+}
+
+int pisa_bsa_select(const pisa_cfg* cfg, const void* Q, const float* pyr, int32_t* idx, void* stream) {
+    int s = check_gpu(cfg);
+    if (s) return s;
+    if (cfg->N == 0) return PISA_OK;
+    if (!Q || !pyr || !idx) return PISA_E_INVALID;
+    if (!aligned16(Q) || !aligned16(pyr) || !aligned16(idx)) return PISA_E_ALIGNMENT;
+    Geom g;
+    make_geom(cfg->N, cfg->C, &g);
+    return cuda_status(launch_bsa(cfg->dtype, cfg->d, Q, pyr, idx, select_params(cfg, g), (cudaStream_t)stream));
+}
+
+int pisa_build_pyramid_prefix(const pisa_cfg* cfg, const void* Kc, const int32_t* len, float* pyr, void* stream) {
+    int s = check_gpu(cfg);
+    if (s) return s;
+    if (cfg->N == 0) return PISA_OK;
+    if (!Kc || !len || !pyr) return PISA_E_INVALID;
+    if (!aligned16(Kc) || !aligned16(pyr)) return PISA_E_ALIGNMENT;
+    Geom g;
+    make_geom(cfg->N, cfg->C, &g);
+    return cuda_status(launch_pool(cfg->dtype, cfg->d, Kc, pyr, pool_params(cfg, g, len), (cudaStream_t)stream));
+}
+
+int pisa_pyramid_append(const pisa_cfg* cfg, void* Kc, void* Vc, float* pyr, const void* k_new, const void* v_new,
+                        const int32_t* pos, void* stream) {
+    int s = check_gpu(cfg);
+    if (s) return s;
+    if (cfg->N == 0) return PISA_OK;
+    if (!Kc || !Vc || !pyr || !k_new || !v_new || !pos) return PISA_E_INVALID;
+    if (!aligned16(Kc) || !aligned16(Vc) || !aligned16(pyr) || !aligned16(k_new) || !aligned16(v_new))
+        return PISA_E_ALIGNMENT;
+    Geom g;
+    make_geom(cfg->N, cfg->C, &g);
+    return cuda_status(launch_append(cfg->dtype, cfg->d, Kc, Vc, pyr, k_new, v_new, pos, decode_params(cfg, g),
+                                     (cudaStream_t)stream));
+}
+
+int pisa_decode(const pisa_cfg* cfg, const void* q_new, const void* Kc, const void* Vc, const float* pyr,
+                const int32_t* pos, int32_t* idx, void* o, void* stream) {
+    int s = check_gpu(cfg);
+    if (s) return s;
+    if (cfg->causal != 1) return PISA_E_INVALID;  // the new token sees only the past
+    if (cfg->N == 0) return PISA_OK;
+    if (!q_new || !Kc || !Vc || !pyr || !pos || !idx || !o) return PISA_E_INVALID;
+    if (!aligned16(q_new) || !aligned16(Kc) || !aligned16(Vc) || !aligned16(pyr) || !aligned16(o))
+        return PISA_E_ALIGNMENT;
+    Geom g;
+    make_geom(cfg->N, cfg->C, &g);
+    return cuda_status(launch_decode(cfg->dtype, cfg->d, q_new, Kc, Vc, pyr, pos, idx, o, decode_params(cfg, g),
+                                     (cudaStream_t)stream));
+}
+
+const char* pisa_status_string(int status) {
+    switch (status) {
+        case PISA_OK: return "ok";
+        case PISA_E_INVALID: return "invalid argument";
+        case PISA_E_UNSUPPORTED: return "configuration outside the GPU kernels' limits";
+        case PISA_E_CUDA: return "CUDA launch or runtime error";
+        case PISA_E_ALIGNMENT: return "tensor pointer not 16-byte aligned";
+    }
+    return "unknown status";
+}
+
+const char* pisa_version(void) { return "pisa-b200 0.1.0 sm_100a"; }
+
+}  // extern "C"

@@ -1,0 +1,48 @@
+// pisa_internal.h -- parameter blocks and launchers shared between the C-ABI
+// layer (api.cu) and the kernel translation units. Not part of the public ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "pisa_device.cuh"
+
+namespace pisa {
+
+struct PoolParams {
+    int B, Hkv, N, C;
+    int64_t k_rows;      // rows per head in K (N for prefill, capacity for caches)
+    const int32_t* len;  // optional per-sequence key count (device), else N
+    Geom geom;           // pyramid layout (for N or for the capacity)
+};
+
+struct SelectParams {
+    int B, Hq, Hkv, N, C, K, causal, forced_mask;
+    float qscale;  // log2(e) / sqrt(d)
+    Geom geom;
+};
+
+struct AttnParams {
+    int B, Hq, Hkv, N, C, K, causal;
+    float qscale;  // log2(e) / sqrt(d)
+};
+
+struct DecodeParams {
+    int B, Hq, Hkv, N, C, K, forced_mask;
+    float qscale;  // log2(e) / sqrt(d)
+    Geom geom;     // layout for the capacity N
+};
+
+cudaError_t launch_pool(int dtype, int d, const void* K, float* pyr, const PoolParams& p, cudaStream_t st);
+cudaError_t launch_select(int dtype, int d, const void* Q, const void* K, const float* pyr, int32_t* idx,
+                          const SelectParams& p, cudaStream_t st);
+cudaError_t launch_attn(int dtype, int d, const void* Q, const void* K, const void* V, const int32_t* idx,
+                        void* O, const AttnParams& p, cudaStream_t st);
+cudaError_t launch_bsa(int dtype, int d, const void* Q, const float* pyr, int32_t* idx, const SelectParams& p,
+                       cudaStream_t st);
+cudaError_t launch_append(int dtype, int d, void* Kc, void* Vc, float* pyr, const void* k_new, const void* v_new,
+                          const int32_t* pos, const DecodeParams& p, cudaStream_t st);
+cudaError_t launch_decode(int dtype, int d, const void* q_new, const void* Kc, const void* Vc, const float* pyr,
+                          const int32_t* pos, int32_t* idx, void* o, const DecodeParams& p, cudaStream_t st);
+
+}  // namespace pisa

@@ -1,0 +1,202 @@
+"""Thin Python binding of ``libpisa.so`` (include/pisa.h), same names as the C ABI.
+
+Argument marshalling only: torch tensors are passed as raw device pointers
+together with torch's current CUDA stream; every step of the path runs in the
+library's CUDA kernels. If the library is missing or a tensor is not on a CUDA
+device, the call raises -- there is no CPU fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+import threading
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libpisa.so")
+HEADER = os.path.join(os.path.dirname(_PKG), "include", "pisa.h")
+
+PISA_DTYPE_F32, PISA_DTYPE_BF16 = 0, 1
+STATUS = {0: "PISA_OK", -1: "PISA_E_INVALID", -2: "PISA_E_UNSUPPORTED", -3: "PISA_E_CUDA",
+          -4: "PISA_E_ALIGNMENT"}
+
+
+class PisaError(RuntimeError):
+    def __init__(self, fn: str, status: int, msg: str):
+        super().__init__(f"{fn} failed: {STATUS.get(status, status)} ({msg})")
+        self.status = status
+
+
+class PisaCfg(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in
+                ("B", "Hq", "Hkv", "N", "d", "C", "K", "g", "causal", "forced_mask", "dtype")]
+
+
+_lock = threading.Lock()
+_lib = None
+
+
+def exported_names() -> list[str]:
+    """Function names declared in include/pisa.h."""
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[a-z0-9_]+\s*\*?\s*(pisa_[a-z0-9_]+)\s*\(", src, re.M)))
+
+
+def load(path: str | None = None):
+    """Load libpisa.so (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is not None and path is None:
+            return _lib
+        p = path or LIB_PATH
+        if not os.path.exists(p):
+            raise RuntimeError(f"{p} is missing: build it with `python -m hierarchical_block_sparse_b200.build`")
+        lib = ctypes.CDLL(p)
+        P = ctypes.c_void_p
+        cfgp = ctypes.POINTER(PisaCfg)
+        sig = {
+            "pisa_num_levels": (ctypes.c_int, [cfgp]),
+            "pisa_level_nodes": (ctypes.c_int64, [cfgp, ctypes.c_int]),
+            "pisa_level_offset": (ctypes.c_int64, [cfgp, ctypes.c_int]),
+            "pisa_pyramid_rows": (ctypes.c_int64, [cfgp]),
+            "pisa_build_pyramid": (ctypes.c_int, [cfgp, P, P, P]),
+            "pisa_select": (ctypes.c_int, [cfgp, P, P, P, P, P]),
+            "pisa_sparse_attn": (ctypes.c_int, [cfgp, P, P, P, P, P, P]),
+            "pisa_forward": (ctypes.c_int, [cfgp, P, P, P, P, P, P, P]),
+            "pisa_bsa_select": (ctypes.c_int, [cfgp, P, P, P, P]),
+            "pisa_build_pyramid_prefix": (ctypes.c_int, [cfgp, P, P, P, P]),
+            "pisa_pyramid_append": (ctypes.c_int, [cfgp, P, P, P, P, P, P, P]),
+            "pisa_decode": (ctypes.c_int, [cfgp, P, P, P, P, P, P, P, P]),
+            "pisa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+            "pisa_version": (ctypes.c_char_p, []),
+        }
+        for name, (res, args) in sig.items():
+            fn = getattr(lib, name)
+            fn.restype, fn.argtypes = res, args
+        if path is None:
+            _lib = lib
+        return lib
+
+
+def make_cfg(*, B: int, Hq: int, Hkv: int, N: int, d: int, C: int, K: int, g: int = 2, causal: bool = True,
+             forced_mask: int = 7, dtype=torch.bfloat16) -> PisaCfg:
+    dt = {torch.bfloat16: PISA_DTYPE_BF16, torch.float32: PISA_DTYPE_F32}.get(dtype, dtype)
+    return PisaCfg(B, Hq, Hkv, N, d, C, K, g, int(causal), forced_mask, int(dt))
+
+
+def cfg_for(Q: torch.Tensor, K: torch.Tensor, *, C: int, K_: int, causal: bool = True, forced_mask: int = 7,
+            g: int = 2) -> PisaCfg:
+    B, Hq, N, d = Q.shape
+    return make_cfg(B=B, Hq=Hq, Hkv=K.shape[1], N=N, d=d, C=C, K=K_, g=g, causal=causal,
+                    forced_mask=forced_mask, dtype=Q.dtype)
+
+
+def _ptr(t: torch.Tensor | None):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensors must live on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _check(name: str, status: int):
+    if status != 0:
+        raise PisaError(name, status, load().pisa_status_string(status).decode())
+
+
+# ---- geometry -------------------------------------------------------------------
+
+def pisa_num_levels(cfg: PisaCfg) -> int:
+    return int(load().pisa_num_levels(ctypes.byref(cfg)))
+
+
+def pisa_level_nodes(cfg: PisaCfg, level: int) -> int:
+    return int(load().pisa_level_nodes(ctypes.byref(cfg), level))
+
+
+def pisa_level_offset(cfg: PisaCfg, level: int) -> int:
+    return int(load().pisa_level_offset(ctypes.byref(cfg), level))
+
+
+def pisa_pyramid_rows(cfg: PisaCfg) -> int:
+    r = int(load().pisa_pyramid_rows(ctypes.byref(cfg)))
+    if r < 0:
+        _check("pisa_pyramid_rows", r)
+    return r
+
+
+# ---- prefill ----------------------------------------------------------------------
+
+def pisa_build_pyramid(cfg, K, pyr):
+    _check("pisa_build_pyramid", load().pisa_build_pyramid(ctypes.byref(cfg), _ptr(K), _ptr(pyr), _stream()))
+
+
+def pisa_select(cfg, Q, K, pyr, idx):
+    _check("pisa_select", load().pisa_select(ctypes.byref(cfg), _ptr(Q), _ptr(K), _ptr(pyr), _ptr(idx), _stream()))
+
+
+def pisa_sparse_attn(cfg, Q, K, V, idx, O):
+    _check("pisa_sparse_attn", load().pisa_sparse_attn(ctypes.byref(cfg), _ptr(Q), _ptr(K), _ptr(V), _ptr(idx),
+                                                       _ptr(O), _stream()))
+
+
+def pisa_forward(cfg, Q, K, V, pyr, idx, O):
+    _check("pisa_forward", load().pisa_forward(ctypes.byref(cfg), _ptr(Q), _ptr(K), _ptr(V), _ptr(pyr), _ptr(idx),
+                                               _ptr(O), _stream()))
+
+
+def pisa_bsa_select(cfg, Q, pyr, idx):
+    _check("pisa_bsa_select", load().pisa_bsa_select(ctypes.byref(cfg), _ptr(Q), _ptr(pyr), _ptr(idx), _stream()))
+
+
+# ---- decode -------------------------------------------------------------------------
+
+def pisa_build_pyramid_prefix(cfg, Kc, length, pyr):
+    _check("pisa_build_pyramid_prefix", load().pisa_build_pyramid_prefix(ctypes.byref(cfg), _ptr(Kc), _ptr(length),
+                                                                         _ptr(pyr), _stream()))
+
+
+def pisa_pyramid_append(cfg, Kc, Vc, pyr, k_new, v_new, pos):
+    _check("pisa_pyramid_append", load().pisa_pyramid_append(ctypes.byref(cfg), _ptr(Kc), _ptr(Vc), _ptr(pyr),
+                                                             _ptr(k_new), _ptr(v_new), _ptr(pos), _stream()))
+
+
+def pisa_decode(cfg, q_new, Kc, Vc, pyr, pos, idx, o):
+    _check("pisa_decode", load().pisa_decode(ctypes.byref(cfg), _ptr(q_new), _ptr(Kc), _ptr(Vc), _ptr(pyr),
+                                             _ptr(pos), _ptr(idx), _ptr(o), _stream()))
+
+
+def pisa_status_string(status: int) -> str:
+    return load().pisa_status_string(status).decode()
+
+
+def pisa_version() -> str:
+    return load().pisa_version().decode()
+
+
+# ---- allocation helpers (torch owns the memory) --------------------------------------
+
+def alloc_outputs(cfg: PisaCfg, device="cuda", dtype=torch.bfloat16):
+    """pyr (fp32), idx (int32) and O tensors sized for cfg."""
+    R = pisa_pyramid_rows(cfg)
+    pyr = torch.empty((cfg.B, cfg.Hkv, R, cfg.d), dtype=torch.float32, device=device)
+    idx = torch.empty((cfg.B, cfg.Hkv, cfg.N, cfg.K), dtype=torch.int32, device=device)
+    O = torch.empty((cfg.B, cfg.Hq, cfg.N, cfg.d), dtype=dtype, device=device)
+    return pyr, idx, O
+
+
+def forward(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, *, C: int, K_: int, causal: bool = True,
+            forced_mask: int = 7):
+    """Allocate outputs and run pisa_forward. Returns (O, idx, pyr)."""
+    cfg = cfg_for(Q, K, C=C, K_=K_, causal=causal, forced_mask=forced_mask)
+    pyr, idx, O = alloc_outputs(cfg, Q.device, Q.dtype)
+    pisa_forward(cfg, Q, K, V, pyr, idx, O)
+    return O, idx, pyr

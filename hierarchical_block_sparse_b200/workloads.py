@@ -18,7 +18,8 @@ import dataclasses
 
 import numpy as np
 
-__all__ = ["Workload", "WORKLOADS", "workload", "make_inputs", "decode_pool"]
+__all__ = ["Workload", "WORKLOADS", "workload", "make_inputs", "decode_pool", "decode_offset",
+           "decode_cache", "decode_rows", "decode_step_inputs"]
 
 
 @dataclasses.dataclass(frozen=True)
@@ -115,13 +116,47 @@ def decode_pool(w: Workload, rows: int, *, seed: int | None = None):
     rng = np.random.default_rng((w.seed if seed is None else seed) + 1000)
     Kp = rng.standard_normal((w.Hkv, rows, w.d), dtype=np.float32)
     Vp = rng.standard_normal((w.Hkv, rows, w.d), dtype=np.float32)
-    Qn = rng.standard_normal((w.decode_batch, w.Hq, w.d), dtype=np.float32)
-    kn = rng.standard_normal((w.decode_batch, w.Hkv, w.d), dtype=np.float32)
-    vn = rng.standard_normal((w.decode_batch, w.Hkv, w.d), dtype=np.float32)
-    return (_round(Kp, w.dtype), _round(Vp, w.dtype), _round(Qn, w.dtype),
-            _round(kn, w.dtype), _round(vn, w.dtype))
+    return _round(Kp, w.dtype), _round(Vp, w.dtype)
 
 
 def decode_offset(seq: int, rows: int, stride: int = 7919) -> int:
     """Row of the pool where sequence ``seq``'s cache starts (wraps around)."""
     return (seq * stride) % rows
+
+
+def decode_cache(w: Workload, cap: int, prefix: int, device, *, seed: int | None = None):
+    """Device caches Kc, Vc [decode_batch, Hkv, cap, d] whose first ``prefix``
+    rows hold each sequence's keys/values, drawn from one seeded host pool
+    (see ``decode_pool``). Rows from ``prefix`` on are zero.
+    Returns (Kc, Vc, Kpool, Vpool) with the pools on the host."""
+    import torch
+    Kp, Vp = decode_pool(w, prefix, seed=seed)
+    B = w.decode_batch
+    dt = Kp.dtype
+    Kc = torch.zeros((B, w.Hkv, cap, w.d), dtype=dt, device=device)
+    Vc = torch.zeros((B, w.Hkv, cap, w.d), dtype=dt, device=device)
+    Kd, Vd = Kp.to(device), Vp.to(device)
+    for s in range(B):
+        off = decode_offset(s, prefix)
+        for src, dst in ((Kd, Kc), (Vd, Vc)):
+            dst[s, :, : prefix - off].copy_(src[:, off:])
+            if off:
+                dst[s, :, prefix - off: prefix].copy_(src[:, :off])
+    return Kc, Vc, Kp, Vp
+
+
+def decode_rows(pool, seq: int, prefix: int):
+    """Host copy of sequence ``seq``'s first ``prefix`` cached rows [Hkv, prefix, d]."""
+    import torch
+    off = decode_offset(seq, prefix)
+    return torch.cat([pool[:, off:prefix], pool[:, :off]], dim=1)
+
+
+def decode_step_inputs(w: Workload, step: int, *, B: int | None = None, seed: int | None = None):
+    """q_new [B, Hq, d], k_new and v_new [B, Hkv, d] for decode step ``step``."""
+    B = w.decode_batch if B is None else B
+    rng = np.random.default_rng([(w.seed if seed is None else seed), 2000 + step])
+    q = rng.standard_normal((B, w.Hq, w.d), dtype=np.float32)
+    k = rng.standard_normal((B, w.Hkv, w.d), dtype=np.float32)
+    v = rng.standard_normal((B, w.Hkv, w.d), dtype=np.float32)
+    return _round(q, w.dtype), _round(k, w.dtype), _round(v, w.dtype)

@@ -1,0 +1,104 @@
+"""Host-side checks of the C ABI: the library loads without a GPU, exports every
+function include/pisa.h declares, computes the pyramid geometry the oracle
+computes, and rejects bad arguments before anything reaches a device."""
+import ctypes
+
+import pytest
+import torch
+
+from hierarchical_block_sparse_b200 import build as pisa_build
+from hierarchical_block_sparse_b200 import pisa
+from oracle import oracle
+
+
+@pytest.fixture(scope="module")
+def lib():
+    pisa_build.build()
+    return pisa.load()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = pisa.exported_names()
+    assert len(names) >= 14
+    for n in names:
+        assert hasattr(lib, n), n
+    for required in ("pisa_build_pyramid", "pisa_select", "pisa_sparse_attn", "pisa_forward"):
+        assert required in names
+
+
+def test_version_and_status_strings(lib):
+    assert "sm_100a" in pisa.pisa_version()
+    for s in (0, -1, -2, -3, -4):
+        assert pisa.pisa_status_string(s)
+    assert pisa.pisa_status_string(-99) == "unknown status"
+
+
+@pytest.mark.parametrize("N,C", [(1024, 16), (1000, 16), (16384, 64), (262144, 64), (262145, 64), (1, 64), (64, 64)])
+def test_geometry_matches_oracle(lib, N, C):
+    cfg = pisa.make_cfg(B=1, Hq=1, Hkv=1, N=N, d=128, C=C, K=16)
+    L, M, off = oracle.geometry(N, C, 2)
+    assert pisa.pisa_num_levels(cfg) == L
+    for lvl in range(1, L + 1):
+        assert pisa.pisa_level_nodes(cfg, lvl) == M[lvl]
+        assert pisa.pisa_level_offset(cfg, lvl) == off[lvl]
+    assert pisa.pisa_pyramid_rows(cfg) == oracle.total_nodes(N, C, 2)
+
+
+def test_geometry_general_branching(lib):
+    cfg = pisa.make_cfg(B=1, Hq=1, Hkv=1, N=5000, d=64, C=10, K=4, g=3)
+    L, M, off = oracle.geometry(5000, 10, 3)
+    assert pisa.pisa_num_levels(cfg) == L
+    assert pisa.pisa_pyramid_rows(cfg) == oracle.total_nodes(5000, 10, 3)
+
+
+def _call_select(lib, cfg, ptrs=(16, 16, 16, 16)):
+    P = [ctypes.c_void_p(p) if p else None for p in ptrs]
+    return lib.pisa_select(ctypes.byref(cfg), *P, None)
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("B", 0, -1), ("Hq", 3, -1), ("N", -5, -1), ("C", 0, -1), ("K", 0, -1),
+    ("causal", 2, -1), ("forced_mask", 9, -1), ("dtype", 7, -1),
+    ("K", 2, -1),            # three forced leaves need K >= 3
+    ("g", 3, -2), ("d", 96, -2), ("K", 17, -2), ("C", 2048, -2),
+])
+def test_invalid_configs_are_rejected_before_launch(lib, field, value, status):
+    cfg = pisa.make_cfg(B=1, Hq=4, Hkv=2, N=256, d=128, C=16, K=4)
+    setattr(cfg, field, value)
+    assert _call_select(lib, cfg) == status
+
+
+def test_group_size_limits(lib):
+    cfg = pisa.make_cfg(B=1, Hq=6, Hkv=2, N=256, d=128, C=16, K=4)   # G = 3
+    assert _call_select(lib, cfg) == -2
+    cfg = pisa.make_cfg(B=1, Hq=64, Hkv=2, N=256, d=128, C=16, K=4)  # G = 32
+    assert _call_select(lib, cfg) == -2
+
+
+def test_null_and_misaligned_pointers(lib):
+    cfg = pisa.make_cfg(B=1, Hq=1, Hkv=1, N=256, d=128, C=16, K=4)
+    assert _call_select(lib, cfg, (16, 0, 16, 16)) == -1
+    assert _call_select(lib, cfg, (16, 18, 16, 16)) == -4
+    assert lib.pisa_build_pyramid(ctypes.byref(cfg), None, None, None) == -1
+    assert lib.pisa_forward(None, None, None, None, None, None, None, None) == -1
+
+
+def test_empty_sequence_is_a_noop(lib):
+    cfg = pisa.make_cfg(B=1, Hq=1, Hkv=1, N=0, d=128, C=16, K=4)
+    assert pisa.pisa_num_levels(cfg) == 0
+    assert pisa.pisa_pyramid_rows(cfg) == 0
+    assert lib.pisa_forward(ctypes.byref(cfg), None, None, None, None, None, None, None) == 0
+
+
+def test_decode_requires_causal(lib):
+    cfg = pisa.make_cfg(B=1, Hq=1, Hkv=1, N=256, d=128, C=16, K=4, causal=False, forced_mask=4)
+    P = [ctypes.c_void_p(16)] * 7
+    assert lib.pisa_decode(ctypes.byref(cfg), *P, None) == -1
+
+
+def test_binding_refuses_cpu_tensors(lib):
+    cfg = pisa.make_cfg(B=1, Hq=1, Hkv=1, N=64, d=64, C=16, K=4, dtype=torch.float32)
+    K = torch.zeros(1, 1, 64, 64)
+    pyr = torch.zeros(1, 1, pisa.pisa_pyramid_rows(cfg), 64)
+    with pytest.raises(ValueError):
+        pisa.pisa_build_pyramid(cfg, K, pyr)

@@ -1,0 +1,144 @@
+"""GPU parity of the decode path (incremental pyramid append + the fused
+single-stage step) against the oracle: the oracle rebuilds each sequence's
+pyramid for the grown prefix and selects/attends for the newest query."""
+import numpy as np
+import pytest
+import torch
+
+from hierarchical_block_sparse_b200 import pisa
+from hierarchical_block_sparse_b200.workloads import (WORKLOADS, Workload, decode_cache, decode_rows,
+                                                      decode_step_inputs)
+from oracle import oracle
+from tests import parity
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.fail("a CUDA device is required for the gpu-marked tests")
+    pisa.load()
+
+
+def _cfg(w, B, cap):
+    return pisa.make_cfg(B=B, Hq=w.Hq, Hkv=w.Hkv, N=cap, d=w.d, C=w.C, K=w.K, causal=True,
+                         forced_mask=w.forced_mask, dtype=torch.bfloat16 if w.dtype == "bf16" else torch.float32)
+
+
+def _check_seq(w, cap, Khost, Vhost, pyr_gpu, n, q, idx_g, o_g, check_pyr=True):
+    """One sequence after its token at position n was appended."""
+    G = w.Hq // w.Hkv
+    worst, exempt = 0.0, 0
+    for h in range(w.Hkv):
+        Kh = oracle.to_f64(Khost[h, : n + 1])
+        Vh = oracle.to_f64(Vhost[h, : n + 1])
+        P = oracle.build_pyramid(Kh, w.C, N=n + 1, N_layout=cap)
+        if check_pyr:
+            L, M, off = oracle.geometry(cap, w.C)
+            gp = oracle.to_f64(pyr_gpu[h])
+            for lvl in range(1, L + 1):
+                live = -(-(n + 1) // (w.C * 2 ** (lvl - 1)))
+                np.testing.assert_allclose(gp[off[lvl]:off[lvl] + live], P[off[lvl]:off[lvl] + live],
+                                           rtol=1e-5, atol=2e-6)
+        qg = oracle.to_f64(q[h * G:(h + 1) * G])[None]
+        want, gap = oracle.select_rows(qg, np.array([n]), Kh, P, C=w.C, K=w.K, N=n + 1, N_layout=cap,
+                                       forced_mask=w.forced_mask)
+        got = idx_g[h].cpu().numpy()
+        parity.check_row_valid(got, n, n + 1, w.C, w.K, True, w.forced_mask)
+        if gap[0] >= parity.TIE_BAND:
+            np.testing.assert_array_equal(got, want[0])
+        else:
+            exempt += 1
+        for j in range(G):
+            O_o = oracle.attn_rows(qg[:, j], np.array([n]), Kh, Vh, got[None], C=w.C, causal=True)
+            worst = max(worst, float(np.abs(O_o[0] - oracle.to_f64(o_g[h * G + j])).max()))
+    assert worst <= parity.O_TOL[w.dtype], worst
+    return exempt
+
+
+@pytest.mark.parametrize("G", [1, 2])
+def test_decode_steps_small(G):
+    w = Workload("dec_small", 120, B=1, Hq=2 * G, Hkv=2, N=0, d=128, C=64, K=8, decode_batch=3)
+    cap = 4096
+    dev = torch.device("cuda", 0)
+    prefix = [1000, 2048, 3071]
+    Kc, Vc, Kp, Vp = decode_cache(w, cap, 3100, dev)
+    Khost = [decode_rows(Kp, s, 3100) for s in range(3)]
+    Vhost = [decode_rows(Vp, s, 3100) for s in range(3)]
+    for s in range(3):  # zero the rows past each sequence's prefix
+        Kc[s, :, prefix[s]:] = 0
+        Vc[s, :, prefix[s]:] = 0
+        Khost[s] = torch.cat([Khost[s][:, : prefix[s]], torch.zeros_like(Khost[s][:, :1]).expand(-1, cap - prefix[s], -1)], 1)
+        Vhost[s] = torch.cat([Vhost[s][:, : prefix[s]], torch.zeros_like(Vhost[s][:, :1]).expand(-1, cap - prefix[s], -1)], 1)
+    cfg = _cfg(w, 3, cap)
+    R = pisa.pisa_pyramid_rows(cfg)
+    pyr = torch.zeros((3, w.Hkv, R, w.d), dtype=torch.float32, device=dev)
+    lens = torch.tensor(prefix, dtype=torch.int32, device=dev)
+    pisa.pisa_build_pyramid_prefix(cfg, Kc, lens, pyr)
+    pos = lens.clone()
+    exempt = 0
+    for step in range(6):
+        q, k, v = decode_step_inputs(w, step, B=3)
+        idx = torch.full((3, w.Hkv, w.K), -7, dtype=torch.int32, device=dev)
+        o = torch.empty((3, w.Hq, w.d), dtype=q.dtype, device=dev)
+        pisa.pisa_pyramid_append(cfg, Kc, Vc, pyr, k.to(dev), v.to(dev), pos)
+        pisa.pisa_decode(cfg, q.to(dev), Kc, Vc, pyr, pos, idx, o)
+        torch.cuda.synchronize()
+        for s in range(3):
+            n = int(pos[s])
+            Khost[s][:, n] = k[s]
+            Vhost[s][:, n] = v[s]
+            exempt += _check_seq(w, cap, Khost[s], Vhost[s], pyr[s], n, q[s], idx[s], o[s])
+        # the caches now hold the new rows verbatim
+        for s in range(3):
+            n = int(pos[s])
+            assert torch.equal(Kc[s, :, n].cpu(), k[s]) and torch.equal(Vc[s, :, n].cpu(), v[s])
+        pos += 1
+    assert exempt <= 2
+
+
+def test_decode_out_of_range_positions():
+    w = Workload("dec_bad", 121, B=1, Hq=2, Hkv=2, N=0, d=64, C=16, K=4, decode_batch=2, dtype="f32")
+    cap = 256
+    dev = torch.device("cuda", 0)
+    cfg = _cfg(w, 2, cap)
+    Kc = torch.randn(2, 2, cap, 64, device=dev)
+    Vc = torch.randn(2, 2, cap, 64, device=dev)
+    K0, V0 = Kc.clone(), Vc.clone()
+    pyr = torch.zeros(2, 2, pisa.pisa_pyramid_rows(cfg), 64, device=dev)
+    pos = torch.tensor([-1, cap], dtype=torch.int32, device=dev)
+    q, k, v = decode_step_inputs(w, 0, B=2)
+    idx = torch.full((2, 2, 4), 5, dtype=torch.int32, device=dev)
+    o = torch.ones(2, 2, 64, device=dev)
+    pisa.pisa_pyramid_append(cfg, Kc, Vc, pyr, k.to(dev), v.to(dev), pos)
+    pisa.pisa_decode(cfg, q.to(dev), Kc, Vc, pyr, pos, idx, o)
+    torch.cuda.synchronize()
+    assert torch.equal(Kc, K0) and torch.equal(Vc, V0)
+    assert bool((idx == -1).all()) and bool((o == 0).all()) and bool((pyr == 0).all())
+
+
+def test_decode_full_size_sampled():
+    # 64 sequences x 8 heads against 262144-key caches (bench launch shape)
+    w = WORKLOADS["mha8_n256k"]
+    prefix = w.N
+    cap = prefix + 64
+    dev = torch.device("cuda", 0)
+    Kc, Vc, Kp, Vp = decode_cache(w, cap, prefix, dev)
+    B = w.decode_batch
+    cfg = _cfg(w, B, cap)
+    pyr = torch.empty((B, w.Hkv, pisa.pisa_pyramid_rows(cfg), w.d), dtype=torch.float32, device=dev)
+    lens = torch.full((B,), prefix, dtype=torch.int32, device=dev)
+    pisa.pisa_build_pyramid_prefix(cfg, Kc, lens, pyr)
+    q, k, v = decode_step_inputs(w, 0)
+    idx = torch.full((B, w.Hkv, w.K), -7, dtype=torch.int32, device=dev)
+    o = torch.empty((B, w.Hq, w.d), dtype=q.dtype, device=dev)
+    pos = lens.clone()
+    pisa.pisa_pyramid_append(cfg, Kc, Vc, pyr, k.to(dev), v.to(dev), pos)
+    pisa.pisa_decode(cfg, q.to(dev), Kc, Vc, pyr, pos, idx, o)
+    torch.cuda.synchronize()
+    assert int((idx == -7).sum()) == 0
+    for s in (0, 17, 63):
+        Kh = torch.cat([decode_rows(Kp, s, prefix), k[s][:, None]], 1)
+        Vh = torch.cat([decode_rows(Vp, s, prefix), v[s][:, None]], 1)
+        _check_seq(w, cap, Kh, Vh, pyr[s], prefix, q[s], idx[s], o[s], check_pyr=(s == 0))
