@@ -119,6 +119,8 @@ def algorithmic(w, N: int):
     pyr_b = w.B * w.Hkv * rows * d * 4
     idx_b = w.B * w.Hkv * N * w.K * 4
     return {
+        "internal_flops": float(units * G * internal.sum() * 2 * d),
+        "leaf_flops": float(units * G * leafkeys.sum() * 2 * d),
         "select_flops": float(units * G * (internal.sum() + leafkeys.sum()) * 2 * d),
         "attn_flops": float(units * G * attended.sum() * 4 * d),
         "select_dots_per_query": float((internal.sum() + leafkeys.sum()) / N),
@@ -139,6 +141,10 @@ def source_sha(files):
 
 
 KERNEL_SOURCES = {
+    "stage1": ["hierarchical_block_sparse_b200/csrc/blockmajor.cu", "hierarchical_block_sparse_b200/csrc/pisa_walk.cuh",
+               "hierarchical_block_sparse_b200/csrc/pisa_device.cuh"],
+    "leaf_scores": ["hierarchical_block_sparse_b200/csrc/blockmajor.cu", "hierarchical_block_sparse_b200/csrc/tc.cuh"],
+    "attn_tiles": ["hierarchical_block_sparse_b200/csrc/blockmajor.cu", "hierarchical_block_sparse_b200/csrc/tc.cuh"],
     "pool": ["hierarchical_block_sparse_b200/csrc/pool.cu", "hierarchical_block_sparse_b200/csrc/pisa_device.cuh"],
     "select": ["hierarchical_block_sparse_b200/csrc/select.cu", "hierarchical_block_sparse_b200/csrc/pisa_walk.cuh",
                "hierarchical_block_sparse_b200/csrc/pisa_device.cuh"],
@@ -274,6 +280,7 @@ def main():
     ap.add_argument("--workload", default="mha8_n256k")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-bsa", action="store_true")
+    ap.add_argument("--no-per-query", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     args = ap.parse_args()
@@ -317,40 +324,43 @@ def main():
     Qd, Kd, Vd = Q.to(dev), K.to(dev), V.to(dev)
     cfg = pisa.cfg_for(Qd, Kd, C=w.C, K_=w.K, causal=w.causal, forced_mask=w.forced_mask)
     pyr, idx, O = pisa.alloc_outputs(cfg, dev, Qd.dtype)
+    work = pisa.alloc_workspace(cfg, dev)
     stream = torch.cuda.current_stream()
-    launches_per_step = 3 + (1 if pisa.pisa_num_levels(cfg) >= 6 else 0)
+    nph = len(pisa.PHASES)
+    pool_launches = 2 if pisa.pisa_num_levels(cfg) >= 6 else 1
+    # our kernels per step: pyramid, stage 1, 3 grouping kernels, leaf scores,
+    # Top-K, 3 grouping kernels, attention tiles, output conversion
+    launches_per_step = pool_launches + 1 + 3 + 1 + 1 + 3 + 1 + 1
 
     def step(ev=None):
-        if ev is not None:
-            ev[0].record(stream)
-        pisa.pisa_build_pyramid(cfg, Kd, pyr)
-        if ev is not None:
-            ev[1].record(stream)
-        pisa.pisa_select(cfg, Qd, Kd, pyr, idx)
-        if ev is not None:
-            ev[2].record(stream)
-        pisa.pisa_sparse_attn(cfg, Qd, Kd, Vd, idx, O)
-        if ev is not None:
-            ev[3].record(stream)
+        if ev is None:
+            pisa.pisa_forward_ws(cfg, Qd, Kd, Vd, pyr, idx, O, work)
+        else:
+            pisa.pisa_forward_ws_events(cfg, Qd, Kd, Vd, pyr, idx, O, work, ev)
 
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
+    if pisa.pisa_workspace_status(cfg, work) != 0:
+        raise RuntimeError("a tensor-core tile timed out during warm-up")
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nph + 1)] for _ in range(args.steps)]
+    for e in evs:  # create the underlying events before the timed region
+        for x in e:
+            x.record(stream)
+    torch.cuda.synchronize()
     with ClockSampler(dev.index) as clk:
-        for s in range(args.steps):
-            step(evs[s])
+        for s_ in range(args.steps):
+            step(evs[s_])
         torch.cuda.synchronize()
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
-    total_ms = evs[0][0].elapsed_time(evs[-1][3])
-    pool_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
-    sel_ms = float(np.mean([e[1].elapsed_time(e[2]) for e in evs]))
-    attn_ms = float(np.mean([e[2].elapsed_time(e[3]) for e in evs]))
+    total_ms = evs[0][0].elapsed_time(evs[-1][nph])
+    phase_ms = {name: float(np.mean([e[i].elapsed_time(e[i + 1]) for e in evs]))
+                for i, name in enumerate(pisa.PHASES)}
     if dist:
         tt = torch.tensor([total_ms], device=dev)
         dist.all_reduce(tt, op=dist.ReduceOp.MAX)
@@ -363,43 +373,62 @@ def main():
     pk = peaks()
     clocks = clk.summary()
     fma_peak = fp32_fma_peak_tflops(pk["sm_max_mhz"])
-    times = {"pool": pool_ms, "select": sel_ms, "attn": attn_ms}
-    dom = max(times, key=times.get)
-    if dom == "pool":
-        achieved = alg["pool_bytes"] / (pool_ms / 1e3) / 1e9
-        roof = {"kernel": "pool_leaves_kernel+pool_top_kernel", "bound": "hbm", "achieved": achieved,
-                "peak": pk["hbm_gbs"], "unit": "GB/s"}
-    else:
-        flops = alg["select_flops"] if dom == "select" else alg["attn_flops"]
-        achieved = flops / (times[dom] / 1e3) / 1e12
-        roof = {"kernel": "select_kernel" if dom == "select" else "attn_kernel", "bound": "alu",
-                "achieved": achieved, "peak": fma_peak, "unit": "TFLOP/s",
+    tc_peak = pk["bf16_tflops_sustained"] or pk["bf16_tflops"]
+    dom = max(phase_ms, key=phase_ms.get)
+    t_dom = phase_ms[dom] / 1e3
+    if dom == "attn_tiles":
+        roof = {"kernel": "attn_tile_kernel", "bound": "tensor", "achieved": alg["attn_flops"] / t_dom / 1e12,
+                "peak": tc_peak, "unit": "TFLOP/s", "algorithmic_per_launch": alg["attn_flops"],
+                "peak_note": "bf16 dense, sustained (MEASURED_PEAKS.json)"}
+    elif dom == "leaf_scores":
+        roof = {"kernel": "leaf_score_kernel", "bound": "tensor", "achieved": alg["leaf_flops"] / t_dom / 1e12,
+                "peak": tc_peak, "unit": "TFLOP/s", "algorithmic_per_launch": alg["leaf_flops"],
+                "peak_note": "bf16 dense, sustained (MEASURED_PEAKS.json)"}
+    elif dom == "stage1":
+        roof = {"kernel": "stage1_kernel", "bound": "alu", "achieved": alg["internal_flops"] / t_dom / 1e12,
+                "peak": fma_peak, "unit": "TFLOP/s", "algorithmic_per_launch": alg["internal_flops"],
                 "peak_note": "fp32 FMA: 148 SMs x 128 lanes x 2 FLOP x max SM clock"}
+    else:
+        b = alg["pool_bytes"] if dom == "pyramid" else alg["selection_bytes"]
+        roof = {"kernel": dom, "bound": "hbm", "achieved": b / t_dom / 1e9, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "algorithmic_per_launch": b}
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["traffic"] = measured_traffic(dom, w.name)
-    roof["algorithmic_per_launch"] = alg["pool_bytes"] if dom == "pool" else (
-        alg["select_flops"] if dom == "select" else alg["attn_flops"])
-    roof["launch_ms"] = times[dom]
+    roof["launch_ms"] = phase_ms[dom]
 
-    sel_total = pool_ms + sel_ms
+    sel_total = sum(phase_ms[k] for k in ("pyramid", "stage1", "group_candidates", "leaf_scores", "topk"))
     hbm = pk["hbm_gbs"] * 1e9
     out = {
         "metric": metric, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic (seeded i.i.d. N(0,1))",
         "config": config,
-        "selection_ms": sel_total, "pool_ms": pool_ms, "select_ms": sel_ms, "attn_ms": attn_ms,
+        "path": "block-major tensor-core (pisa_forward_ws)",
+        "selection_ms": sel_total, "attention_ms": ms_per_step - sel_total, "phase_ms": phase_ms,
         "hbm_roofline_frac": {"prefill": alg["prefill_bytes"] / (ms_per_step / 1e3) / hbm,
                               "selection": alg["selection_bytes"] / (sel_total / 1e3) / hbm,
-                              "pool": alg["pool_bytes"] / (pool_ms / 1e3) / hbm},
+                              "pyramid": alg["pool_bytes"] / (phase_ms["pyramid"] / 1e3) / hbm},
         "work": {"select_dots_per_query": alg["select_dots_per_query"],
                  "attended_keys_per_query": alg["attended_keys_per_query"],
-                 "select_tflop": alg["select_flops"] / 1e12, "attn_tflop": alg["attn_flops"] / 1e12},
+                 "internal_tflop": alg["internal_flops"] / 1e12, "leaf_tflop": alg["leaf_flops"] / 1e12,
+                 "attn_tflop": alg["attn_flops"] / 1e12},
         "roofline": roof,
         "peaks_source": pk["source"],
         "clocks": clocks,
         "gpu_launches": launches_per_step * args.steps,
     }
+    if pisa.pisa_workspace_status(cfg, work) != 0:
+        raise RuntimeError("a tensor-core tile timed out in the timed region")
+
+    # the per-query CUDA-core path (pisa_forward), for comparison
+    if not args.no_per_query:
+        pisa.pisa_forward(cfg, Qd, Kd, Vd, pyr, idx, O)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        pisa.pisa_forward(cfg, Qd, Kd, Vd, pyr, idx, O)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        out["per_query_path_ms_per_step"] = e0.elapsed_time(e1)
 
     # ---- end to end through the public API: pinned host -> device -> host ----
     Qh, Kh, Vh = Q.pin_memory(), K.pin_memory(), V.pin_memory()
@@ -410,7 +439,7 @@ def main():
         Qd.copy_(Qh, non_blocking=True)
         Kd.copy_(Kh, non_blocking=True)
         Vd.copy_(Vh, non_blocking=True)
-        pisa.pisa_forward(cfg, Qd, Kd, Vd, pyr, idx, O)
+        pisa.pisa_forward_ws(cfg, Qd, Kd, Vd, pyr, idx, O, work)
         Oh.copy_(O, non_blocking=True)
         Ih.copy_(idx, non_blocking=True)
 
@@ -447,6 +476,7 @@ def main():
         b1.record(stream)
         torch.cuda.synchronize()
         out["bsa_selection_ms"] = b0.elapsed_time(b1)
+        out["bsa_kernel"] = "per-query CUDA-core flat scan (bsa_kernel)"
         out["pisa_vs_bsa_selection_speedup"] = out["bsa_selection_ms"] / sel_total
         del bidx
 
@@ -454,7 +484,7 @@ def main():
     if not args.no_decode and w.decode_batch:
         out["decode"] = bench_decode(w, dev, stream)
 
-    del Qd, Kd, Vd, pyr, idx, O
+    del Qd, Kd, Vd, pyr, idx, O, work
     torch.cuda.empty_cache()
 
     if dist:

@@ -10,6 +10,8 @@ from .pisa import (  # noqa: F401
     pisa_num_levels, pisa_level_nodes, pisa_level_offset, pisa_pyramid_rows,
     pisa_build_pyramid, pisa_select, pisa_sparse_attn, pisa_forward, pisa_bsa_select,
     pisa_build_pyramid_prefix, pisa_pyramid_append, pisa_decode, pisa_status_string, pisa_version,
+    pisa_workspace_bytes, pisa_select_ws, pisa_sparse_attn_ws, pisa_forward_ws, alloc_workspace,
+    pisa_workspace_status,
 )
 
 __version__ = "0.1.0"

@@ -78,6 +78,30 @@ PoolParams pool_params(const pisa_cfg* c, const Geom& g, const int32_t* len) {
     return p;
 }
 
+// limits of the block-major tensor-core path
+int check_bm(const pisa_cfg* c) {
+    int s = check_gpu(c);
+    if (s) return s;
+    if (c->dtype != PISA_DTYPE_BF16 || c->d != 128 || c->C != 64) return PISA_E_UNSUPPORTED;
+    if (c->N >= (1 << 27)) return PISA_E_UNSUPPORTED;
+    if ((int64_t)c->B * c->Hkv * c->N * 32 >= ((int64_t)1 << 31)) return PISA_E_UNSUPPORTED;
+    return PISA_OK;
+}
+
+BmShape bm_shape(const pisa_cfg* c) {
+    BmShape s;
+    s.B = c->B; s.Hq = c->Hq; s.Hkv = c->Hkv; s.N = c->N; s.G = c->Hq / c->Hkv;
+    s.M1 = ((int64_t)c->N + c->C - 1) / c->C;
+    return s;
+}
+
+int check_ws(const pisa_cfg* c, const void* ws, size_t bytes) {
+    if (!ws) return PISA_E_INVALID;
+    if (((uintptr_t)ws & 255u) != 0) return PISA_E_ALIGNMENT;
+    if (bytes < blockmajor_layout(bm_shape(c)).total) return PISA_E_INVALID;
+    return PISA_OK;
+}
+
 DecodeParams decode_params(const pisa_cfg* c, const Geom& g) {
     DecodeParams p;
     p.B = c->B; p.Hq = c->Hq; p.Hkv = c->Hkv; p.N = c->N; p.C = c->C; p.K = c->K;
@@ -190,6 +214,89 @@ int pisa_bsa_select(const pisa_cfg* cfg, const void* Q, const float* pyr, int32_
     return cuda_status(launch_bsa(cfg->dtype, cfg->d, Q, pyr, idx, select_params(cfg, g), (cudaStream_t)stream));
 }
 
+int64_t pisa_workspace_bytes(const pisa_cfg* cfg) {
+    int s = check_bm(cfg);
+    if (s) return s;
+    if (cfg->N == 0) return 0;
+    return (int64_t)blockmajor_layout(bm_shape(cfg)).total;
+}
+
+int pisa_workspace_status(const pisa_cfg* cfg, const void* workspace, void* stream) {
+    int s = check_bm(cfg);
+    if (s) return s;
+    if (cfg->N == 0) return PISA_OK;
+    if (!workspace) return PISA_E_INVALID;
+    const BmLayout L = blockmajor_layout(bm_shape(cfg));
+    int word = 0;
+    cudaError_t e = cudaMemcpyAsync(&word, (const uint8_t*)workspace + L.misc + 4, 4, cudaMemcpyDeviceToHost,
+                                    (cudaStream_t)stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize((cudaStream_t)stream);
+    if (e != cudaSuccess) return PISA_E_CUDA;
+    return word == 0 ? PISA_OK : PISA_E_TIMEOUT;
+}
+
+int pisa_select_ws(const pisa_cfg* cfg, const void* Q, const void* K, const float* pyr, int32_t* idx,
+                   void* workspace, size_t workspace_bytes, void* stream) {
+    int s = check_bm(cfg);
+    if (s) return s;
+    if (cfg->N == 0) return PISA_OK;
+    if (!Q || !K || !pyr || !idx) return PISA_E_INVALID;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(pyr) || !aligned16(idx)) return PISA_E_ALIGNMENT;
+    s = check_ws(cfg, workspace, workspace_bytes);
+    if (s) return s;
+    Geom g;
+    make_geom(cfg->N, cfg->C, &g);
+    return cuda_status(launch_select_bm(Q, K, pyr, idx, select_params(cfg, g), bm_shape(cfg), workspace, nullptr,
+                                        (cudaStream_t)stream));
+}
+
+int pisa_sparse_attn_ws(const pisa_cfg* cfg, const void* Q, const void* K, const void* V, const int32_t* idx,
+                        void* O, void* workspace, size_t workspace_bytes, void* stream) {
+    int s = check_bm(cfg);
+    if (s) return s;
+    if (cfg->N == 0) return PISA_OK;
+    if (!Q || !K || !V || !idx || !O) return PISA_E_INVALID;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(idx) || !aligned16(O)) return PISA_E_ALIGNMENT;
+    s = check_ws(cfg, workspace, workspace_bytes);
+    if (s) return s;
+    Geom g;
+    make_geom(cfg->N, cfg->C, &g);
+    return cuda_status(launch_attn_bm(Q, K, V, idx, O, select_params(cfg, g), bm_shape(cfg), workspace, false,
+                                      nullptr, (cudaStream_t)stream));
+}
+
+int pisa_forward_ws_events(const pisa_cfg* cfg, const void* Q, const void* K, const void* V, float* pyr,
+                           int32_t* idx, void* O, void* workspace, size_t workspace_bytes, void* const* events,
+                           int n_events, void* stream) {
+    int s = check_bm(cfg);
+    if (s) return s;
+    if (cfg->N == 0) return PISA_OK;
+    if (!Q || !K || !V || !pyr || !idx || !O) return PISA_E_INVALID;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(pyr) || !aligned16(idx) || !aligned16(O))
+        return PISA_E_ALIGNMENT;
+    if (n_events < 0 || (n_events > 0 && !events)) return PISA_E_INVALID;
+    s = check_ws(cfg, workspace, workspace_bytes);
+    if (s) return s;
+    const PhaseEvents ev{events, n_events};
+    cudaStream_t st = (cudaStream_t)stream;
+    if (n_events > 0 && events[0]) cudaEventRecord((cudaEvent_t)events[0], st);
+    s = pisa_build_pyramid(cfg, K, pyr, stream);
+    if (s) return s;
+    if (n_events > 1 && events[1]) cudaEventRecord((cudaEvent_t)events[1], st);
+    Geom g;
+    make_geom(cfg->N, cfg->C, &g);
+    const SelectParams sp = select_params(cfg, g);
+    const BmShape sh = bm_shape(cfg);
+    s = cuda_status(launch_select_bm(Q, K, pyr, idx, sp, sh, workspace, &ev, st));
+    if (s) return s;
+    return cuda_status(launch_attn_bm(Q, K, V, idx, O, sp, sh, workspace, true, &ev, st));
+}
+
+int pisa_forward_ws(const pisa_cfg* cfg, const void* Q, const void* K, const void* V, float* pyr, int32_t* idx,
+                    void* O, void* workspace, size_t workspace_bytes, void* stream) {
+    return pisa_forward_ws_events(cfg, Q, K, V, pyr, idx, O, workspace, workspace_bytes, nullptr, 0, stream);
+}
+
 int pisa_build_pyramid_prefix(const pisa_cfg* cfg, const void* Kc, const int32_t* len, float* pyr, void* stream) {
     int s = check_gpu(cfg);
     if (s) return s;
@@ -237,6 +344,7 @@ const char* pisa_status_string(int status) {
         case PISA_E_UNSUPPORTED: return "configuration outside the GPU kernels' limits";
         case PISA_E_CUDA: return "CUDA launch or runtime error";
         case PISA_E_ALIGNMENT: return "tensor pointer not 16-byte aligned";
+        case PISA_E_TIMEOUT: return "a tensor-core tile gave up a bounded wait";
     }
     return "unknown status";
 }

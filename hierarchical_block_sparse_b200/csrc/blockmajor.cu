@@ -1,0 +1,692 @@
+// blockmajor.cu -- the two-stage, key-block-reuse form of PISA prefill on the
+// tensor cores (close reading §05 Algorithm 1 and §5.1, Eq.(12)-(13)).
+//
+// Stage 1 (stage1_kernel): one warp per (b, kv-head, t) walks levels L..2
+//   exactly as select_kernel does and writes the eligible leaf candidates
+//   (at most 2K) of level 1 -- forced ones included -- to the workspace.
+// Grouping (bucket_*): a counting sort turns the (query, slot) pairs into one
+//   list per (b, kv-head, leaf), cut into tiles of 128/G queries.
+// Stage 2 (leaf_score_kernel): one tile per step: the queries' rows of every
+//   head of the group are gathered into shared memory (cp.async, canonical
+//   K-major layout), the leaf's 64 keys are loaded once, one tcgen05 MMA
+//   (M=128, N=64, K=128) writes the logits to TMEM and the epilogue turns each
+//   row into its exact per-head LSE (Eq.7 at the leaves; causal mask inside the
+//   current leaf).
+// Final Top-K (topk_kernel): per query, forced + best-ranked candidates by the
+//   LSE summed over the group (Eq.11), written sorted; it also records each
+//   head's softmax normaliser Z = log2 sum over the kept leaves of 2^LSE.
+// Attention (attn_tile_kernel): the kept (query, leaf) pairs are grouped the
+//   same way; per tile S = Q K^T (tcgen05, TMEM), P = 2^(S*scale - Z) in bf16
+//   (causal mask in the current leaf), O_part = P V (tcgen05, V as an MN-major
+//   operand), and O_part is added into an fp32 accumulator with vector
+//   reductions; since P is already normalised no rescaling is needed.
+// finalize_kernel converts the accumulator to the output dtype.
+#include "pisa_internal.h"
+#include "pisa_walk.cuh"
+#include "tc.cuh"
+
+namespace pisa {
+
+constexpr int kSlots = 32;   // level-1 candidates per query (2K <= 32)
+constexpr int kBlk = 64;     // leaf size handled by the tensor-core tiles
+constexpr int kD = 128;      // head dimension handled by the tensor-core tiles
+
+// ------------------------------------------------------------------ stage 1 ----
+
+template <int G>
+__global__ void __launch_bounds__(256) stage1_kernel(const __nv_bfloat16* __restrict__ Q,
+                                                     const float* __restrict__ pyr, int32_t* __restrict__ cand_out,
+                                                     SelectParams p) {
+    const int lane = threadIdx.x & 31;
+    const int64_t unit = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    const int64_t units = (int64_t)p.B * p.Hkv * p.N;
+    if (unit >= units) return;
+    const int64_t bh = unit / p.N;
+    const int64_t t = unit - bh * p.N;
+    const int64_t b = bh / p.Hkv;
+    const int kvh = (int)(bh - b * p.Hkv);
+    Walk<__nv_bfloat16, kD, G> w;
+    {
+        const __nv_bfloat16* qrow[G];
+#pragma unroll
+        for (int h = 0; h < G; ++h) qrow[h] = Q + (((b * p.Hq + (int64_t)kvh * G + h) * p.N) + t) * kD;
+        w.load_q(qrow, p.qscale, lane);
+    }
+    const float* P = pyr + bh * p.geom.rows * kD;
+    const Forced F(t, p.C, p.causal, p.forced_mask);
+    int cand = lane == 0 ? 0 : -1;
+    for (int l = p.geom.L; l >= 2; --l) {
+        const LevelState s = level_state(cand, l, p.C, p.N, t, p.causal, F);
+        float score = -INFINITY;
+        if (s.n > p.K) {
+            const unsigned fmask = __ballot_sync(kFull, s.forced);
+            if (__popc(fmask) < p.K)
+                score = w.score_internal(cand, s.vmask & ~fmask, P + p.geom.off[l - 1] * kD,
+                                         (int64_t)p.C << (l - 2), p.N, lane);
+        }
+        int id = cand;
+        const int kept = keep_topk(id, score, s, p.K, lane);
+        const int parent = __shfl_sync(kFull, id, lane >> 1);
+        cand = lane < 2 * kept ? 2 * parent + (lane & 1) : -1;
+    }
+    const LevelState s = level_state(cand, 1, p.C, p.N, t, p.causal, F);
+    cand_out[unit * kSlots + lane] = s.valid ? cand : -1;
+}
+
+// --------------------------------------------------------------- grouping ----
+
+// one thread per query unit; `src` holds `stride` leaf ids per unit (-1 = none).
+// Lanes of a warp that add to the same bucket are merged into one atomic.
+__global__ void bucket_count_kernel(const int32_t* __restrict__ src, int stride, int64_t units, int N,
+                                    int64_t M1, int32_t* __restrict__ counts) {
+    const int lane = threadIdx.x & 31;
+    const int64_t unit = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const bool active = unit < units;
+    const int64_t bh = active ? unit / N : 0;
+    for (int s = 0; s < stride; ++s) {
+        const int leaf = active ? src[unit * stride + s] : -1;
+        const long long key = leaf >= 0 ? (long long)(bh * M1 + leaf) : -1ll;
+        const unsigned peers = __match_any_sync(kFull, key);
+        if (key >= 0 && lane == __ffs(peers) - 1) atomicAdd(&counts[key], __popc(peers));
+    }
+}
+
+// single CTA: exclusive scan of all bucket counts into entry offsets, and the
+// tile list (b*Hkv + kvh, leaf, first entry, entries) of every bucket.
+__global__ void __launch_bounds__(1024) bucket_scan_kernel(const int32_t* __restrict__ counts, int64_t nbuckets,
+                                                           int64_t M1, int per_tile, int32_t* __restrict__ offsets,
+                                                           int4* __restrict__ tiles, int32_t* __restrict__ ntiles) {
+    __shared__ long long s_e[1024], s_t[1024];
+    const int tid = threadIdx.x;
+    const int64_t per = (nbuckets + 1023) / 1024;
+    const int64_t lo = tid * per, hi = min(lo + per, nbuckets);
+    long long e = 0, tt = 0;
+    for (int64_t i = lo; i < hi; ++i) {
+        e += counts[i];
+        tt += (counts[i] + per_tile - 1) / per_tile;
+    }
+    s_e[tid] = e;
+    s_t[tid] = tt;
+    __syncthreads();
+    for (int off = 1; off < 1024; off <<= 1) {  // inclusive Hillis-Steele scan
+        long long ve = tid >= off ? s_e[tid - off] : 0, vt = tid >= off ? s_t[tid - off] : 0;
+        __syncthreads();
+        s_e[tid] += ve;
+        s_t[tid] += vt;
+        __syncthreads();
+    }
+    long long be = s_e[tid] - e, bt = s_t[tid] - tt;
+    for (int64_t i = lo; i < hi; ++i) {
+        const int c = counts[i];
+        offsets[i] = (int32_t)be;
+        const int nt = (c + per_tile - 1) / per_tile;
+        for (int j = 0; j < nt; ++j)
+            tiles[bt + j] = make_int4((int)(i / M1), (int)(i % M1), (int)(be + (int64_t)j * per_tile),
+                                      min(per_tile, c - j * per_tile));
+        be += c;
+        bt += nt;
+    }
+    if (tid == 1023) *ntiles = (int32_t)s_t[1023];
+}
+
+// one thread per query unit: write (t << 5 | slot) into each bucket
+__global__ void bucket_fill_kernel(const int32_t* __restrict__ src, int stride, int64_t units, int N, int64_t M1,
+                                   const int32_t* __restrict__ offsets, int32_t* __restrict__ cursor,
+                                   uint32_t* __restrict__ entries) {
+    const int lane = threadIdx.x & 31;
+    const int64_t unit = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const bool active = unit < units;
+    const int64_t bh = active ? unit / N : 0;
+    const int64_t t = active ? unit - bh * N : 0;
+    for (int s = 0; s < stride; ++s) {
+        const int leaf = active ? src[unit * stride + s] : -1;
+        const long long key = leaf >= 0 ? (long long)(bh * M1 + leaf) : -1ll;
+        const unsigned peers = __match_any_sync(kFull, key);
+        const int leader = __ffs(peers) - 1;
+        int base = 0;
+        if (key >= 0 && lane == leader) base = atomicAdd(&cursor[key], __popc(peers));
+        base = __shfl_sync(kFull, base, leader);
+        if (key >= 0) {
+            const int rank = __popc(peers & ((1u << lane) - 1u));
+            entries[offsets[key] + base + rank] = (uint32_t)((t << 5) | s);
+        }
+    }
+}
+
+// ---------------------------------------------------------- tile plumbing ----
+
+struct TileRows {
+    int t[128];     // query position of each MMA row (-1: empty row)
+    int slot[128];  // candidate slot of that query
+};
+
+// Row r of a tile is (entry r / G, head r % G). Fills row metadata.
+template <int G>
+__device__ __forceinline__ void tile_rows(TileRows& tr, const uint32_t* entries, int start, int len, int tid) {
+    const int e = tid / G;
+    if (e < len) {
+        const uint32_t v = entries[start + e];
+        tr.t[tid] = (int)(v >> 5);
+        tr.slot[tid] = (int)(v & 31u);
+    } else {
+        tr.t[tid] = -1;
+        tr.slot[tid] = 0;
+    }
+}
+
+// gather the 128 query rows (head kvh*G + r%G, position t) into the K-major A tile
+template <int G>
+__device__ __forceinline__ void gather_q(uint32_t a_smem, const TileRows& tr, const __nv_bfloat16* Q, int64_t b,
+                                         int kvh, int Hq, int N, int tid) {
+    const int i = tid & 7, c = tid >> 3;  // row within the 8-row group, 16-byte chunk
+#pragma unroll 4
+    for (int g = 0; g < 16; ++g) {
+        const int r = g * 8 + i;
+        const int t = tr.t[r];
+        if (t >= 0) {
+            const __nv_bfloat16* src = Q + (((b * Hq + (int64_t)kvh * G + (r % G)) * N) + t) * kD + c * 8;
+            tc::cp_async16(a_smem + tc::kmajor128_off(r, c), src);
+        }
+    }
+}
+
+// the leaf's 64 key rows into a K-major B tile (rows past n_keys are zero)
+__device__ __forceinline__ void load_kblock(uint32_t b_smem, const __nv_bfloat16* Kh, int64_t row0, int64_t n_keys,
+                                            int tid) {
+    const int i = tid & 7, c = tid >> 3;
+#pragma unroll
+    for (int g = 0; g < 8; ++g) {
+        const int r = g * 8 + i;
+        const int64_t row = row0 + r;
+        const __nv_bfloat16* src = Kh + (row < n_keys ? row : row0) * kD + c * 8;
+        if (row < n_keys) tc::cp_async16(b_smem + tc::kmajor128_off(r, c), src);
+        else tc::cp_async_zero16(b_smem + tc::kmajor128_off(r, c), src);
+    }
+}
+
+// the leaf's 64 value rows into the MN-major V tile (rows past n_keys are zero)
+__device__ __forceinline__ void load_vblock(uint32_t v_smem, const __nv_bfloat16* Vh, int64_t row0, int64_t n_keys,
+                                            int tid) {
+    const int k = tid & 63, j0 = tid >> 6;  // key, first dim chunk
+#pragma unroll
+    for (int j = j0; j < 16; j += 2) {
+        const int64_t row = row0 + k;
+        const __nv_bfloat16* src = Vh + (row < n_keys ? row : row0) * kD + j * 8;
+        if (row < n_keys) tc::cp_async16(v_smem + tc::mnmajor_v_off(k, j), src);
+        else tc::cp_async_zero16(v_smem + tc::mnmajor_v_off(k, j), src);
+    }
+}
+
+__device__ __forceinline__ void issue_qk(uint32_t tmem_s, uint32_t a_smem, uint32_t b_smem) {
+    constexpr uint32_t idesc = tc::idesc_bf16(128, 64, 0);
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+        tc::mma_bf16(tmem_s, tc::smem_desc(a_smem + k * 256, 128, 2048), tc::smem_desc(b_smem + k * 256, 128, 2048),
+                     idesc, k > 0);
+}
+
+// ------------------------------------------------------- stage 2: leaf LSEs ----
+
+struct TileParams {
+    int B, Hq, Hkv, N, causal;
+    int64_t M1;
+    float qscale;  // log2(e) / sqrt(d)
+};
+
+// Per-head LSE (log2 units) of every listed (query, candidate leaf):
+// lse[(unit * 32 + slot) * G + head].
+template <int G>
+__global__ void __launch_bounds__(128) leaf_score_kernel(const __nv_bfloat16* __restrict__ Q,
+                                                         const __nv_bfloat16* __restrict__ Kmat,
+                                                         const int4* __restrict__ tiles,
+                                                         const int32_t* __restrict__ ntiles_ptr,
+                                                         const uint32_t* __restrict__ entries,
+                                                         float* __restrict__ lse, int* __restrict__ err,
+                                                         TileParams p) {
+    extern __shared__ __align__(1024) uint8_t dsm[];
+    uint8_t* sA = dsm;           // 32 KB gathered query rows
+    uint8_t* sB = dsm + 32768;   // 16 KB key block
+    __shared__ TileRows tr;
+    __shared__ __align__(8) uint64_t mbar;
+    __shared__ uint32_t tmem_base;
+    const int tid = threadIdx.x, warp = tid >> 5;
+    if (warp == 0) tc::tmem_alloc(&tmem_base, 64);
+    if (tid == 0) {
+        tc::mbar_init(&mbar, 1);
+        tc::fence_mbar_init();
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    const uint32_t tmem = tmem_base;
+    const uint32_t a_smem = tc::smem_u32(sA), b_smem = tc::smem_u32(sB);
+    const int ntiles = *ntiles_ptr;
+    uint32_t phase = 0;
+    bool ok;
+    for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+        const int4 td = tiles[tile];
+        const int64_t bh = td.x, leaf = td.y;
+        const int64_t b = bh / p.Hkv;
+        const int kvh = (int)(bh - b * p.Hkv);
+        tile_rows<G>(tr, entries, td.z, td.w, tid);
+        __syncthreads();
+        gather_q<G>(a_smem, tr, Q, b, kvh, p.Hq, p.N, tid);
+        load_kblock(b_smem, Kmat + bh * p.N * kD, leaf * kBlk, p.N, tid);
+        tc::cp_async_commit();
+        tc::cp_async_wait_all();
+        tc::fence_async_smem();
+        __syncthreads();
+        if (tid == 0) {
+            tc::tc_fence_after();
+            issue_qk(tmem, a_smem, b_smem);
+            tc::mma_commit(&mbar);
+        }
+        // a CTA-uniform verdict: every thread polls, all agree before moving on
+        ok = __syncthreads_and(tc::mbar_wait(&mbar, phase, err, 1)) != 0;
+        phase ^= 1;
+        if (!ok) break;
+        tc::tc_fence_after();
+        float v[64];
+        const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16);
+        tc::tmem_ld32(taddr, v);
+        tc::tmem_ld32(taddr + 32, v + 32);
+        tc::tmem_ld_wait();
+        const int t = tr.t[tid];
+        if (t >= 0) {
+            int nvalid = (int)min((int64_t)kBlk, (int64_t)p.N - leaf * kBlk);
+            if (p.causal && leaf == t / kBlk) nvalid = min(nvalid, t - (int)(leaf * kBlk) + 1);
+            float m = -INFINITY;
+#pragma unroll
+            for (int j = 0; j < 64; ++j)
+                if (j < nvalid) m = fmaxf(m, v[j] * p.qscale);
+            float s = 0.f;
+#pragma unroll
+            for (int j = 0; j < 64; ++j)
+                if (j < nvalid) s += exp2f(v[j] * p.qscale - m);
+            const int64_t unit = bh * p.N + t;
+            lse[(unit * kSlots + tr.slot[tid]) * G + (tid % G)] = m + log2f(s);
+        }
+        tc::tc_fence_before();
+        __syncthreads();
+    }
+    __syncthreads();
+    if (warp == 0) {
+        tc::tc_fence_after();
+        tc::tmem_dealloc(tmem, 64);
+    }
+}
+
+// ----------------------------------------------------------- final Top-K ----
+
+// One warp per (b, kv-head, t): lane = candidate slot. Keeps forced + best by
+// the LSE summed over the group (ties: lower leaf), writes idx sorted and the
+// per-head normaliser z2[unit * G + h] = log2 sum_{kept} 2^lse.
+template <int G>
+__global__ void __launch_bounds__(256) topk_kernel(const int32_t* __restrict__ cand, const float* __restrict__ lse,
+                                                   int32_t* __restrict__ idx, float* __restrict__ z2,
+                                                   SelectParams p) {
+    const int lane = threadIdx.x & 31;
+    const int64_t unit = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    const int64_t units = (int64_t)p.B * p.Hkv * p.N;
+    if (unit >= units) return;
+    const int64_t bh = unit / p.N;
+    const int64_t t = unit - bh * p.N;
+    const Forced F(t, p.C, p.causal, p.forced_mask);
+    const int leaf = cand[unit * kSlots + lane];
+    float l2[G];
+    float score = 0.f;
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+        l2[h] = leaf >= 0 ? lse[(unit * kSlots + lane) * G + h] : -INFINITY;
+        score += l2[h];
+    }
+    LevelState s;
+    s.valid = leaf >= 0;
+    s.forced = s.valid && F.has(leaf, 1);
+    s.vmask = __ballot_sync(kFull, s.valid);
+    s.n = __popc(s.vmask);
+    int id = leaf;
+    const int kept = keep_topk(id, s.valid ? score : -INFINITY, s, p.K, lane);
+    bool mine = false;
+    for (int j = 0; j < kept; ++j) mine |= (__shfl_sync(kFull, id, j) == leaf) && s.valid;
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+        const float x = mine ? l2[h] : -INFINITY;
+        float m = x;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, o));
+        float e = mine ? exp2f(x - m) : 0.f;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) e += __shfl_xor_sync(kFull, e, o);
+        if (lane == 0) z2[unit * G + h] = m + log2f(e);
+    }
+    int v = lane < kept ? id : 0x7fffffff;
+    warp_sort_asc(v, lane);
+    if (lane < p.K) idx[unit * p.K + lane] = v == 0x7fffffff ? -1 : v;
+}
+
+// ------------------------------------------------------ attention tiles ----
+
+// For every listed (query, kept leaf): O_acc[row] += sum_j 2^(s_j*scale - z) v_j
+template <int G>
+__global__ void __launch_bounds__(128) attn_tile_kernel(const __nv_bfloat16* __restrict__ Q,
+                                                        const __nv_bfloat16* __restrict__ Kmat,
+                                                        const __nv_bfloat16* __restrict__ Vmat,
+                                                        const int4* __restrict__ tiles,
+                                                        const int32_t* __restrict__ ntiles_ptr,
+                                                        const uint32_t* __restrict__ entries,
+                                                        const float* __restrict__ z2, float* __restrict__ oacc,
+                                                        int* __restrict__ err, TileParams p) {
+    extern __shared__ __align__(1024) uint8_t dsm[];
+    uint8_t* sA = dsm;                 // 32 KB gathered Q rows
+    uint8_t* sK = dsm + 32768;         // 16 KB key block
+    uint8_t* sV = dsm + 49152;         // 16 KB value block (MN-major)
+    uint8_t* sP = dsm + 65536;         // 16 KB probabilities (K-major)
+    __shared__ TileRows tr;
+    __shared__ __align__(8) uint64_t mbar;
+    __shared__ uint32_t tmem_base;
+    const int tid = threadIdx.x, warp = tid >> 5;
+    if (warp == 0) tc::tmem_alloc(&tmem_base, 256);
+    if (tid == 0) {
+        tc::mbar_init(&mbar, 1);
+        tc::fence_mbar_init();
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    const uint32_t tmem_s = tmem_base, tmem_o = tmem_base + 128;
+    const uint32_t a_smem = tc::smem_u32(sA), k_smem = tc::smem_u32(sK), v_smem = tc::smem_u32(sV),
+                   p_smem = tc::smem_u32(sP);
+    const int ntiles = *ntiles_ptr;
+    uint32_t phase = 0;
+    bool ok;
+    for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+        const int4 td = tiles[tile];
+        const int64_t bh = td.x, leaf = td.y;
+        const int64_t b = bh / p.Hkv;
+        const int kvh = (int)(bh - b * p.Hkv);
+        tile_rows<G>(tr, entries, td.z, td.w, tid);
+        __syncthreads();
+        gather_q<G>(a_smem, tr, Q, b, kvh, p.Hq, p.N, tid);
+        load_kblock(k_smem, Kmat + bh * p.N * kD, leaf * kBlk, p.N, tid);
+        load_vblock(v_smem, Vmat + bh * p.N * kD, leaf * kBlk, p.N, tid);
+        tc::cp_async_commit();
+        tc::cp_async_wait_all();
+        tc::fence_async_smem();
+        __syncthreads();
+        if (tid == 0) {
+            tc::tc_fence_after();
+            issue_qk(tmem_s, a_smem, k_smem);
+            tc::mma_commit(&mbar);
+        }
+        ok = __syncthreads_and(tc::mbar_wait(&mbar, phase, err, 2)) != 0;
+        phase ^= 1;
+        if (!ok) break;
+        tc::tc_fence_after();
+        // P = 2^(S*scale - z), masked, packed to bf16 in the K-major P tile
+        {
+            float v[64];
+            const uint32_t taddr = tmem_s + ((uint32_t)(warp * 32) << 16);
+            tc::tmem_ld32(taddr, v);
+            tc::tmem_ld32(taddr + 32, v + 32);
+            tc::tmem_ld_wait();
+            const int t = tr.t[tid];
+            int nvalid = 0;
+            float z = 0.f;
+            if (t >= 0) {
+                nvalid = (int)min((int64_t)kBlk, (int64_t)p.N - leaf * kBlk);
+                if (p.causal && leaf == t / kBlk) nvalid = min(nvalid, t - (int)(leaf * kBlk) + 1);
+                z = z2[(bh * p.N + t) * G + (tid % G)];
+            }
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                uint32_t w4[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int j = c * 8 + q * 2;
+                    const float p0 = j < nvalid ? exp2f(v[j] * p.qscale - z) : 0.f;
+                    const float p1 = j + 1 < nvalid ? exp2f(v[j + 1] * p.qscale - z) : 0.f;
+                    __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+                    w4[q] = *reinterpret_cast<uint32_t*>(&h2);
+                }
+                *reinterpret_cast<uint4*>(sP + tc::kmajor64_off(tid, c)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+            }
+        }
+        tc::fence_async_smem();
+        tc::tc_fence_before();
+        __syncthreads();
+        if (tid == 0) {
+            tc::tc_fence_after();
+            constexpr uint32_t idesc = tc::idesc_bf16(128, 128, 1);
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                tc::mma_bf16(tmem_o, tc::smem_desc(p_smem + k * 256, 128, 1024),
+                             tc::smem_desc(v_smem + k * 256, 128, 1024), idesc, k > 0);
+            tc::mma_commit(&mbar);
+        }
+        ok = __syncthreads_and(tc::mbar_wait(&mbar, phase, err, 3)) != 0;
+        phase ^= 1;
+        if (!ok) break;
+        tc::tc_fence_after();
+        {
+            const int t = tr.t[tid];
+            float* dst = t >= 0 ? oacc + (((b * p.Hq + (int64_t)kvh * G + (tid % G)) * p.N) + t) * kD : nullptr;
+            const uint32_t taddr = tmem_o + ((uint32_t)(warp * 32) << 16);
+#pragma unroll
+            for (int part = 0; part < 4; ++part) {
+                float v[32];
+                tc::tmem_ld32(taddr + part * 32, v);
+                tc::tmem_ld_wait();
+                if (dst) {
+#pragma unroll
+                    for (int q = 0; q < 32; q += 4) tc::red_add_v4(dst + part * 32 + q, v[q], v[q + 1], v[q + 2], v[q + 3]);
+                }
+            }
+        }
+        tc::tc_fence_before();
+        __syncthreads();
+    }
+    __syncthreads();
+    if (warp == 0) {
+        tc::tc_fence_after();
+        tc::tmem_dealloc(tmem_base, 256);
+    }
+}
+
+// z2[unit * G + h] = log2 sum over the listed leaves of 2^lse (slot = index in idx)
+template <int G>
+__global__ void z2_kernel(const int32_t* __restrict__ idx, const float* __restrict__ lse, float* __restrict__ z2,
+                          int64_t units, int K) {
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= units * G) return;
+    const int64_t unit = i / G;
+    const int h = (int)(i - unit * G);
+    float m = -INFINITY;
+    for (int k = 0; k < K; ++k)
+        if (idx[unit * K + k] >= 0) m = fmaxf(m, lse[(unit * kSlots + k) * G + h]);
+    float e = 0.f;
+    for (int k = 0; k < K; ++k)
+        if (idx[unit * K + k] >= 0) e += exp2f(lse[(unit * kSlots + k) * G + h] - m);
+    z2[i] = m + log2f(e);
+}
+
+__global__ void finalize_kernel(const float* __restrict__ oacc, __nv_bfloat16* __restrict__ O, int64_t n4) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (int64_t)gridDim.x * blockDim.x) {
+        const float4 v = reinterpret_cast<const float4*>(oacc)[i];
+        __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y), c = __floats2bfloat162_rn(v.z, v.w);
+        uint2 u;
+        u.x = *reinterpret_cast<uint32_t*>(&a);
+        u.y = *reinterpret_cast<uint32_t*>(&c);
+        reinterpret_cast<uint2*>(O)[i] = u;
+    }
+}
+
+// -------------------------------------------------------------- host side ----
+
+BmLayout blockmajor_layout(const BmShape& s) {
+    const int64_t units = (int64_t)s.B * s.Hkv * s.N;
+    const int64_t nb = (int64_t)s.B * s.Hkv * s.M1;
+    const int per_tile = 128 / s.G;
+    const int64_t max_tiles = (units * kSlots + per_tile - 1) / per_tile + nb + 1;
+    BmLayout L;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        size_t o = off;
+        off += (bytes + 255) & ~size_t(255);
+        return o;
+    };
+    L.cand = take(units * kSlots * 4);
+    L.lse = take(units * kSlots * s.G * 4);
+    L.z2 = take(units * s.G * 4);
+    L.counts = take(nb * 4);
+    L.cursor = take(nb * 4);
+    L.offsets = take(nb * 4);
+    L.entries = take(units * kSlots * 4);
+    L.tiles = take(max_tiles * 16);
+    L.misc = take(256);  // [0] tile count, [1] error word
+    L.oacc = take((int64_t)s.B * s.Hq * s.N * kD * 4);
+    L.total = off;
+    return L;
+}
+
+static int grid_for(int64_t n, int per) { return (int)((n + per - 1) / per); }
+
+static void mark(const PhaseEvents* ev, int i, cudaStream_t st) {
+    if (ev && ev->events && i < ev->n && ev->events[i]) cudaEventRecord((cudaEvent_t)ev->events[i], st);
+}
+
+// groups the entries of `src` (stride ids per unit) into tiles; returns launch error
+static cudaError_t build_tiles(const int32_t* src, int stride, const BmShape& s, uint8_t* ws, const BmLayout& L,
+                               cudaStream_t st) {
+    const int64_t units = (int64_t)s.B * s.Hkv * s.N;
+    const int64_t nb = (int64_t)s.B * s.Hkv * s.M1;
+    int32_t* counts = (int32_t*)(ws + L.counts);
+    int32_t* cursor = (int32_t*)(ws + L.cursor);
+    cudaError_t e = cudaMemsetAsync(counts, 0, nb * 4, st);
+    if (e != cudaSuccess) return e;
+    e = cudaMemsetAsync(cursor, 0, nb * 4, st);
+    if (e != cudaSuccess) return e;
+    bucket_count_kernel<<<grid_for(units, 256), 256, 0, st>>>(src, stride, units, s.N, s.M1, counts);
+    bucket_scan_kernel<<<1, 1024, 0, st>>>(counts, nb, s.M1, 128 / s.G, (int32_t*)(ws + L.offsets),
+                                           (int4*)(ws + L.tiles), (int32_t*)(ws + L.misc));
+    bucket_fill_kernel<<<grid_for(units, 256), 256, 0, st>>>(src, stride, units, s.N, s.M1,
+                                                             (const int32_t*)(ws + L.offsets), cursor,
+                                                             (uint32_t*)(ws + L.entries));
+    return cudaGetLastError();
+}
+
+static int sm_count() {
+    int dev = 0, n = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n;
+}
+
+constexpr size_t kScoreSmem = 32768 + 16384;
+constexpr size_t kAttnSmem = 4 * 16384 + 16384;
+
+template <int G>
+static cudaError_t leaf_scores(const void* Q, const void* K, const SelectParams& sp, const BmShape& s, uint8_t* ws,
+                               const BmLayout& L, cudaStream_t st) {
+    TileParams tp{s.B, s.Hq, s.Hkv, s.N, sp.causal, s.M1, sp.qscale};
+    auto kern = leaf_score_kernel<G>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kScoreSmem);
+    if (e != cudaSuccess) return e;
+    kern<<<sm_count() * 4, 128, kScoreSmem, st>>>((const __nv_bfloat16*)Q, (const __nv_bfloat16*)K,
+                                                  (const int4*)(ws + L.tiles), (const int32_t*)(ws + L.misc),
+                                                  (const uint32_t*)(ws + L.entries), (float*)(ws + L.lse),
+                                                  (int*)(ws + L.misc) + 1, tp);
+    return cudaGetLastError();
+}
+
+template <int G>
+static cudaError_t select_bm_t(const void* Q, const void* K, const float* pyr, int32_t* idx, const SelectParams& sp,
+                               const BmShape& s, uint8_t* ws, const PhaseEvents* ev, cudaStream_t st) {
+    const BmLayout L = blockmajor_layout(s);
+    const int64_t units = (int64_t)s.B * s.Hkv * s.N;
+    int32_t* cand = (int32_t*)(ws + L.cand);
+    stage1_kernel<G><<<grid_for(units, 8), 256, 0, st>>>((const __nv_bfloat16*)Q, pyr, cand, sp);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    mark(ev, 2, st);
+    e = cudaMemsetAsync(ws + L.misc, 0, 256, st);
+    if (e != cudaSuccess) return e;
+    e = build_tiles(cand, kSlots, s, ws, L, st);
+    if (e != cudaSuccess) return e;
+    mark(ev, 3, st);
+    e = leaf_scores<G>(Q, K, sp, s, ws, L, st);
+    if (e != cudaSuccess) return e;
+    mark(ev, 4, st);
+    topk_kernel<G><<<grid_for(units, 8), 256, 0, st>>>(cand, (const float*)(ws + L.lse), idx, (float*)(ws + L.z2), sp);
+    e = cudaGetLastError();
+    mark(ev, 5, st);
+    return e;
+}
+
+template <int G>
+static cudaError_t attn_bm_t(const void* Q, const void* K, const void* V, const int32_t* idx, void* O,
+                             const SelectParams& sp, const BmShape& s, uint8_t* ws, bool have_z2,
+                             const PhaseEvents* ev, cudaStream_t st) {
+    const BmLayout L = blockmajor_layout(s);
+    float* oacc = (float*)(ws + L.oacc);
+    const int64_t units = (int64_t)s.B * s.Hkv * s.N;
+    const int64_t nO = (int64_t)s.B * s.Hq * s.N * kD;
+    cudaError_t e = cudaMemsetAsync(oacc, 0, nO * 4, st);
+    if (e != cudaSuccess) return e;
+    if (!have_z2) {
+        e = cudaMemsetAsync(ws + L.misc, 0, 256, st);
+        if (e != cudaSuccess) return e;
+    }
+    e = build_tiles(idx, sp.K, s, ws, L, st);
+    if (e != cudaSuccess) return e;
+    mark(ev, 6, st);
+    if (!have_z2) {  // per-head LSE of every listed leaf, then the normalisers
+        e = leaf_scores<G>(Q, K, sp, s, ws, L, st);
+        if (e != cudaSuccess) return e;
+        z2_kernel<G><<<grid_for(units * G, 256), 256, 0, st>>>(idx, (const float*)(ws + L.lse),
+                                                                (float*)(ws + L.z2), units, sp.K);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    TileParams tp{s.B, s.Hq, s.Hkv, s.N, sp.causal, s.M1, sp.qscale};
+    auto kern = attn_tile_kernel<G>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kAttnSmem);
+    if (e != cudaSuccess) return e;
+    kern<<<sm_count() * 2, 128, kAttnSmem, st>>>((const __nv_bfloat16*)Q, (const __nv_bfloat16*)K,
+                                                 (const __nv_bfloat16*)V, (const int4*)(ws + L.tiles),
+                                                 (const int32_t*)(ws + L.misc), (const uint32_t*)(ws + L.entries),
+                                                 (const float*)(ws + L.z2), oacc, (int*)(ws + L.misc) + 1, tp);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    mark(ev, 7, st);
+    finalize_kernel<<<sm_count() * 8, 256, 0, st>>>(oacc, (__nv_bfloat16*)O, nO / 4);
+    e = cudaGetLastError();
+    mark(ev, 8, st);
+    return e;
+}
+
+cudaError_t launch_select_bm(const void* Q, const void* K, const float* pyr, int32_t* idx, const SelectParams& sp,
+                             const BmShape& s, void* ws, const PhaseEvents* ev, cudaStream_t st) {
+    switch (s.G) {
+        case 1: return select_bm_t<1>(Q, K, pyr, idx, sp, s, (uint8_t*)ws, ev, st);
+        case 2: return select_bm_t<2>(Q, K, pyr, idx, sp, s, (uint8_t*)ws, ev, st);
+        case 4: return select_bm_t<4>(Q, K, pyr, idx, sp, s, (uint8_t*)ws, ev, st);
+        case 8: return select_bm_t<8>(Q, K, pyr, idx, sp, s, (uint8_t*)ws, ev, st);
+        case 16: return select_bm_t<16>(Q, K, pyr, idx, sp, s, (uint8_t*)ws, ev, st);
+    }
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_attn_bm(const void* Q, const void* K, const void* V, const int32_t* idx, void* O,
+                           const SelectParams& sp, const BmShape& s, void* ws, bool have_z2, const PhaseEvents* ev,
+                           cudaStream_t st) {
+    switch (s.G) {
+        case 1: return attn_bm_t<1>(Q, K, V, idx, O, sp, s, (uint8_t*)ws, have_z2, ev, st);
+        case 2: return attn_bm_t<2>(Q, K, V, idx, O, sp, s, (uint8_t*)ws, have_z2, ev, st);
+        case 4: return attn_bm_t<4>(Q, K, V, idx, O, sp, s, (uint8_t*)ws, have_z2, ev, st);
+        case 8: return attn_bm_t<8>(Q, K, V, idx, O, sp, s, (uint8_t*)ws, have_z2, ev, st);
+        case 16: return attn_bm_t<16>(Q, K, V, idx, O, sp, s, (uint8_t*)ws, have_z2, ev, st);
+    }
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace pisa

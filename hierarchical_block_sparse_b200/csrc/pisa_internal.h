@@ -33,6 +33,25 @@ struct DecodeParams {
     Geom geom;     // layout for the capacity N
 };
 
+// block-major tensor-core path (bf16, d = 128, C = 64)
+struct BmShape {
+    int B, Hq, Hkv, N, G;
+    int64_t M1;  // leaves per sequence
+};
+struct BmLayout {  // byte offsets of the workspace regions
+    size_t cand, lse, z2, counts, cursor, offsets, entries, tiles, misc, oacc, total;
+};
+struct PhaseEvents {  // optional caller events recorded at phase boundaries
+    void* const* events;
+    int n;
+};
+BmLayout blockmajor_layout(const BmShape& s);
+cudaError_t launch_select_bm(const void* Q, const void* K, const float* pyr, int32_t* idx, const SelectParams& sp,
+                             const BmShape& s, void* ws, const PhaseEvents* ev, cudaStream_t st);
+cudaError_t launch_attn_bm(const void* Q, const void* K, const void* V, const int32_t* idx, void* O,
+                           const SelectParams& sp, const BmShape& s, void* ws, bool have_z2, const PhaseEvents* ev,
+                           cudaStream_t st);
+
 cudaError_t launch_pool(int dtype, int d, const void* K, float* pyr, const PoolParams& p, cudaStream_t st);
 cudaError_t launch_select(int dtype, int d, const void* Q, const void* K, const float* pyr, int32_t* idx,
                           const SelectParams& p, cudaStream_t st);

@@ -20,7 +20,7 @@ HEADER = os.path.join(os.path.dirname(_PKG), "include", "pisa.h")
 
 PISA_DTYPE_F32, PISA_DTYPE_BF16 = 0, 1
 STATUS = {0: "PISA_OK", -1: "PISA_E_INVALID", -2: "PISA_E_UNSUPPORTED", -3: "PISA_E_CUDA",
-          -4: "PISA_E_ALIGNMENT"}
+          -4: "PISA_E_ALIGNMENT", -5: "PISA_E_TIMEOUT"}
 
 
 class PisaError(RuntimeError):
@@ -66,6 +66,13 @@ def load(path: str | None = None):
             "pisa_sparse_attn": (ctypes.c_int, [cfgp, P, P, P, P, P, P]),
             "pisa_forward": (ctypes.c_int, [cfgp, P, P, P, P, P, P, P]),
             "pisa_bsa_select": (ctypes.c_int, [cfgp, P, P, P, P]),
+            "pisa_workspace_bytes": (ctypes.c_int64, [cfgp]),
+            "pisa_workspace_status": (ctypes.c_int, [cfgp, P, P]),
+            "pisa_select_ws": (ctypes.c_int, [cfgp, P, P, P, P, P, ctypes.c_size_t, P]),
+            "pisa_sparse_attn_ws": (ctypes.c_int, [cfgp, P, P, P, P, P, P, ctypes.c_size_t, P]),
+            "pisa_forward_ws": (ctypes.c_int, [cfgp, P, P, P, P, P, P, P, ctypes.c_size_t, P]),
+            "pisa_forward_ws_events": (ctypes.c_int, [cfgp, P, P, P, P, P, P, P, ctypes.c_size_t,
+                                                      ctypes.POINTER(ctypes.c_void_p), ctypes.c_int, P]),
             "pisa_build_pyramid_prefix": (ctypes.c_int, [cfgp, P, P, P, P]),
             "pisa_pyramid_append": (ctypes.c_int, [cfgp, P, P, P, P, P, P, P]),
             "pisa_decode": (ctypes.c_int, [cfgp, P, P, P, P, P, P, P, P]),
@@ -155,6 +162,55 @@ def pisa_forward(cfg, Q, K, V, pyr, idx, O):
 
 def pisa_bsa_select(cfg, Q, pyr, idx):
     _check("pisa_bsa_select", load().pisa_bsa_select(ctypes.byref(cfg), _ptr(Q), _ptr(pyr), _ptr(idx), _stream()))
+
+
+# ---- block-major tensor-core prefill (workspace) -----------------------------------
+
+def pisa_workspace_bytes(cfg) -> int:
+    r = int(load().pisa_workspace_bytes(ctypes.byref(cfg)))
+    if r < 0:
+        _check("pisa_workspace_bytes", r)
+    return r
+
+
+def alloc_workspace(cfg, device="cuda") -> torch.Tensor:
+    """Caller-owned workspace for the *_ws calls (torch allocates; 256-byte aligned)."""
+    return torch.empty(max(pisa_workspace_bytes(cfg), 256), dtype=torch.uint8, device=device)
+
+
+def pisa_workspace_status(cfg, ws) -> int:
+    """0, or -5 (PISA_E_TIMEOUT) when a tensor-core tile gave up a bounded wait (synchronises)."""
+    return int(load().pisa_workspace_status(ctypes.byref(cfg), _ptr(ws), _stream()))
+
+
+def pisa_select_ws(cfg, Q, K, pyr, idx, ws):
+    _check("pisa_select_ws", load().pisa_select_ws(ctypes.byref(cfg), _ptr(Q), _ptr(K), _ptr(pyr), _ptr(idx),
+                                                   _ptr(ws), ws.numel(), _stream()))
+
+
+def pisa_sparse_attn_ws(cfg, Q, K, V, idx, O, ws):
+    _check("pisa_sparse_attn_ws", load().pisa_sparse_attn_ws(ctypes.byref(cfg), _ptr(Q), _ptr(K), _ptr(V),
+                                                             _ptr(idx), _ptr(O), _ptr(ws), ws.numel(), _stream()))
+
+
+def pisa_forward_ws(cfg, Q, K, V, pyr, idx, O, ws):
+    _check("pisa_forward_ws", load().pisa_forward_ws(ctypes.byref(cfg), _ptr(Q), _ptr(K), _ptr(V), _ptr(pyr),
+                                                     _ptr(idx), _ptr(O), _ptr(ws), ws.numel(), _stream()))
+
+
+PHASES = ["pyramid", "stage1", "group_candidates", "leaf_scores", "topk", "group_kept", "attn_tiles", "finalize"]
+
+
+def pisa_forward_ws_events(cfg, Q, K, V, pyr, idx, O, ws, events):
+    """pisa_forward_ws recording torch.cuda.Event objects (len(PHASES) + 1) at phase boundaries."""
+    stream = torch.cuda.current_stream()
+    for e in events:
+        if e.cuda_event == 0:  # torch creates the underlying event on first record
+            e.record(stream)
+    arr = (ctypes.c_void_p * len(events))(*[ctypes.c_void_p(e.cuda_event) for e in events])
+    _check("pisa_forward_ws_events", load().pisa_forward_ws_events(
+        ctypes.byref(cfg), _ptr(Q), _ptr(K), _ptr(V), _ptr(pyr), _ptr(idx), _ptr(O), _ptr(ws), ws.numel(),
+        arr, len(events), _stream()))
 
 
 # ---- decode -------------------------------------------------------------------------

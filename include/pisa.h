@@ -58,7 +58,8 @@ enum pisa_status {
     PISA_E_INVALID = -1,      /* null pointer, bad size, inconsistent config */
     PISA_E_UNSUPPORTED = -2,  /* valid for the method, outside the GPU limits */
     PISA_E_CUDA = -3,         /* a CUDA launch or runtime call failed */
-    PISA_E_ALIGNMENT = -4     /* a tensor pointer is not 16-byte aligned */
+    PISA_E_ALIGNMENT = -4,    /* a tensor pointer is not 16-byte aligned */
+    PISA_E_TIMEOUT = -5       /* a kernel gave up a bounded wait (see pisa_workspace_status) */
 };
 
 /* Problem statement (close reading §02-§04: N, d, C, K, g, causal). */
@@ -128,6 +129,57 @@ int pisa_forward(const pisa_cfg *cfg, const void *Q, const void *K, const void *
  * Q: [B, Hq, N, d]; idx: int32 [B, Hkv, N, K] (written). */
 int pisa_bsa_select(const pisa_cfg *cfg, const void *Q, const float *pyr, int32_t *idx,
                     void *stream);
+
+/* ---- block-major tensor-core prefill (close reading §05 Algorithm 1, §5.1) ------
+ * The pages' two-stage form: Stage 1 walks the internal levels per query;
+ * Stage 2 groups the (query, candidate leaf) pairs by leaf so that each leaf's
+ * 64 keys are loaded once per tile of up to 128 query rows and scored with one
+ * tcgen05 MMA (exact leaf LSE in the epilogue, Eq.(7)); a final Top-K per
+ * query follows. Attention runs the same way: per (leaf, tile of queries that
+ * kept it) S = Q K^T and O += softmax-weighted V on the tensor cores, using the
+ * per-query normaliser taken from the leaf LSEs. Results equal pisa_select /
+ * pisa_sparse_attn up to fp32 rounding.
+ * Limits: dtype bf16, d = 128, C = 64, K <= 16, G in {1,2,4,8,16}, N < 2^27,
+ * B * Hkv * N * 32 < 2^31. Other shapes return PISA_E_UNSUPPORTED.
+ * Workspace: caller-owned device memory of pisa_workspace_bytes(cfg) bytes,
+ * 256-byte aligned; its contents are scratch (overwritten by every call, nothing
+ * persists between calls except what pisa_forward_ws passes from its selection
+ * to its attention). Calls sharing one workspace must not overlap on the GPU. */
+
+/* Bytes of workspace the *_ws calls need for cfg (negative status on error). */
+int64_t pisa_workspace_bytes(const pisa_cfg *cfg);
+
+/* Waits for `stream`, then reads the error word the *_ws kernels leave in the
+ * workspace: PISA_OK, or PISA_E_TIMEOUT if a tensor-core tile gave up waiting
+ * for its MMA (each wait is bounded to about one second; the tile's output is
+ * then left unwritten). Synchronous; for tests and diagnostics. */
+int pisa_workspace_status(const pisa_cfg *cfg, const void *workspace, void *stream);
+
+/* Same contract and outputs as pisa_select, block-major on the tensor cores. */
+int pisa_select_ws(const pisa_cfg *cfg, const void *Q, const void *K, const float *pyr, int32_t *idx,
+                   void *workspace, size_t workspace_bytes, void *stream);
+
+/* Same contract and output as pisa_sparse_attn, block-major on the tensor cores
+ * (first scores the listed leaves for the per-query softmax normaliser). */
+int pisa_sparse_attn_ws(const pisa_cfg *cfg, const void *Q, const void *K, const void *V, const int32_t *idx,
+                        void *O, void *workspace, size_t workspace_bytes, void *stream);
+
+/* pisa_build_pyramid, pisa_select_ws, then the attention of pisa_sparse_attn_ws
+ * reusing the selection's leaf LSEs for the normaliser. */
+int pisa_forward_ws(const pisa_cfg *cfg, const void *Q, const void *K, const void *V, float *pyr, int32_t *idx,
+                    void *O, void *workspace, size_t workspace_bytes, void *stream);
+
+/* pisa_forward_ws that also records caller-created CUDA events (cudaEvent_t
+ * passed as void*, NULL entries skipped) on `stream` at its phase boundaries,
+ * for per-phase timing with cudaEventElapsedTime. Index i marks the start of
+ * phase i: 0 pyramid, 1 stage 1 (internal levels), 2 grouping of candidates,
+ * 3 leaf scoring tiles, 4 final Top-K, 5 grouping of kept leaves, 6 attention
+ * tiles, 7 output conversion; index 8 marks the end. n_events <= 9 are used.
+ * Records only: no synchronisation, no allocation. */
+#define PISA_NUM_PHASES 8
+int pisa_forward_ws_events(const pisa_cfg *cfg, const void *Q, const void *K, const void *V, float *pyr,
+                           int32_t *idx, void *O, void *workspace, size_t workspace_bytes, void *const *events,
+                           int n_events, void *stream);
 
 /* ---- decode path (close reading §5.1 last paragraph; §5.3 "decode cache") ----
  * For decode calls cfg->N is the cache CAPACITY: Kc, Vc: [B, Hkv, N, d] and the

@@ -27,15 +27,22 @@ def tdtype(w):
     return torch.bfloat16 if w.dtype == "bf16" else torch.float32
 
 
-def gpu_prefill(w, Q, K, V, bsa: bool = False):
-    """Run pisa_forward (and optionally pisa_bsa_select) on cuda:0; returns GPU tensors."""
+def gpu_prefill(w, Q, K, V, bsa: bool = False, ws: bool = False):
+    """Run pisa_forward (or, with ws=True, the block-major pisa_forward_ws) and
+    optionally pisa_bsa_select on cuda:0; returns GPU tensors."""
     dev = torch.device("cuda", 0)
     Qd, Kd, Vd = Q.to(dev), K.to(dev), V.to(dev)
     cfg = pisa.make_cfg(B=w.B, Hq=w.Hq, Hkv=w.Hkv, N=Q.shape[2], d=w.d, C=w.C, K=w.K, g=w.g, causal=w.causal,
                         forced_mask=w.forced_mask, dtype=Q.dtype)
     pyr, idx, O = pisa.alloc_outputs(cfg, dev, Q.dtype)
     idx.fill_(-7)
-    pisa.pisa_forward(cfg, Qd, Kd, Vd, pyr, idx, O)
+    if ws:
+        work = pisa.alloc_workspace(cfg, dev)
+        work.fill_(0xAB)  # scratch must not need zeroing by the caller
+        pisa.pisa_forward_ws(cfg, Qd, Kd, Vd, pyr, idx, O, work)
+        assert pisa.pisa_workspace_status(cfg, work) == 0, "a tensor-core tile timed out"
+    else:
+        pisa.pisa_forward(cfg, Qd, Kd, Vd, pyr, idx, O)
     out = {"cfg": cfg, "pyr": pyr, "idx": idx, "O": O}
     if bsa:
         bidx = torch.full_like(idx, -7)

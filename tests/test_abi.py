@@ -102,3 +102,25 @@ def test_binding_refuses_cpu_tensors(lib):
     pyr = torch.zeros(1, 1, pisa.pisa_pyramid_rows(cfg), 64)
     with pytest.raises(ValueError):
         pisa.pisa_build_pyramid(cfg, K, pyr)
+
+
+def test_workspace_bytes_and_limits(lib):
+    cfg = pisa.make_cfg(B=1, Hq=8, Hkv=8, N=262144, d=128, C=64, K=16)
+    n = pisa.pisa_workspace_bytes(cfg)
+    # candidates + LSEs + grouping lists + the fp32 output accumulator dominate
+    assert 1.0e9 < n < 3.0e9
+    for field, value in (("C", 32), ("d", 64), ("dtype", 0)):
+        bad = pisa.make_cfg(B=1, Hq=8, Hkv=8, N=262144, d=128, C=64, K=16)
+        setattr(bad, field, value)
+        assert lib.pisa_workspace_bytes(ctypes.byref(bad)) == -2
+    zero = pisa.make_cfg(B=1, Hq=1, Hkv=1, N=0, d=128, C=64, K=4)
+    assert pisa.pisa_workspace_bytes(zero) == 0
+
+
+def test_workspace_calls_validate_before_launch(lib):
+    cfg = pisa.make_cfg(B=1, Hq=2, Hkv=2, N=1000, d=128, C=64, K=8)
+    need = pisa.pisa_workspace_bytes(cfg)
+    P = [ctypes.c_void_p(4096)] * 4
+    assert lib.pisa_select_ws(ctypes.byref(cfg), *P, None, need, None) == -1           # no workspace
+    assert lib.pisa_select_ws(ctypes.byref(cfg), *P, ctypes.c_void_p(4096 + 16), need, None) == -4  # misaligned
+    assert lib.pisa_select_ws(ctypes.byref(cfg), *P, ctypes.c_void_p(8192), need - 1, None) == -1   # too small

@@ -1,0 +1,108 @@
+"""GPU parity of the block-major tensor-core path (pisa_forward_ws,
+pisa_select_ws, pisa_sparse_attn_ws) against the oracle, and its agreement
+with the per-query path."""
+import numpy as np
+import pytest
+import torch
+
+from hierarchical_block_sparse_b200 import pisa
+from hierarchical_block_sparse_b200.workloads import WORKLOADS, Workload, make_inputs
+from tests import parity
+from tests.test_gpu_parity import _report
+
+pytestmark = pytest.mark.gpu
+
+SMALL = {
+    # ragged tail (3000 = 46*64 + 56), two sequences
+    "bm_ragged": Workload("bm_ragged", 130, B=2, Hq=2, Hkv=2, N=3000, d=128, C=64, K=8),
+    # GQA group of 4, K = 16: 32 candidates per level
+    "bm_gqa4": Workload("bm_gqa4", 131, B=1, Hq=8, Hkv=2, N=5000, d=128, C=64, K=16),
+    # non-causal, only the first leaf forced
+    "bm_noncausal": Workload("bm_noncausal", 132, B=1, Hq=2, Hkv=2, N=2000, d=128, C=64, K=6, causal=False,
+                             forced_mask=1),
+    # GQA group of 16: 8 queries per tile
+    "bm_gqa16": Workload("bm_gqa16", 133, B=1, Hq=32, Hkv=2, N=1500, d=128, C=64, K=8),
+    # the smallest budget the forced leaves allow
+    "bm_k3": Workload("bm_k3", 134, B=1, Hq=1, Hkv=1, N=4096, d=128, C=64, K=3),
+    # a single leaf: the root is the leaf
+    "bm_one_leaf": Workload("bm_one_leaf", 135, B=1, Hq=2, Hkv=1, N=50, d=128, C=64, K=4),
+}
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.fail("a CUDA device is required for the gpu-marked tests")
+    pisa.load()
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_blockmajor_small_every_row(name):
+    w = SMALL[name]
+    Q, K, V, _ = make_inputs(w)
+    res = parity.gpu_prefill(w, Q, K, V, ws=True)
+    stats = [parity.check_head(w, Q, K, V, res, b, h, list(range(w.N)))
+             for b in range(w.B) for h in range(w.Hkv)]
+    _report("ws:" + name, stats)
+
+
+@pytest.mark.parametrize("name", ["mha16_n16k", "needle_mha16_n64k", "gqa32x8_n128k", "mha8_n256k"])
+def test_blockmajor_named_workload_full_size(name):
+    w = WORKLOADS[name]
+    Q, K, V, _ = make_inputs(w)
+    res = parity.gpu_prefill(w, Q, K, V, ws=True)
+    idx = res["idx"]
+    assert int((idx == -7).sum()) == 0
+    stats = [parity.check_head(w, Q, K, V, res, 0, h,
+                               parity.sample_rows(w.N, w.C, 24, seed=100 + h)) for h in range(w.Hkv)]
+    _report("ws:" + name, stats)
+    t = torch.arange(w.N, device=idx.device)
+    assert bool((idx.max(-1).values == t // w.C).all())
+    # agreement with the per-query path on every row (near-ties aside)
+    ref = parity.gpu_prefill(w, Q, K, V, ws=False)
+    same = (ref["idx"] == idx).all(-1).float().mean().item()
+    print(f"[blockmajor] {name}: rows equal to the per-query path {same:.5f}")
+    assert same > 0.98
+    dO = (ref["O"].float() - res["O"].float()).abs().max().item()
+    assert dO <= 2 * parity.O_TOL["bf16"] or same < 1.0
+
+
+@pytest.mark.parametrize("name", ["bm_ragged", "bm_gqa4", "bm_noncausal"])
+def test_select_ws_and_attn_ws_standalone(name):
+    w = SMALL[name]
+    Q, K, V, _ = make_inputs(w)
+    dev = torch.device("cuda", 0)
+    Qd, Kd, Vd = Q.to(dev), K.to(dev), V.to(dev)
+    cfg = pisa.cfg_for(Qd, Kd, C=w.C, K_=w.K, causal=w.causal, forced_mask=w.forced_mask)
+    pyr, idx, O = pisa.alloc_outputs(cfg, dev, Qd.dtype)
+    work = pisa.alloc_workspace(cfg, dev)
+    pisa.pisa_build_pyramid(cfg, Kd, pyr)
+    pisa.pisa_select_ws(cfg, Qd, Kd, pyr, idx, work)
+    # attention from indices alone (it derives its own normalisers)
+    O2 = torch.empty_like(O)
+    pisa.pisa_sparse_attn_ws(cfg, Qd, Kd, Vd, idx, O2, work)
+    assert pisa.pisa_workspace_status(cfg, work) == 0
+    res = {"cfg": cfg, "pyr": pyr, "idx": idx, "O": O2}
+    stats = [parity.check_head(w, Q, K, V, res, b, h, list(range(0, w.N, 3)))
+             for b in range(w.B) for h in range(w.Hkv)]
+    _report("ws-standalone:" + name, stats)
+    # the per-query attention on the same indices agrees
+    pisa.pisa_sparse_attn(cfg, Qd, Kd, Vd, idx, O)
+    torch.cuda.synchronize()
+    assert (O.float() - O2.float()).abs().max().item() <= 2e-2
+
+
+def test_workspace_errors():
+    w = SMALL["bm_ragged"]
+    cfg = pisa.make_cfg(B=1, Hq=2, Hkv=2, N=1000, d=128, C=64, K=8)
+    need = pisa.pisa_workspace_bytes(cfg)
+    dev = torch.device("cuda", 0)
+    Q = torch.zeros(1, 2, 1000, 128, dtype=torch.bfloat16, device=dev)
+    pyr, idx, O = pisa.alloc_outputs(cfg, dev)
+    small = torch.empty(need - 256, dtype=torch.uint8, device=dev)
+    with pytest.raises(pisa.PisaError):
+        pisa.pisa_select_ws(cfg, Q, Q, pyr, idx, small)
+    bad = pisa.make_cfg(B=1, Hq=2, Hkv=2, N=1000, d=128, C=32, K=8)
+    with pytest.raises(pisa.PisaError):
+        pisa.pisa_workspace_bytes(bad)
+    _ = w
