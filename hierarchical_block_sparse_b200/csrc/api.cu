@@ -345,6 +345,7 @@ const char* pisa_status_string(int status) {
         case PISA_E_CUDA: return "CUDA launch or runtime error";
         case PISA_E_ALIGNMENT: return "tensor pointer not 16-byte aligned";
         case PISA_E_TIMEOUT: return "a tensor-core tile gave up a bounded wait";
+        case PISA_E_SCRATCH_LIMIT: return "problem exceeds the fixed scratch of pisa_select_noalloc";
     }
     return "unknown status";
 }

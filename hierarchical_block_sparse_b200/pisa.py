@@ -20,7 +20,7 @@ HEADER = os.path.join(os.path.dirname(_PKG), "include", "pisa.h")
 
 PISA_DTYPE_F32, PISA_DTYPE_BF16 = 0, 1
 STATUS = {0: "PISA_OK", -1: "PISA_E_INVALID", -2: "PISA_E_UNSUPPORTED", -3: "PISA_E_CUDA",
-          -4: "PISA_E_ALIGNMENT", -5: "PISA_E_TIMEOUT"}
+          -4: "PISA_E_ALIGNMENT", -5: "PISA_E_TIMEOUT", -6: "PISA_E_SCRATCH_LIMIT"}
 
 
 class PisaError(RuntimeError):
@@ -73,6 +73,7 @@ def load(path: str | None = None):
             "pisa_forward_ws": (ctypes.c_int, [cfgp, P, P, P, P, P, P, P, ctypes.c_size_t, P]),
             "pisa_forward_ws_events": (ctypes.c_int, [cfgp, P, P, P, P, P, P, P, ctypes.c_size_t,
                                                       ctypes.POINTER(ctypes.c_void_p), ctypes.c_int, P]),
+            "pisa_select_noalloc": (ctypes.c_int, [cfgp, P, P, P, P, P]),
             "pisa_build_pyramid_prefix": (ctypes.c_int, [cfgp, P, P, P, P]),
             "pisa_pyramid_append": (ctypes.c_int, [cfgp, P, P, P, P, P, P, P]),
             "pisa_decode": (ctypes.c_int, [cfgp, P, P, P, P, P, P, P, P]),
@@ -196,6 +197,14 @@ def pisa_sparse_attn_ws(cfg, Q, K, V, idx, O, ws):
 def pisa_forward_ws(cfg, Q, K, V, pyr, idx, O, ws):
     _check("pisa_forward_ws", load().pisa_forward_ws(ctypes.byref(cfg), _ptr(Q), _ptr(K), _ptr(V), _ptr(pyr),
                                                      _ptr(idx), _ptr(O), _ptr(ws), ws.numel(), _stream()))
+
+
+def pisa_select_noalloc(cfg, Q, K, pyr, idx):
+    """pisa_select_ws without a workspace: for callers that cannot allocate device
+    memory, the library's fixed 32 MiB scratch array is used instead (calls on a
+    device share it, so they must not overlap on the GPU)."""
+    _check("pisa_select_noalloc", load().pisa_select_noalloc(ctypes.byref(cfg), _ptr(Q), _ptr(K), _ptr(pyr),
+                                                             _ptr(idx), _stream()))
 
 
 PHASES = ["pyramid", "stage1", "group_candidates", "leaf_scores", "topk", "group_kept", "attn_tiles", "finalize"]

@@ -59,7 +59,8 @@ enum pisa_status {
     PISA_E_UNSUPPORTED = -2,  /* valid for the method, outside the GPU limits */
     PISA_E_CUDA = -3,         /* a CUDA launch or runtime call failed */
     PISA_E_ALIGNMENT = -4,    /* a tensor pointer is not 16-byte aligned */
-    PISA_E_TIMEOUT = -5       /* a kernel gave up a bounded wait (see pisa_workspace_status) */
+    PISA_E_TIMEOUT = -5,      /* a kernel gave up a bounded wait (see pisa_workspace_status) */
+    PISA_E_SCRATCH_LIMIT = -6 /* problem too large for pisa_select_noalloc's fixed scratch */
 };
 
 /* Problem statement (close reading §02-§04: N, d, C, K, g, causal). */
@@ -180,6 +181,25 @@ int pisa_forward_ws(const pisa_cfg *cfg, const void *Q, const void *K, const voi
 int pisa_forward_ws_events(const pisa_cfg *cfg, const void *Q, const void *K, const void *V, float *pyr,
                            int32_t *idx, void *O, void *workspace, size_t workspace_bytes, void *const *events,
                            int n_events, void *stream);
+
+/* Allocation-free selection. The pages have no counterpart to this call: it
+ * exists for callers that cannot allocate device memory (a host application
+ * that owns the GPU memory pool and gives plugins no allocator, serving loops
+ * that forbid allocations after start-up, plain C callers without an
+ * allocator). Same contract and outputs as pisa_select_ws, but its scratch is
+ * a fixed array of PISA_NOALLOC_SCRATCH_BYTES compiled into the library (held
+ * on every GPU that loads the library until the process exits) instead of a
+ * caller workspace; it calls no allocating routine.
+ * - Problems whose selection scratch exceeds that size return
+ *   PISA_E_SCRATCH_LIMIT (about 80 K query units B*Hkv*N for G = 1).
+ * - The first call on a device looks up the array's device address (once per
+ *   device, that device current); make it before any stream capture.
+ * - All calls on a device share the array and it keeps the previous call's
+ *   contents; each call clears what must start at zero. Calls that overlap on
+ *   the GPU (other streams, other threads) race on the array: serialise them. */
+#define PISA_NOALLOC_SCRATCH_BYTES (32u << 20)
+int pisa_select_noalloc(const pisa_cfg *cfg, const void *Q, const void *K, const float *pyr, int32_t *idx,
+                        void *stream);
 
 /* ---- decode path (close reading §5.1 last paragraph; §5.3 "decode cache") ----
  * For decode calls cfg->N is the cache CAPACITY: Kc, Vc: [B, Hkv, N, d] and the
