@@ -85,6 +85,7 @@ int check_bm(const pisa_cfg* c) {
     if (c->dtype != PISA_DTYPE_BF16 || c->d != 128 || c->C != 64) return PISA_E_UNSUPPORTED;
     if (c->N >= (1 << 27)) return PISA_E_UNSUPPORTED;
     if ((int64_t)c->B * c->Hkv * c->N * 32 >= ((int64_t)1 << 31)) return PISA_E_UNSUPPORTED;
+    if ((int64_t)c->B * c->Hkv > 65535) return PISA_E_UNSUPPORTED;  // one grid row per (b, kv-head)
     return PISA_OK;
 }
 

@@ -4,24 +4,32 @@
 // Stage 1 (stage1_kernel): one warp per (b, kv-head, t) walks levels L..2
 //   exactly as select_kernel does and writes the eligible leaf candidates
 //   (at most 2K) of level 1 -- forced ones included -- to the workspace.
-// Grouping (bucket_*): a counting sort turns the (query, slot) pairs into one
-//   list per (b, kv-head, leaf), cut into tiles of 128/G queries.
+// Grouping (bucket_*): a counting sort turns the (query, slot) pairs of
+//   non-forced leaves into one list per (b, kv-head, leaf), cut into tiles of
+//   128/G queries.
 // Stage 2 (leaf_score_kernel): one tile per step: the queries' rows of every
 //   head of the group are gathered into shared memory (cp.async, canonical
 //   K-major layout), the leaf's 64 keys are loaded once, one tcgen05 MMA
 //   (M=128, N=64, K=128) writes the logits to TMEM and the epilogue turns each
-//   row into its exact per-head LSE (Eq.7 at the leaves; causal mask inside the
-//   current leaf).
+//   row into its exact per-head LSE (Eq.7 at the leaves).
 // Final Top-K (topk_kernel): per query, forced + best-ranked candidates by the
 //   LSE summed over the group (Eq.11), written sorted; it also records each
-//   head's softmax normaliser Z = log2 sum over the kept leaves of 2^LSE.
-// Attention (attn_tile_kernel): the kept (query, leaf) pairs are grouped the
-//   same way; per tile S = Q K^T (tcgen05, TMEM), P = 2^(S*scale - Z) in bf16
-//   (causal mask in the current leaf), O_part = P V (tcgen05, V as an MN-major
-//   operand), and O_part is added into an fp32 accumulator with vector
-//   reductions; since P is already normalised no rescaling is needed.
+//   head's partial softmax normaliser over the kept non-forced leaves.
+// Forced leaves (forced_tile_kernel): the first, previous and current leaves
+//   are shared by all queries of a leaf block, so they are scored and attended
+//   densely per tile of consecutive queries; this completes each row's
+//   normaliser Z and writes the initial fp32 output accumulator. They never go
+//   through the grouping, whose atomics would otherwise pile onto a few leaves.
+// Attention (attn_tile_kernel): the kept non-forced (query, leaf) pairs are
+//   grouped the same way; per tile S = Q K^T (tcgen05, TMEM), P = 2^(S*scale - Z)
+//   in bf16, O_part = P V (tcgen05, V as an MN-major operand), and O_part is
+//   added into the accumulator with vector reductions; P is already
+//   normalised, so no rescaling is needed.
 // finalize_kernel converts the accumulator to the output dtype.
+#include <type_traits>
+
 #include "pisa_internal.h"
+#include "pisa_stage1.cuh"
 #include "pisa_walk.cuh"
 #include "tc.cuh"
 
@@ -33,19 +41,30 @@ constexpr int kD = 128;      // head dimension handled by the tensor-core tiles
 
 // ------------------------------------------------------------------ stage 1 ----
 
-template <int G>
-__global__ void __launch_bounds__(256) stage1_kernel(const __nv_bfloat16* __restrict__ Q,
+// Walker: Walk4S<G> (4 lanes per child row, q in shared memory) for G <= 2,
+// the 32-slot reduce-scatter walker otherwise. Levels with at most K
+// candidates keep them all (gather by rank); scored levels keep the forced
+// nodes and the best by (score, lower index) through an all-pairs rank.
+#ifndef PISA_STAGE1_MINBLOCKS
+#define PISA_STAGE1_MINBLOCKS 4  // 64 registers: 32 warps per SM hide the gathers' latency
+#endif
+// Grid: x = blocks of 8 query positions, y = b * Hkv + kvh. Besides the
+// candidates, each lane adds its non-forced candidate to the leaf's bucket
+// count (the grouping of stage 2).
+template <int G, class W>
+__global__ void __launch_bounds__(256, PISA_STAGE1_MINBLOCKS) stage1_kernel(const __nv_bfloat16* __restrict__ Q,
                                                      const float* __restrict__ pyr, int32_t* __restrict__ cand_out,
-                                                     SelectParams p) {
+                                                     int32_t* __restrict__ counts, int64_t M1, SelectParams p) {
     const int lane = threadIdx.x & 31;
-    const int64_t unit = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-    const int64_t units = (int64_t)p.B * p.Hkv * p.N;
-    if (unit >= units) return;
-    const int64_t bh = unit / p.N;
-    const int64_t t = unit - bh * p.N;
+    const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (t >= p.N) return;
+    const int64_t bh = blockIdx.y;
+    const int64_t unit = bh * p.N + t;
     const int64_t b = bh / p.Hkv;
     const int kvh = (int)(bh - b * p.Hkv);
-    Walk<__nv_bfloat16, kD, G> w;
+    W w;
+    __shared__ __align__(16) float s_q[8][128 * (G <= 2 ? G : 1)];
+    if constexpr (G <= 2) w.qs = s_q[threadIdx.x >> 5];
     {
         const __nv_bfloat16* qrow[G];
 #pragma unroll
@@ -57,38 +76,53 @@ __global__ void __launch_bounds__(256) stage1_kernel(const __nv_bfloat16* __rest
     int cand = lane == 0 ? 0 : -1;
     for (int l = p.geom.L; l >= 2; --l) {
         const LevelState s = level_state(cand, l, p.C, p.N, t, p.causal, F);
-        float score = -INFINITY;
-        if (s.n > p.K) {
-            const unsigned fmask = __ballot_sync(kFull, s.forced);
-            if (__popc(fmask) < p.K)
-                score = w.score_internal(cand, s.vmask & ~fmask, P + p.geom.off[l - 1] * kD,
-                                         (int64_t)p.C << (l - 2), p.N, lane);
+        int parent;
+        if (s.n <= p.K) {
+            parent = compact_by_rank(cand, s.vmask, lane >> 1);
+            cand = lane < 2 * s.n ? 2 * parent + (lane & 1) : -1;
+            continue;
         }
+        float score = -INFINITY;
+        const unsigned fmask = __ballot_sync(kFull, s.forced);
+        if (__popc(fmask) < p.K)
+            score = w.score_internal(cand, s.vmask & ~fmask, P + p.geom.off[l - 1] * kD,
+                                     (int64_t)p.C << (l - 2), p.N, lane);
         int id = cand;
-        const int kept = keep_topk(id, score, s, p.K, lane);
-        const int parent = __shfl_sync(kFull, id, lane >> 1);
+        const int kept = keep_topk_rank(id, s.forced ? INFINITY : score, s.valid, p.K, lane);
+        parent = __shfl_sync(kFull, id, lane >> 1);
         cand = lane < 2 * kept ? 2 * parent + (lane & 1) : -1;
     }
     const LevelState s = level_state(cand, 1, p.C, p.N, t, p.causal, F);
     cand_out[unit * kSlots + lane] = s.valid ? cand : -1;
+    if (s.valid && !s.forced) atomicAdd(&counts[bh * M1 + cand], 1);
 }
 
 // --------------------------------------------------------------- grouping ----
 
-// one thread per query unit; `src` holds `stride` leaf ids per unit (-1 = none).
-// Lanes of a warp that add to the same bucket are merged into one atomic.
-__global__ void bucket_count_kernel(const int32_t* __restrict__ src, int stride, int64_t units, int N,
-                                    int64_t M1, int32_t* __restrict__ counts) {
+// Grouping of the (query, leaf) pairs that are not forced leaves of the query
+// (the forced ones are handled densely by forced_tile_kernel). One warp per
+// query position (grid x = blocks of 8 positions, y = b * Hkv + kvh); lane =
+// slot of `src` (stride <= 32 leaf ids per query, -1 = none).
+struct GroupParams {
+    int N, C, causal, forced_mask, stride;
+    int64_t M1;
+};
+
+__device__ __forceinline__ int free_leaf(const int32_t* src, const GroupParams& g, int64_t unit, int t, int lane) {
+    if (lane >= g.stride) return -1;
+    const int leaf = src[unit * g.stride + lane];
+    if (leaf < 0) return -1;
+    const Forced F(t, g.C, g.causal, g.forced_mask);
+    return F.has(leaf, 1) ? -1 : leaf;
+}
+
+__global__ void bucket_count_kernel(const int32_t* __restrict__ src, GroupParams g, int32_t* __restrict__ counts) {
     const int lane = threadIdx.x & 31;
-    const int64_t unit = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    const bool active = unit < units;
-    const int64_t bh = active ? unit / N : 0;
-    for (int s = 0; s < stride; ++s) {
-        const int leaf = active ? src[unit * stride + s] : -1;
-        const long long key = leaf >= 0 ? (long long)(bh * M1 + leaf) : -1ll;
-        const unsigned peers = __match_any_sync(kFull, key);
-        if (key >= 0 && lane == __ffs(peers) - 1) atomicAdd(&counts[key], __popc(peers));
-    }
+    const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (t >= g.N) return;
+    const int64_t bh = blockIdx.y;
+    const int leaf = free_leaf(src, g, bh * g.N + t, t, lane);
+    if (leaf >= 0) atomicAdd(&counts[bh * g.M1 + leaf], 1);
 }
 
 // single CTA: exclusive scan of all bucket counts into entry offsets, and the
@@ -129,28 +163,19 @@ __global__ void __launch_bounds__(1024) bucket_scan_kernel(const int32_t* __rest
     if (tid == 1023) *ntiles = (int32_t)s_t[1023];
 }
 
-// one thread per query unit: write (t << 5 | slot) into each bucket
-__global__ void bucket_fill_kernel(const int32_t* __restrict__ src, int stride, int64_t units, int N, int64_t M1,
+// one warp per query position: write (t << 5 | slot) into each bucket
+__global__ void bucket_fill_kernel(const int32_t* __restrict__ src, GroupParams g,
                                    const int32_t* __restrict__ offsets, int32_t* __restrict__ cursor,
                                    uint32_t* __restrict__ entries) {
     const int lane = threadIdx.x & 31;
-    const int64_t unit = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    const bool active = unit < units;
-    const int64_t bh = active ? unit / N : 0;
-    const int64_t t = active ? unit - bh * N : 0;
-    for (int s = 0; s < stride; ++s) {
-        const int leaf = active ? src[unit * stride + s] : -1;
-        const long long key = leaf >= 0 ? (long long)(bh * M1 + leaf) : -1ll;
-        const unsigned peers = __match_any_sync(kFull, key);
-        const int leader = __ffs(peers) - 1;
-        int base = 0;
-        if (key >= 0 && lane == leader) base = atomicAdd(&cursor[key], __popc(peers));
-        base = __shfl_sync(kFull, base, leader);
-        if (key >= 0) {
-            const int rank = __popc(peers & ((1u << lane) - 1u));
-            entries[offsets[key] + base + rank] = (uint32_t)((t << 5) | s);
-        }
-    }
+    const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (t >= g.N) return;
+    const int64_t bh = blockIdx.y;
+    const int leaf = free_leaf(src, g, bh * g.N + t, t, lane);
+    if (leaf < 0) return;
+    const int64_t key = bh * g.M1 + leaf;
+    const int pos = offsets[key] + atomicAdd(&cursor[key], 1);
+    entries[pos] = ((uint32_t)t << 5) | (uint32_t)lane;
 }
 
 // ---------------------------------------------------------- tile plumbing ----
@@ -225,6 +250,18 @@ __device__ __forceinline__ void issue_qk(uint32_t tmem_s, uint32_t a_smem, uint3
                      idesc, k > 0);
 }
 
+// keys of leaf `leaf` that query t may attend to (0 when none)
+__device__ __forceinline__ int visible_keys(int64_t leaf, int64_t t, int N, int causal) {
+    int64_t n = min((int64_t)kBlk, (int64_t)N - leaf * kBlk);
+    if (causal) n = min(n, t - leaf * kBlk + 1);
+    return n > 0 ? (int)n : 0;
+}
+
+__device__ __forceinline__ float logaddexp2f(float a, float b) {
+    const float m = fmaxf(a, b);
+    return m == -INFINITY ? -INFINITY : m + log2f(exp2f(a - m) + exp2f(b - m));
+}
+
 // ------------------------------------------------------- stage 2: leaf LSEs ----
 
 struct TileParams {
@@ -293,8 +330,7 @@ __global__ void __launch_bounds__(128) leaf_score_kernel(const __nv_bfloat16* __
         tc::tmem_ld_wait();
         const int t = tr.t[tid];
         if (t >= 0) {
-            int nvalid = (int)min((int64_t)kBlk, (int64_t)p.N - leaf * kBlk);
-            if (p.causal && leaf == t / kBlk) nvalid = min(nvalid, t - (int)(leaf * kBlk) + 1);
+            const int nvalid = visible_keys(leaf, t, p.N, p.causal);
             float m = -INFINITY;
 #pragma unroll
             for (int j = 0; j < 64; ++j)
@@ -320,17 +356,17 @@ __global__ void __launch_bounds__(128) leaf_score_kernel(const __nv_bfloat16* __
 
 // One warp per (b, kv-head, t): lane = candidate slot. Keeps forced + best by
 // the LSE summed over the group (ties: lower leaf), writes idx sorted and the
-// per-head normaliser z2[unit * G + h] = log2 sum_{kept} 2^lse.
+// per-head partial normaliser z2[unit * G + h] = log2 sum 2^lse over the kept
+// leaves that are not forced (forced_tile_kernel adds the forced ones).
 template <int G>
 __global__ void __launch_bounds__(256) topk_kernel(const int32_t* __restrict__ cand, const float* __restrict__ lse,
                                                    int32_t* __restrict__ idx, float* __restrict__ z2,
-                                                   SelectParams p) {
+                                                   int32_t* __restrict__ counts, int64_t M1, SelectParams p) {
     const int lane = threadIdx.x & 31;
-    const int64_t unit = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-    const int64_t units = (int64_t)p.B * p.Hkv * p.N;
-    if (unit >= units) return;
-    const int64_t bh = unit / p.N;
-    const int64_t t = unit - bh * p.N;
+    const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (t >= p.N) return;
+    const int64_t bh = blockIdx.y;
+    const int64_t unit = bh * p.N + t;
     const Forced F(t, p.C, p.causal, p.forced_mask);
     const int leaf = cand[unit * kSlots + lane];
     float l2[G];
@@ -349,6 +385,8 @@ __global__ void __launch_bounds__(256) topk_kernel(const int32_t* __restrict__ c
     const int kept = keep_topk(id, s.valid ? score : -INFINITY, s, p.K, lane);
     bool mine = false;
     for (int j = 0; j < kept; ++j) mine |= (__shfl_sync(kFull, id, j) == leaf) && s.valid;
+    mine = mine && !s.forced;
+    if (mine) atomicAdd(&counts[bh * M1 + leaf], 1);  // bucket count of the attention grouping
 #pragma unroll
     for (int h = 0; h < G; ++h) {
         const float x = mine ? l2[h] : -INFINITY;
@@ -434,8 +472,7 @@ __global__ void __launch_bounds__(128) attn_tile_kernel(const __nv_bfloat16* __r
             int nvalid = 0;
             float z = 0.f;
             if (t >= 0) {
-                nvalid = (int)min((int64_t)kBlk, (int64_t)p.N - leaf * kBlk);
-                if (p.causal && leaf == t / kBlk) nvalid = min(nvalid, t - (int)(leaf * kBlk) + 1);
+                nvalid = visible_keys(leaf, t, p.N, p.causal);
                 z = z2[(bh * p.N + t) * G + (tid % G)];
             }
 #pragma unroll
@@ -493,21 +530,249 @@ __global__ void __launch_bounds__(128) attn_tile_kernel(const __nv_bfloat16* __r
     }
 }
 
-// z2[unit * G + h] = log2 sum over the listed leaves of 2^lse (slot = index in idx)
+// z2[unit * G + h] = log2 sum of 2^lse over the listed leaves that are not
+// forced leaves of the query (slot = index in idx); forced_tile_kernel adds the rest.
 template <int G>
 __global__ void z2_kernel(const int32_t* __restrict__ idx, const float* __restrict__ lse, float* __restrict__ z2,
-                          int64_t units, int K) {
+                          int64_t units, int K, int N, int C, int causal, int forced_mask) {
     const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= units * G) return;
     const int64_t unit = i / G;
     const int h = (int)(i - unit * G);
+    const Forced F(unit % N, C, causal, forced_mask);
     float m = -INFINITY;
-    for (int k = 0; k < K; ++k)
-        if (idx[unit * K + k] >= 0) m = fmaxf(m, lse[(unit * kSlots + k) * G + h]);
+    for (int k = 0; k < K; ++k) {
+        const int leaf = idx[unit * K + k];
+        if (leaf >= 0 && !F.has(leaf, 1)) m = fmaxf(m, lse[(unit * kSlots + k) * G + h]);
+    }
     float e = 0.f;
-    for (int k = 0; k < K; ++k)
-        if (idx[unit * K + k] >= 0) e += exp2f(lse[(unit * kSlots + k) * G + h] - m);
+    for (int k = 0; k < K; ++k) {
+        const int leaf = idx[unit * K + k];
+        if (leaf >= 0 && !F.has(leaf, 1)) e += exp2f(lse[(unit * kSlots + k) * G + h] - m);
+    }
     z2[i] = m + log2f(e);
+}
+
+// ---------------------------------------------------- forced leaves, dense ----
+
+// The forced leaves of a query (first, previous, current; close reading §5.3)
+// are the same for every query of a leaf block, so they are attended densely:
+// a tile holds 128/G consecutive positions (x G heads) of one (b, kv-head),
+// whose forced leaves are at most 4 distinct leaves U. Pass 1 runs S = Q K_u^T
+// per leaf u (tcgen05, TMEM) and folds each row's masked LSE into the
+// normaliser Z = log2(2^z2 + sum_u 2^LSE_u) (z2 holds the non-forced part on
+// entry, Z on exit). Pass 2 recomputes S, forms P = 2^(S*scale - Z) and
+// accumulates O = sum_u P_u V_u on the tensor cores; the rows are stored into
+// the fp32 accumulator as its initial value (the non-forced tiles add to it).
+// A leaf counts for a row only if it is a forced leaf of that query and is
+// listed in the query's idx row.
+struct ForcedParams {
+    int B, Hq, Hkv, N, causal, forced_mask, K;
+    float qscale;
+    int64_t tiles_per_head;
+};
+
+__device__ __forceinline__ int forced_union(int64_t t0, int64_t t1, int causal, int mask, int* U) {
+    int n = 0;
+    auto add = [&](int v) {
+        for (int i = 0; i < n; ++i)
+            if (U[i] == v) return;
+        U[n++] = v;
+    };
+    for (int64_t c = t0 / kBlk; c <= (t1 - 1) / kBlk; ++c) {
+        if (mask & 1) add(0);
+        if ((mask & 2) && c >= 1) add((int)c - 1);
+        if ((mask & 4) || causal) add((int)c);
+    }
+    return n;
+}
+
+template <int G>
+__global__ void __launch_bounds__(128) forced_tile_kernel(const __nv_bfloat16* __restrict__ Q,
+                                                          const __nv_bfloat16* __restrict__ Kmat,
+                                                          const __nv_bfloat16* __restrict__ Vmat,
+                                                          const int32_t* __restrict__ idx, float* __restrict__ z2,
+                                                          float* __restrict__ oacc, int* __restrict__ err,
+                                                          ForcedParams p) {
+    constexpr int QPT = 128 / G;  // query positions per tile
+    extern __shared__ __align__(1024) uint8_t dsm[];
+    uint8_t* sA = dsm;          // 32 KB query rows
+    uint8_t* sK = dsm + 32768;  // 16 KB key block
+    uint8_t* sV = dsm + 49152;  // 16 KB value block (MN-major)
+    uint8_t* sP = dsm + 65536;  // 16 KB probabilities
+    __shared__ TileRows tr;
+    __shared__ __align__(8) uint64_t mbar;
+    __shared__ uint32_t tmem_base;
+    const int tid = threadIdx.x, warp = tid >> 5;
+    if (warp == 0) tc::tmem_alloc(&tmem_base, 256);
+    if (tid == 0) {
+        tc::mbar_init(&mbar, 1);
+        tc::fence_mbar_init();
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    const uint32_t tmem_s = tmem_base, tmem_o = tmem_base + 128;
+    const uint32_t a_smem = tc::smem_u32(sA), k_smem = tc::smem_u32(sK), v_smem = tc::smem_u32(sV),
+                   p_smem = tc::smem_u32(sP);
+    const int64_t ntiles = (int64_t)p.B * p.Hkv * p.tiles_per_head;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int64_t tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+        const int64_t bh = tile / p.tiles_per_head;
+        const int64_t t0 = (tile - bh * p.tiles_per_head) * QPT;
+        const int64_t t1 = min(t0 + QPT, (int64_t)p.N);
+        const int64_t b = bh / p.Hkv;
+        const int kvh = (int)(bh - b * p.Hkv);
+        const int64_t t = t0 + tid / G;
+        const bool row_ok = t < t1;
+        tr.t[tid] = row_ok ? (int)t : -1;
+        tr.slot[tid] = 0;
+        int U[4];
+        const int nu = forced_union(t0, t1, p.causal, p.forced_mask, U);
+        // which of U count for this row: forced for t and listed in idx[t]
+        unsigned member = 0;
+        if (row_ok) {
+            const Forced F(t, kBlk, p.causal, p.forced_mask);
+            const int32_t* row = idx + (bh * p.N + t) * p.K;
+            for (int k = 0; k < p.K; ++k) {
+                const int leaf = row[k];
+                for (int i = 0; i < nu; ++i)
+                    if (leaf == U[i] && F.has(leaf, 1)) member |= 1u << i;
+            }
+        }
+        __syncthreads();
+        gather_q<G>(a_smem, tr, Q, b, kvh, p.Hq, p.N, tid);
+        // pass 1: per-row LSE of every member leaf -> Z
+        float lse_f = -INFINITY;
+        for (int i = 0; i < nu && ok; ++i) {
+            load_kblock(k_smem, Kmat + bh * p.N * kD, (int64_t)U[i] * kBlk, p.N, tid);
+            tc::cp_async_commit();
+            tc::cp_async_wait_all();
+            tc::fence_async_smem();
+            __syncthreads();
+            if (tid == 0) {
+                tc::tc_fence_after();
+                issue_qk(tmem_s, a_smem, k_smem);
+                tc::mma_commit(&mbar);
+            }
+            ok = __syncthreads_and(tc::mbar_wait(&mbar, phase, err, 4)) != 0;
+            phase ^= 1;
+            if (!ok) break;
+            tc::tc_fence_after();
+            float v[64];
+            const uint32_t taddr = tmem_s + ((uint32_t)(warp * 32) << 16);
+            tc::tmem_ld32(taddr, v);
+            tc::tmem_ld32(taddr + 32, v + 32);
+            tc::tmem_ld_wait();
+            if ((member >> i) & 1u) {
+                const int nvalid = visible_keys(U[i], t, p.N, p.causal);
+                float m = -INFINITY;
+#pragma unroll
+                for (int j = 0; j < 64; ++j)
+                    if (j < nvalid) m = fmaxf(m, v[j] * p.qscale);
+                float sum = 0.f;
+#pragma unroll
+                for (int j = 0; j < 64; ++j)
+                    if (j < nvalid) sum += exp2f(v[j] * p.qscale - m);
+                lse_f = logaddexp2f(lse_f, m + log2f(sum));
+            }
+            tc::tc_fence_before();
+            __syncthreads();
+        }
+        if (!ok) break;
+        float z = -INFINITY;
+        if (row_ok) {
+            float* zp = z2 + (bh * p.N + t) * G + (tid % G);
+            z = logaddexp2f(*zp, lse_f);
+            *zp = z;
+        }
+        // pass 2: O = sum_u P_u V_u
+        for (int i = 0; i < nu && ok; ++i) {
+            load_kblock(k_smem, Kmat + bh * p.N * kD, (int64_t)U[i] * kBlk, p.N, tid);
+            load_vblock(v_smem, Vmat + bh * p.N * kD, (int64_t)U[i] * kBlk, p.N, tid);
+            tc::cp_async_commit();
+            tc::cp_async_wait_all();
+            tc::fence_async_smem();
+            __syncthreads();
+            if (tid == 0) {
+                tc::tc_fence_after();
+                issue_qk(tmem_s, a_smem, k_smem);
+                tc::mma_commit(&mbar);
+            }
+            ok = __syncthreads_and(tc::mbar_wait(&mbar, phase, err, 5)) != 0;
+            phase ^= 1;
+            if (!ok) break;
+            tc::tc_fence_after();
+            {
+                float v[64];
+                const uint32_t taddr = tmem_s + ((uint32_t)(warp * 32) << 16);
+                tc::tmem_ld32(taddr, v);
+                tc::tmem_ld32(taddr + 32, v + 32);
+                tc::tmem_ld_wait();
+                const int nvalid = ((member >> i) & 1u) ? visible_keys(U[i], t, p.N, p.causal) : 0;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    uint32_t w4[4];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const int j = c * 8 + q * 2;
+                        const float p0 = j < nvalid ? exp2f(v[j] * p.qscale - z) : 0.f;
+                        const float p1 = j + 1 < nvalid ? exp2f(v[j + 1] * p.qscale - z) : 0.f;
+                        __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+                        w4[q] = *reinterpret_cast<uint32_t*>(&h2);
+                    }
+                    *reinterpret_cast<uint4*>(sP + tc::kmajor64_off(tid, c)) =
+                        make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                }
+            }
+            tc::fence_async_smem();
+            tc::tc_fence_before();
+            __syncthreads();
+            if (tid == 0) {
+                tc::tc_fence_after();
+                constexpr uint32_t idesc = tc::idesc_bf16(128, 128, 1);
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    tc::mma_bf16(tmem_o, tc::smem_desc(p_smem + k * 256, 128, 1024),
+                                 tc::smem_desc(v_smem + k * 256, 128, 1024), idesc, (i > 0 || k > 0) ? 1u : 0u);
+                tc::mma_commit(&mbar);
+            }
+            ok = __syncthreads_and(tc::mbar_wait(&mbar, phase, err, 6)) != 0;
+            phase ^= 1;
+            if (!ok) break;
+            tc::tc_fence_after();
+        }
+        if (!ok) break;
+        // initial value of the output accumulator for these rows
+        {
+            float* dst = row_ok ? oacc + (((b * p.Hq + (int64_t)kvh * G + (tid % G)) * p.N) + t) * kD : nullptr;
+            const uint32_t taddr = tmem_o + ((uint32_t)(warp * 32) << 16);
+#pragma unroll
+            for (int part = 0; part < 4; ++part) {
+                float v[32];
+                if (nu > 0) {
+                    tc::tmem_ld32(taddr + part * 32, v);
+                    tc::tmem_ld_wait();
+                } else {
+#pragma unroll
+                    for (int q = 0; q < 32; ++q) v[q] = 0.f;
+                }
+                if (dst) {
+#pragma unroll
+                    for (int q = 0; q < 32; q += 4)
+                        *reinterpret_cast<float4*>(dst + part * 32 + q) = make_float4(v[q], v[q + 1], v[q + 2], v[q + 3]);
+                }
+            }
+        }
+        tc::tc_fence_before();
+        __syncthreads();
+    }
+    __syncthreads();
+    if (warp == 0) {
+        tc::tc_fence_after();
+        tc::tmem_dealloc(tmem_base, 256);
+    }
 }
 
 __global__ void finalize_kernel(const float* __restrict__ oacc, __nv_bfloat16* __restrict__ O, int64_t n4) {
@@ -555,24 +820,41 @@ static void mark(const PhaseEvents* ev, int i, cudaStream_t st) {
     if (ev && ev->events && i < ev->n && ev->events[i]) cudaEventRecord((cudaEvent_t)ev->events[i], st);
 }
 
-// groups the entries of `src` (stride ids per unit) into tiles; returns launch error
-static cudaError_t build_tiles(const int32_t* src, int stride, const BmShape& s, uint8_t* ws, const BmLayout& L,
-                               cudaStream_t st) {
-    const int64_t units = (int64_t)s.B * s.Hkv * s.N;
+static dim3 unit_grid(const BmShape& s) { return dim3((unsigned)((s.N + 7) / 8), (unsigned)(s.B * s.Hkv)); }
+
+static GroupParams group_params(int stride, const SelectParams& sp, const BmShape& s) {
+    return GroupParams{s.N, sp.C, sp.causal, sp.forced_mask, stride, s.M1};
+}
+
+static cudaError_t zero_counts(const BmShape& s, uint8_t* ws, const BmLayout& L, cudaStream_t st) {
     const int64_t nb = (int64_t)s.B * s.Hkv * s.M1;
-    int32_t* counts = (int32_t*)(ws + L.counts);
-    int32_t* cursor = (int32_t*)(ws + L.cursor);
-    cudaError_t e = cudaMemsetAsync(counts, 0, nb * 4, st);
+    cudaError_t e = cudaMemsetAsync(ws + L.counts, 0, nb * 4, st);
     if (e != cudaSuccess) return e;
-    e = cudaMemsetAsync(cursor, 0, nb * 4, st);
-    if (e != cudaSuccess) return e;
-    bucket_count_kernel<<<grid_for(units, 256), 256, 0, st>>>(src, stride, units, s.N, s.M1, counts);
-    bucket_scan_kernel<<<1, 1024, 0, st>>>(counts, nb, s.M1, 128 / s.G, (int32_t*)(ws + L.offsets),
-                                           (int4*)(ws + L.tiles), (int32_t*)(ws + L.misc));
-    bucket_fill_kernel<<<grid_for(units, 256), 256, 0, st>>>(src, stride, units, s.N, s.M1,
-                                                             (const int32_t*)(ws + L.offsets), cursor,
-                                                             (uint32_t*)(ws + L.entries));
+    return cudaMemsetAsync(ws + L.cursor, 0, nb * 4, st);
+}
+
+// bucket counts of the non-forced entries of `src` must already be in place
+// (stage 1 and Top-K add them as they go); scan them and fill the lists
+static cudaError_t place_tiles(const int32_t* src, int stride, const SelectParams& sp, const BmShape& s,
+                               uint8_t* ws, const BmLayout& L, cudaStream_t st) {
+    const int64_t nb = (int64_t)s.B * s.Hkv * s.M1;
+    bucket_scan_kernel<<<1, 1024, 0, st>>>((const int32_t*)(ws + L.counts), nb, s.M1, 128 / s.G,
+                                           (int32_t*)(ws + L.offsets), (int4*)(ws + L.tiles),
+                                           (int32_t*)(ws + L.misc));
+    bucket_fill_kernel<<<unit_grid(s), 256, 0, st>>>(src, group_params(stride, sp, s), (const int32_t*)(ws + L.offsets),
+                                                     (int32_t*)(ws + L.cursor), (uint32_t*)(ws + L.entries));
     return cudaGetLastError();
+}
+
+// count, scan and fill for a caller-provided list (standalone attention)
+static cudaError_t build_tiles(const int32_t* src, int stride, const SelectParams& sp, const BmShape& s, uint8_t* ws,
+                               const BmLayout& L, cudaStream_t st) {
+    cudaError_t e = zero_counts(s, ws, L, st);
+    if (e != cudaSuccess) return e;
+    bucket_count_kernel<<<unit_grid(s), 256, 0, st>>>(src, group_params(stride, sp, s), (int32_t*)(ws + L.counts));
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    return place_tiles(src, stride, sp, s, ws, L, st);
 }
 
 static int sm_count() {
@@ -602,21 +884,27 @@ template <int G>
 static cudaError_t select_bm_t(const void* Q, const void* K, const float* pyr, int32_t* idx, const SelectParams& sp,
                                const BmShape& s, uint8_t* ws, const PhaseEvents* ev, cudaStream_t st) {
     const BmLayout L = blockmajor_layout(s);
-    const int64_t units = (int64_t)s.B * s.Hkv * s.N;
     int32_t* cand = (int32_t*)(ws + L.cand);
-    stage1_kernel<G><<<grid_for(units, 8), 256, 0, st>>>((const __nv_bfloat16*)Q, pyr, cand, sp);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = cudaMemsetAsync(ws + L.misc, 0, 256, st);
+    if (e != cudaSuccess) return e;
+    e = zero_counts(s, ws, L, st);
+    if (e != cudaSuccess) return e;
+    using W = typename std::conditional<(G <= 2), Walk4S<(G <= 2 ? G : 1)>, Walk<__nv_bfloat16, kD, G>>::type;
+    stage1_kernel<G, W><<<unit_grid(s), 256, 0, st>>>((const __nv_bfloat16*)Q, pyr, cand,
+                                                      (int32_t*)(ws + L.counts), s.M1, sp);
+    e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     mark(ev, 2, st);
-    e = cudaMemsetAsync(ws + L.misc, 0, 256, st);
-    if (e != cudaSuccess) return e;
-    e = build_tiles(cand, kSlots, s, ws, L, st);
+    e = place_tiles(cand, kSlots, sp, s, ws, L, st);
     if (e != cudaSuccess) return e;
     mark(ev, 3, st);
     e = leaf_scores<G>(Q, K, sp, s, ws, L, st);
     if (e != cudaSuccess) return e;
     mark(ev, 4, st);
-    topk_kernel<G><<<grid_for(units, 8), 256, 0, st>>>(cand, (const float*)(ws + L.lse), idx, (float*)(ws + L.z2), sp);
+    e = zero_counts(s, ws, L, st);  // the Top-K counts the kept leaves for the attention grouping
+    if (e != cudaSuccess) return e;
+    topk_kernel<G><<<unit_grid(s), 256, 0, st>>>(cand, (const float*)(ws + L.lse), idx, (float*)(ws + L.z2),
+                                                  (int32_t*)(ws + L.counts), s.M1, sp);
     e = cudaGetLastError();
     mark(ev, 5, st);
     return e;
@@ -630,23 +918,38 @@ static cudaError_t attn_bm_t(const void* Q, const void* K, const void* V, const 
     float* oacc = (float*)(ws + L.oacc);
     const int64_t units = (int64_t)s.B * s.Hkv * s.N;
     const int64_t nO = (int64_t)s.B * s.Hq * s.N * kD;
-    cudaError_t e = cudaMemsetAsync(oacc, 0, nO * 4, st);
-    if (e != cudaSuccess) return e;
+    cudaError_t e;
     if (!have_z2) {
         e = cudaMemsetAsync(ws + L.misc, 0, 256, st);
         if (e != cudaSuccess) return e;
     }
-    e = build_tiles(idx, sp.K, s, ws, L, st);
+    // the selection leaves the kept leaves' bucket counts in place
+    e = have_z2 ? place_tiles(idx, sp.K, sp, s, ws, L, st) : build_tiles(idx, sp.K, sp, s, ws, L, st);
     if (e != cudaSuccess) return e;
-    mark(ev, 6, st);
-    if (!have_z2) {  // per-head LSE of every listed leaf, then the normalisers
+    if (!have_z2) {  // per-head LSE of the listed non-forced leaves, then their part of the normaliser
         e = leaf_scores<G>(Q, K, sp, s, ws, L, st);
         if (e != cudaSuccess) return e;
         z2_kernel<G><<<grid_for(units * G, 256), 256, 0, st>>>(idx, (const float*)(ws + L.lse),
-                                                                (float*)(ws + L.z2), units, sp.K);
+                                                                (float*)(ws + L.z2), units, sp.K, s.N, sp.C,
+                                                                sp.causal, sp.forced_mask);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
+    mark(ev, 6, st);
+    {
+        ForcedParams fp{s.B, s.Hq, s.Hkv, s.N, sp.causal, sp.forced_mask, sp.K, sp.qscale,
+                        ((int64_t)s.N + 128 / G - 1) / (128 / G)};
+        auto fk = forced_tile_kernel<G>;
+        e = cudaFuncSetAttribute(fk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kAttnSmem);
+        if (e != cudaSuccess) return e;
+        const int64_t ntiles = (int64_t)s.B * s.Hkv * fp.tiles_per_head;
+        const int grid = (int)(ntiles < (int64_t)sm_count() * 2 ? ntiles : (int64_t)sm_count() * 2);
+        fk<<<grid, 128, kAttnSmem, st>>>((const __nv_bfloat16*)Q, (const __nv_bfloat16*)K, (const __nv_bfloat16*)V,
+                                         idx, (float*)(ws + L.z2), oacc, (int*)(ws + L.misc) + 1, fp);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    mark(ev, 7, st);
     TileParams tp{s.B, s.Hq, s.Hkv, s.N, sp.causal, s.M1, sp.qscale};
     auto kern = attn_tile_kernel<G>;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kAttnSmem);
@@ -657,10 +960,10 @@ static cudaError_t attn_bm_t(const void* Q, const void* K, const void* V, const 
                                                  (const float*)(ws + L.z2), oacc, (int*)(ws + L.misc) + 1, tp);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    mark(ev, 7, st);
+    mark(ev, 8, st);
     finalize_kernel<<<sm_count() * 8, 256, 0, st>>>(oacc, (__nv_bfloat16*)O, nO / 4);
     e = cudaGetLastError();
-    mark(ev, 8, st);
+    mark(ev, 9, st);
     return e;
 }
 

@@ -1,0 +1,155 @@
+// pisa_stage1.cuh -- the internal levels of the pyramid walk for one query,
+// one warp, laid out for few instructions per scored level (close reading
+// §04 4.2-4.4, Eq.(5)-(7), (11)).
+//
+// A scored level has at most 32 candidates (lane c owns candidate c) and needs
+// the dot products of q with both children of each: 64 fp32 summary rows of
+// 128 elements. Lanes are split into 8 groups of 4: group g handles the two
+// children of candidates 4g..4g+3 (8 rows, 1 KB contiguous per candidate);
+// inside a group lane j reads 16-byte chunks j, j+4, ..., j+28 of each row, so
+// every load instruction touches eight half-lines, and keeps the matching 32
+// elements of q in registers. A 2-stage reduce-scatter over the 4 lanes of
+// the group leaves lane 4g+j with both children of candidate 4g+j, so the
+// candidate's LSE over its children needs no further exchange.
+#pragma once
+
+#include "pisa_walk.cuh"
+
+namespace pisa {
+
+// q is held in shared memory (one 128 x G float slot per warp) and the row loop
+// sits inside the chunk loop: each lane keeps 8 independent row loads in
+// flight per chunk and needs few registers, so more warps fit on an SM.
+template <int G>
+struct Walk4S {
+    static_assert(G == 1 || G == 2, "Walk4S serves group sizes 1 and 2");
+    static constexpr int D = 128;
+    float* qs;  // this warp's slot: qs[h * 128 + (j + 4k) * 4 + e] (scaled)
+
+    __device__ __forceinline__ void load_q(const __nv_bfloat16* const* qrow, float scale, int lane) {
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+            float x[4];
+            Ld<__nv_bfloat16, 4>::run(qrow[h] + lane * 4, x);
+            *reinterpret_cast<float4*>(qs + h * 128 + lane * 4) =
+                make_float4(x[0] * scale, x[1] * scale, x[2] * scale, x[3] * scale);
+        }
+        __syncwarp();
+    }
+
+    __device__ __forceinline__ float score_internal(int cand, unsigned need, const float* child_lvl,
+                                                    int64_t span_child, int64_t n_keys, int lane) const {
+        const int g = lane >> 2, j = lane & 3;
+        int off[8];    // row offsets (floats) of the 8 rows, chunk j
+        bool okr[8];
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+            const int c = 4 * g + jj;
+            const int cc = __shfl_sync(kFull, cand, c);
+            const bool want = (need >> c) & 1u;
+#pragma unroll
+            for (int child = 0; child < 2; ++child) {
+                const int64_t row = 2 * (int64_t)cc + child;
+                const bool ok = want && row * span_child < n_keys;
+                okr[2 * jj + child] = ok;
+                off[2 * jj + child] = (int)((ok ? row : 0) * D) + j * 4;
+            }
+        }
+        float part[8 * G];
+#pragma unroll
+        for (int i = 0; i < 8 * G; ++i) part[i] = 0.f;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            float4 qk[G];
+#pragma unroll
+            for (int h = 0; h < G; ++h) qk[h] = *reinterpret_cast<const float4*>(qs + h * 128 + (j + 4 * k) * 4);
+#pragma unroll
+            for (int r = 0; r < 8; ++r) {
+                const float4 x = __ldg(reinterpret_cast<const float4*>(child_lvl + off[r] + 16 * k));
+#pragma unroll
+                for (int h = 0; h < G; ++h) {
+                    float a = part[r * G + h];
+                    a = fmaf(qk[h].x, x.x, a);
+                    a = fmaf(qk[h].y, x.y, a);
+                    a = fmaf(qk[h].z, x.z, a);
+                    a = fmaf(qk[h].w, x.w, a);
+                    part[r * G + h] = a;
+                }
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < 8; ++r)
+#pragma unroll
+            for (int h = 0; h < G; ++h)
+                if (!okr[r]) part[r * G + h] = 0.f;
+        constexpr int R = 2 * G;
+        {
+            const bool hi = (lane & 2) != 0;
+#pragma unroll
+            for (int i = 0; i < 2 * R; ++i) {
+                const float send = hi ? part[i] : part[i + 2 * R];
+                const float keep = hi ? part[i + 2 * R] : part[i];
+                part[i] = keep + __shfl_xor_sync(kFull, send, 2);
+            }
+        }
+        {
+            const bool hi = (lane & 1) != 0;
+#pragma unroll
+            for (int i = 0; i < R; ++i) {
+                const float send = hi ? part[i] : part[i + R];
+                const float keep = hi ? part[i + R] : part[i];
+                part[i] = keep + __shfl_xor_sync(kFull, send, 1);
+            }
+        }
+        const bool mine = (need >> lane) & 1u;
+        const bool has1 = (2 * (int64_t)cand + 1) * span_child < n_keys;
+        float score = 0.f;
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+            const float z0 = part[h], z1 = has1 ? part[G + h] : -INFINITY;
+            const float m = fmaxf(z0, z1);
+            score += (m == -INFINITY) ? -INFINITY : m + log2f(exp2f(z0 - m) + exp2f(z1 - m));
+        }
+        return mine ? score : -INFINITY;
+    }
+};
+
+// Keep-set of a scored level without a sort: every lane counts the lanes that
+// rank before it (higher key, then lower index) with 31 independent shuffles,
+// so the keep decision has no long dependent chain. Keys: +inf forced, the
+// score otherwise, -inf for invalid lanes. Lanes 0..kept-1 of the result hold
+// the kept ids (in lane order of the kept lanes); returns kept.
+__device__ __forceinline__ int keep_topk_rank(int& id, float key, bool valid, int K, int lane) {
+    const int ix = valid ? id : 0x7fffffff;
+    int before = 0;
+#pragma unroll
+    for (int o = 1; o < 32; ++o) {
+        const float ok = __shfl_xor_sync(kFull, key, o);
+        const int oi = __shfl_xor_sync(kFull, ix, o);
+        before += ranks_before(ok, oi, key, ix) ? 1 : 0;
+    }
+    const unsigned kmask = __ballot_sync(kFull, valid && before < K);
+    const int kept = __popc(kmask);
+    int src = 0;
+#pragma unroll
+    for (int step = 16; step >= 1; step >>= 1) {
+        const int probe = src + step;
+        if (probe <= 31 && __popc(kmask & ((1u << probe) - 1u)) <= lane) src = probe;
+    }
+    id = __shfl_sync(kFull, id, src);
+    return kept;
+}
+
+// Lanes 0..n-1 of the result hold the valid candidates in lane order
+// (a gather by rank: the lane holding the r-th set bit of vmask).
+__device__ __forceinline__ int compact_by_rank(int cand, unsigned vmask, int rank) {
+    int src = 0;
+#pragma unroll
+    for (int step = 16; step >= 1; step >>= 1) {
+        const int probe = src + step;
+        if (__popc(vmask & ((1u << probe) - 1u)) <= rank && probe <= 31) src = probe;
+    }
+    return __shfl_sync(kFull, cand, src);
+}
+
+}  // namespace pisa

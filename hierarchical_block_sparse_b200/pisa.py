@@ -51,6 +51,10 @@ def load(path: str | None = None):
         if _lib is not None and path is None:
             return _lib
         p = path or LIB_PATH
+        if path is None:
+            from . import build as _build
+            if not _build.up_to_date():  # sources newer than the library: rebuild, never run a stale one
+                _build.build()
         if not os.path.exists(p):
             raise RuntimeError(f"{p} is missing: build it with `python -m hierarchical_block_sparse_b200.build`")
         lib = ctypes.CDLL(p)
@@ -207,7 +211,8 @@ def pisa_select_noalloc(cfg, Q, K, pyr, idx):
                                                              _ptr(idx), _stream()))
 
 
-PHASES = ["pyramid", "stage1", "group_candidates", "leaf_scores", "topk", "group_kept", "attn_tiles", "finalize"]
+PHASES = ["pyramid", "stage1", "group_candidates", "leaf_scores", "topk", "group_kept", "forced_tiles",
+          "attn_tiles", "finalize"]
 
 
 def pisa_forward_ws_events(cfg, Q, K, V, pyr, idx, O, ws, events):

@@ -141,7 +141,8 @@ int pisa_bsa_select(const pisa_cfg *cfg, const void *Q, const float *pyr, int32_
  * per-query normaliser taken from the leaf LSEs. Results equal pisa_select /
  * pisa_sparse_attn up to fp32 rounding.
  * Limits: dtype bf16, d = 128, C = 64, K <= 16, G in {1,2,4,8,16}, N < 2^27,
- * B * Hkv * N * 32 < 2^31. Other shapes return PISA_E_UNSUPPORTED.
+ * B * Hkv * N * 32 < 2^31, B * Hkv <= 65535. Other shapes return
+ * PISA_E_UNSUPPORTED.
  * Workspace: caller-owned device memory of pisa_workspace_bytes(cfg) bytes,
  * 256-byte aligned; its contents are scratch (overwritten by every call, nothing
  * persists between calls except what pisa_forward_ws passes from its selection
@@ -174,10 +175,11 @@ int pisa_forward_ws(const pisa_cfg *cfg, const void *Q, const void *K, const voi
  * passed as void*, NULL entries skipped) on `stream` at its phase boundaries,
  * for per-phase timing with cudaEventElapsedTime. Index i marks the start of
  * phase i: 0 pyramid, 1 stage 1 (internal levels), 2 grouping of candidates,
- * 3 leaf scoring tiles, 4 final Top-K, 5 grouping of kept leaves, 6 attention
- * tiles, 7 output conversion; index 8 marks the end. n_events <= 9 are used.
- * Records only: no synchronisation, no allocation. */
-#define PISA_NUM_PHASES 8
+ * 3 leaf scoring tiles, 4 final Top-K, 5 grouping of kept leaves, 6 forced
+ * leaves (dense tiles), 7 attention tiles, 8 output conversion; index 9 marks
+ * the end. n_events <= 10 are used. Records only: no synchronisation, no
+ * allocation. */
+#define PISA_NUM_PHASES 9
 int pisa_forward_ws_events(const pisa_cfg *cfg, const void *Q, const void *K, const void *V, float *pyr,
                            int32_t *idx, void *O, void *workspace, size_t workspace_bytes, void *const *events,
                            int n_events, void *stream);

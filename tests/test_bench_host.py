@@ -24,6 +24,15 @@ def test_walk_counts_match_oracle(N, C, K, mask):
     np.testing.assert_array_equal(leafkeys, counts[:, 0, 1] * C)
     vis = np.array([sum(min(b * C + C, tt + 1) - b * C for b in row if b >= 0) for tt, row in zip(t, idx)])
     np.testing.assert_array_equal(attended, vis)
+    forced = [{0} if mask & 1 else set() for _ in t]
+    fvis = []
+    for tt, row, f in zip(t.tolist(), idx, forced):
+        c = tt // C
+        if mask & 2 and c >= 1:
+            f.add(c - 1)
+        f.add(c)
+        fvis.append(sum(min(b * C + C, tt + 1) - b * C for b in row if b in f))
+    np.testing.assert_array_equal(bench.walk_counts.forced_keys, np.array(fvis))
 
 
 def test_fp32_peak_formula():
