@@ -288,7 +288,7 @@ def main():
     ap.add_argument("--no-bsa", action="store_true")
     ap.add_argument("--no-per-query", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--cpu-seconds", type=float, default=16.0)
     args = ap.parse_args()
     if args.warmup < 3:
         print("warning: --warmup raised to 3", file=sys.stderr)

@@ -93,6 +93,9 @@ BmShape bm_shape(const pisa_cfg* c) {
     BmShape s;
     s.B = c->B; s.Hq = c->Hq; s.Hkv = c->Hkv; s.N = c->N; s.G = c->Hq / c->Hkv;
     s.M1 = ((int64_t)c->N + c->C - 1) / c->C;
+    Geom g;
+    make_geom(c->N, c->C, &g);
+    s.rows = g.rows;
     return s;
 }
 

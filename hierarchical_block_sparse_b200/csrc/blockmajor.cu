@@ -54,7 +54,8 @@ constexpr int kD = 128;      // head dimension handled by the tensor-core tiles
 template <int G, class W>
 __global__ void __launch_bounds__(256, PISA_STAGE1_MINBLOCKS) stage1_kernel(const __nv_bfloat16* __restrict__ Q,
                                                      const float* __restrict__ pyr, int32_t* __restrict__ cand_out,
-                                                     int32_t* __restrict__ counts, int64_t M1, SelectParams p) {
+                                                     int32_t* __restrict__ counts, int64_t M1, int* __restrict__ err,
+                                                     SelectParams p) {
     const int lane = threadIdx.x & 31;
     const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     if (t >= p.N) return;
@@ -93,8 +94,11 @@ __global__ void __launch_bounds__(256, PISA_STAGE1_MINBLOCKS) stage1_kernel(cons
         cand = lane < 2 * kept ? 2 * parent + (lane & 1) : -1;
     }
     const LevelState s = level_state(cand, 1, p.C, p.N, t, p.causal, F);
-    cand_out[unit * kSlots + lane] = s.valid ? cand : -1;
-    if (s.valid && !s.forced) atomicAdd(&counts[bh * M1 + cand], 1);
+    const bool in_range = cand >= 0 && cand < M1;
+    if (s.valid && !in_range && err) atomicCAS(err, 0, 10);  // self-check: never expected
+    const bool ok = s.valid && in_range;
+    cand_out[unit * kSlots + lane] = ok ? cand : -1;
+    if (ok && !s.forced) atomicAdd(&counts[bh * M1 + cand], 1);
 }
 
 // --------------------------------------------------------------- grouping ----
@@ -128,16 +132,27 @@ __global__ void bucket_count_kernel(const int32_t* __restrict__ src, GroupParams
 // single CTA: exclusive scan of all bucket counts into entry offsets, and the
 // tile list (b*Hkv + kvh, leaf, first entry, entries) of every bucket.
 __global__ void __launch_bounds__(1024) bucket_scan_kernel(const int32_t* __restrict__ counts, int64_t nbuckets,
-                                                           int64_t M1, int per_tile, int32_t* __restrict__ offsets,
-                                                           int4* __restrict__ tiles, int32_t* __restrict__ ntiles) {
+                                                           int64_t M1, int per_tile, int N, int32_t* __restrict__ offsets,
+                                                           int4* __restrict__ tiles, int32_t* __restrict__ ntiles,
+                                                           int* __restrict__ err) {
     __shared__ long long s_e[1024], s_t[1024];
     const int tid = threadIdx.x;
     const int64_t per = (nbuckets + 1023) / 1024;
     const int64_t lo = tid * per, hi = min(lo + per, nbuckets);
+    // self-check: a bucket holds at most one entry per query position
+    auto count_of = [&](int64_t i) {
+        const int c = counts[i];
+        if (c < 0 || c > N) {
+            atomicCAS(err, 0, 11);
+            return 0;
+        }
+        return c;
+    };
     long long e = 0, tt = 0;
     for (int64_t i = lo; i < hi; ++i) {
-        e += counts[i];
-        tt += (counts[i] + per_tile - 1) / per_tile;
+        const int c = count_of(i);
+        e += c;
+        tt += (c + per_tile - 1) / per_tile;
     }
     s_e[tid] = e;
     s_t[tid] = tt;
@@ -151,7 +166,7 @@ __global__ void __launch_bounds__(1024) bucket_scan_kernel(const int32_t* __rest
     }
     long long be = s_e[tid] - e, bt = s_t[tid] - tt;
     for (int64_t i = lo; i < hi; ++i) {
-        const int c = counts[i];
+        const int c = count_of(i);
         offsets[i] = (int32_t)be;
         const int nt = (c + per_tile - 1) / per_tile;
         for (int j = 0; j < nt; ++j)
@@ -185,17 +200,27 @@ struct TileRows {
     int slot[128];  // candidate slot of that query
 };
 
+// self-check of a tile descriptor (b*Hkv+kvh, leaf, first entry, entries)
+__device__ __forceinline__ bool tile_sane(const int4& td, int64_t bhs, int64_t M1, int per_tile) {
+    return td.x >= 0 && td.x < bhs && td.y >= 0 && td.y < M1 && td.z >= 0 && td.w > 0 && td.w <= per_tile;
+}
+
 // Row r of a tile is (entry r / G, head r % G). Fills row metadata.
 template <int G>
-__device__ __forceinline__ void tile_rows(TileRows& tr, const uint32_t* entries, int start, int len, int tid) {
+__device__ __forceinline__ void tile_rows(TileRows& tr, const uint32_t* entries, int start, int len, int N,
+                                          int* err, int tid) {
     const int e = tid / G;
+    tr.t[tid] = -1;
+    tr.slot[tid] = 0;
     if (e < len) {
         const uint32_t v = entries[start + e];
-        tr.t[tid] = (int)(v >> 5);
-        tr.slot[tid] = (int)(v & 31u);
-    } else {
-        tr.t[tid] = -1;
-        tr.slot[tid] = 0;
+        const int t = (int)(v >> 5);
+        if (t < N) {
+            tr.t[tid] = t;
+            tr.slot[tid] = (int)(v & 31u);
+        } else if (err) {
+            atomicCAS(err, 0, 13);  // self-check: never expected
+        }
     }
 }
 
@@ -268,6 +293,7 @@ struct TileParams {
     int B, Hq, Hkv, N, causal;
     int64_t M1;
     float qscale;  // log2(e) / sqrt(d)
+    int max_tiles;  // capacity of the tile list
 };
 
 // Per-head LSE (log2 units) of every listed (query, candidate leaf):
@@ -297,7 +323,7 @@ __global__ void __launch_bounds__(128) leaf_score_kernel(const __nv_bfloat16* __
     tc::tc_fence_after();
     const uint32_t tmem = tmem_base;
     const uint32_t a_smem = tc::smem_u32(sA), b_smem = tc::smem_u32(sB);
-    const int ntiles = *ntiles_ptr;
+    const int ntiles = min(*ntiles_ptr, p.max_tiles);
     uint32_t phase = 0;
     bool ok;
     for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
@@ -305,7 +331,11 @@ __global__ void __launch_bounds__(128) leaf_score_kernel(const __nv_bfloat16* __
         const int64_t bh = td.x, leaf = td.y;
         const int64_t b = bh / p.Hkv;
         const int kvh = (int)(bh - b * p.Hkv);
-        tile_rows<G>(tr, entries, td.z, td.w, tid);
+        if (!tile_sane(td, (int64_t)p.B * p.Hkv, p.M1, 128 / G)) {  // self-check: never expected
+            if (tid == 0) atomicCAS(err, 0, 12);
+            continue;
+        }
+        tile_rows<G>(tr, entries, td.z, td.w, p.N, err, tid);
         __syncthreads();
         gather_q<G>(a_smem, tr, Q, b, kvh, p.Hq, p.N, tid);
         load_kblock(b_smem, Kmat + bh * p.N * kD, leaf * kBlk, p.N, tid);
@@ -435,7 +465,7 @@ __global__ void __launch_bounds__(128) attn_tile_kernel(const __nv_bfloat16* __r
     const uint32_t tmem_s = tmem_base, tmem_o = tmem_base + 128;
     const uint32_t a_smem = tc::smem_u32(sA), k_smem = tc::smem_u32(sK), v_smem = tc::smem_u32(sV),
                    p_smem = tc::smem_u32(sP);
-    const int ntiles = *ntiles_ptr;
+    const int ntiles = min(*ntiles_ptr, p.max_tiles);
     uint32_t phase = 0;
     bool ok;
     for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
@@ -443,7 +473,11 @@ __global__ void __launch_bounds__(128) attn_tile_kernel(const __nv_bfloat16* __r
         const int64_t bh = td.x, leaf = td.y;
         const int64_t b = bh / p.Hkv;
         const int kvh = (int)(bh - b * p.Hkv);
-        tile_rows<G>(tr, entries, td.z, td.w, tid);
+        if (!tile_sane(td, (int64_t)p.B * p.Hkv, p.M1, 128 / G)) {  // self-check: never expected
+            if (tid == 0) atomicCAS(err, 0, 12);
+            continue;
+        }
+        tile_rows<G>(tr, entries, td.z, td.w, p.N, err, tid);
         __syncthreads();
         gather_q<G>(a_smem, tr, Q, b, kvh, p.Hq, p.N, tid);
         load_kblock(k_smem, Kmat + bh * p.N * kD, leaf * kBlk, p.N, tid);
@@ -788,11 +822,17 @@ __global__ void finalize_kernel(const float* __restrict__ oacc, __nv_bfloat16* _
 
 // -------------------------------------------------------------- host side ----
 
-BmLayout blockmajor_layout(const BmShape& s) {
+static int max_tiles_of(const BmShape& s) {
     const int64_t units = (int64_t)s.B * s.Hkv * s.N;
     const int64_t nb = (int64_t)s.B * s.Hkv * s.M1;
     const int per_tile = 128 / s.G;
-    const int64_t max_tiles = (units * kSlots + per_tile - 1) / per_tile + nb + 1;
+    return (int)((units * kSlots + per_tile - 1) / per_tile + nb + 1);
+}
+
+BmLayout blockmajor_layout(const BmShape& s) {
+    const int64_t units = (int64_t)s.B * s.Hkv * s.N;
+    const int64_t nb = (int64_t)s.B * s.Hkv * s.M1;
+    const int64_t max_tiles = max_tiles_of(s);
     BmLayout L;
     size_t off = 0;
     auto take = [&](size_t bytes) {
@@ -838,9 +878,9 @@ static cudaError_t zero_counts(const BmShape& s, uint8_t* ws, const BmLayout& L,
 static cudaError_t place_tiles(const int32_t* src, int stride, const SelectParams& sp, const BmShape& s,
                                uint8_t* ws, const BmLayout& L, cudaStream_t st) {
     const int64_t nb = (int64_t)s.B * s.Hkv * s.M1;
-    bucket_scan_kernel<<<1, 1024, 0, st>>>((const int32_t*)(ws + L.counts), nb, s.M1, 128 / s.G,
+    bucket_scan_kernel<<<1, 1024, 0, st>>>((const int32_t*)(ws + L.counts), nb, s.M1, 128 / s.G, s.N,
                                            (int32_t*)(ws + L.offsets), (int4*)(ws + L.tiles),
-                                           (int32_t*)(ws + L.misc));
+                                           (int32_t*)(ws + L.misc), (int*)(ws + L.misc) + 1);
     bucket_fill_kernel<<<unit_grid(s), 256, 0, st>>>(src, group_params(stride, sp, s), (const int32_t*)(ws + L.offsets),
                                                      (int32_t*)(ws + L.cursor), (uint32_t*)(ws + L.entries));
     return cudaGetLastError();
@@ -869,7 +909,7 @@ constexpr size_t kAttnSmem = 4 * 16384 + 16384;
 template <int G>
 static cudaError_t leaf_scores(const void* Q, const void* K, const SelectParams& sp, const BmShape& s, uint8_t* ws,
                                const BmLayout& L, cudaStream_t st) {
-    TileParams tp{s.B, s.Hq, s.Hkv, s.N, sp.causal, s.M1, sp.qscale};
+    TileParams tp{s.B, s.Hq, s.Hkv, s.N, sp.causal, s.M1, sp.qscale, max_tiles_of(s)};
     auto kern = leaf_score_kernel<G>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kScoreSmem);
     if (e != cudaSuccess) return e;
@@ -890,8 +930,8 @@ static cudaError_t select_bm_t(const void* Q, const void* K, const float* pyr, i
     e = zero_counts(s, ws, L, st);
     if (e != cudaSuccess) return e;
     using W = typename std::conditional<(G <= 2), Walk4S<(G <= 2 ? G : 1)>, Walk<__nv_bfloat16, kD, G>>::type;
-    stage1_kernel<G, W><<<unit_grid(s), 256, 0, st>>>((const __nv_bfloat16*)Q, pyr, cand,
-                                                      (int32_t*)(ws + L.counts), s.M1, sp);
+    stage1_kernel<G, W><<<unit_grid(s), 256, 0, st>>>((const __nv_bfloat16*)Q, pyr, cand, (int32_t*)(ws + L.counts),
+                                                      s.M1, (int*)(ws + L.misc) + 1, sp);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     mark(ev, 2, st);
@@ -950,7 +990,7 @@ static cudaError_t attn_bm_t(const void* Q, const void* K, const void* V, const 
         if (e != cudaSuccess) return e;
     }
     mark(ev, 7, st);
-    TileParams tp{s.B, s.Hq, s.Hkv, s.N, sp.causal, s.M1, sp.qscale};
+    TileParams tp{s.B, s.Hq, s.Hkv, s.N, sp.causal, s.M1, sp.qscale, max_tiles_of(s)};
     auto kern = attn_tile_kernel<G>;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kAttnSmem);
     if (e != cudaSuccess) return e;

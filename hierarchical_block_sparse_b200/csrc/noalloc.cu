@@ -69,13 +69,14 @@ extern "C" int pisa_select_noalloc(const pisa_cfg* cfg, const void* Q, const voi
     BmShape s;
     s.B = cfg->B; s.Hq = cfg->Hq; s.Hkv = cfg->Hkv; s.N = cfg->N; s.G = cfg->Hq / cfg->Hkv;
     s.M1 = ((int64_t)cfg->N + cfg->C - 1) / cfg->C;
+    Geom g;
+    make_geom(cfg->N, cfg->C, &g);
+    s.rows = g.rows;
     const BmLayout L = blockmajor_layout(s);
     // the selection uses every region except the attention accumulator, which is last
     if (L.oacc > kScratchBytes) return PISA_E_SCRATCH_LIMIT;
     void* ws = nullptr;
     if (scratch_address(&ws) != cudaSuccess || !ws) return PISA_E_CUDA;
-    Geom g;
-    make_geom(cfg->N, cfg->C, &g);
     SelectParams sp;
     sp.B = cfg->B; sp.Hq = cfg->Hq; sp.Hkv = cfg->Hkv; sp.N = cfg->N; sp.C = cfg->C; sp.K = cfg->K;
     sp.causal = cfg->causal; sp.forced_mask = cfg->forced_mask;

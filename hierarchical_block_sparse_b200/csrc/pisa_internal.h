@@ -36,7 +36,8 @@ struct DecodeParams {
 // block-major tensor-core path (bf16, d = 128, C = 64)
 struct BmShape {
     int B, Hq, Hkv, N, G;
-    int64_t M1;  // leaves per sequence
+    int64_t M1;    // leaves per sequence
+    int64_t rows;  // pyramid rows per (b, kv-head)
 };
 struct BmLayout {  // byte offsets of the workspace regions
     size_t cand, lse, z2, counts, cursor, offsets, entries, tiles, misc, oacc, total;
