@@ -289,6 +289,9 @@ def main():
     ap.add_argument("--no-per-query", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=16.0)
+    ap.add_argument("--decode-batch", type=int, default=0, help="override the decode batch (profiling)")
+    ap.add_argument("--decode-cache", type=int, default=0, help="override the cached keys per sequence")
+    ap.add_argument("--decode-only", action="store_true", help="skip the prefill measurement (profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         print("warning: --warmup raised to 3", file=sys.stderr)
@@ -317,6 +320,12 @@ def main():
     if not torch.cuda.is_available():
         raise RuntimeError("bench.py needs a CUDA device")
     pisa.load()
+    if args.decode_only:
+        dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+        torch.cuda.set_device(dev)
+        print(json.dumps({"decode": bench_decode(w, dev, torch.cuda.current_stream(), batch=args.decode_batch,
+                                                 cache=args.decode_cache), "config": config}))
+        return 0
     dist = None
     if world > 1:
         import datetime
@@ -493,7 +502,7 @@ def main():
 
     # ---- decode: 64 sequences, one new token each, against 256K-key caches ----
     if not args.no_decode and w.decode_batch:
-        out["decode"] = bench_decode(w, dev, stream)
+        out["decode"] = bench_decode(w, dev, stream, batch=args.decode_batch, cache=args.decode_cache)
 
     del Qd, Kd, Vd, pyr, idx, O, work
     torch.cuda.empty_cache()
@@ -515,11 +524,13 @@ def main():
     return 0
 
 
-def bench_decode(w, dev, stream, steps: int = 8):
+def bench_decode(w, dev, stream, steps: int = 8, batch: int = 0, cache: int = 0):
     import torch
     from hierarchical_block_sparse_b200 import pisa
     from hierarchical_block_sparse_b200.workloads import decode_cache, decode_step_inputs
-    prefix = w.N
+    if batch:
+        w = w.replace(decode_batch=batch)
+    prefix = cache or w.N
     cap = prefix + 64
     B = w.decode_batch
     Kc, Vc, _, _ = decode_cache(w, cap, prefix, dev)

@@ -7,11 +7,13 @@
 // Grouping (bucket_*): a counting sort turns the (query, slot) pairs of
 //   non-forced leaves into one list per (b, kv-head, leaf), cut into tiles of
 //   128/G queries.
-// Stage 2 (leaf_score_kernel): one tile per step: the queries' rows of every
-//   head of the group are gathered into shared memory (cp.async, canonical
-//   K-major layout), the leaf's 64 keys are loaded once, one tcgen05 MMA
-//   (M=128, N=64, K=128) writes the logits to TMEM and the epilogue turns each
-//   row into its exact per-head LSE (Eq.7 at the leaves).
+// Stage 2 (leaf_score_kernel): the level-1 candidates come in sibling pairs
+//   (both children of a kept level-2 node), grouped by that node. One tile per
+//   step: the queries' rows of every head of the group are gathered into
+//   shared memory (cp.async, canonical K-major layout), the pair's 128 keys
+//   are loaded once, one tcgen05 MMA (M=128, N=128, K=128) writes the logits
+//   to TMEM and the epilogue turns each row into the exact per-head LSE of
+//   each leaf (Eq.7 at the leaves).
 // Final Top-K (topk_kernel): per query, forced + best-ranked candidates by the
 //   LSE summed over the group (Eq.11), written sorted; it also records each
 //   head's partial softmax normaliser over the kept non-forced leaves.
@@ -98,7 +100,11 @@ __global__ void __launch_bounds__(256, PISA_STAGE1_MINBLOCKS) stage1_kernel(cons
     if (s.valid && !in_range && err) atomicCAS(err, 0, 10);  // self-check: never expected
     const bool ok = s.valid && in_range;
     cand_out[unit * kSlots + lane] = ok ? cand : -1;
-    if (ok && !s.forced) atomicAdd(&counts[bh * M1 + cand], 1);
+    // lanes 2i, 2i+1 hold the two children of one kept level-2 node: the pair
+    // is scored together, so the bucket is that node (counted once per pair)
+    const bool free_leaf = ok && !s.forced;
+    const bool odd_free = __shfl_down_sync(kFull, free_leaf, 1);
+    if ((lane & 1) == 0 && ok && (free_leaf || odd_free)) atomicAdd(&counts[bh * ((M1 + 1) / 2) + (cand >> 1)], 1);
 }
 
 // --------------------------------------------------------------- grouping ----
@@ -193,6 +199,29 @@ __global__ void bucket_fill_kernel(const int32_t* __restrict__ src, GroupParams 
     entries[pos] = ((uint32_t)t << 5) | (uint32_t)lane;
 }
 
+// Sibling pairs of level-1 candidates (slots 2i, 2i+1, children of one kept
+// level-2 node): one entry (t << 5 | i) per pair with at least one non-forced
+// leaf, in the bucket of that level-2 node. One warp per query position.
+__global__ void bucket_fill_pairs_kernel(const int32_t* __restrict__ cand, GroupParams g,
+                                         const int32_t* __restrict__ offsets, int32_t* __restrict__ cursor,
+                                         uint32_t* __restrict__ entries) {
+    const int lane = threadIdx.x & 31;
+    const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (t >= g.N) return;
+    if (lane >= kSlots / 2) return;
+    const int64_t bh = blockIdx.y;
+    const int64_t unit = bh * g.N + t;
+    const int leaf0 = cand[unit * kSlots + 2 * lane];
+    const int leaf1 = cand[unit * kSlots + 2 * lane + 1];
+    if (leaf0 < 0) return;
+    const Forced F(t, g.C, g.causal, g.forced_mask);
+    const bool f0 = !F.has(leaf0, 1), f1 = leaf1 >= 0 && !F.has(leaf1, 1);
+    if (!f0 && !f1) return;
+    const int64_t key = bh * g.M1 + (leaf0 >> 1);  // g.M1 = level-2 nodes per sequence here
+    const int pos = offsets[key] + atomicAdd(&cursor[key], 1);
+    entries[pos] = ((uint32_t)t << 5) | (uint32_t)lane;
+}
+
 // ---------------------------------------------------------- tile plumbing ----
 
 struct TileRows {
@@ -240,12 +269,14 @@ __device__ __forceinline__ void gather_q(uint32_t a_smem, const TileRows& tr, co
     }
 }
 
-// the leaf's 64 key rows into a K-major B tile (rows past n_keys are zero)
+// ROWS key rows (64: one leaf, 128: a sibling pair) into a K-major B tile
+// (rows past n_keys are zero)
+template <int ROWS = 64>
 __device__ __forceinline__ void load_kblock(uint32_t b_smem, const __nv_bfloat16* Kh, int64_t row0, int64_t n_keys,
                                             int tid) {
     const int i = tid & 7, c = tid >> 3;
 #pragma unroll
-    for (int g = 0; g < 8; ++g) {
+    for (int g = 0; g < ROWS / 8; ++g) {
         const int r = g * 8 + i;
         const int64_t row = row0 + r;
         const __nv_bfloat16* src = Kh + (row < n_keys ? row : row0) * kD + c * 8;
@@ -267,8 +298,9 @@ __device__ __forceinline__ void load_vblock(uint32_t v_smem, const __nv_bfloat16
     }
 }
 
+template <int NK = 64>
 __device__ __forceinline__ void issue_qk(uint32_t tmem_s, uint32_t a_smem, uint32_t b_smem) {
-    constexpr uint32_t idesc = tc::idesc_bf16(128, 64, 0);
+    constexpr uint32_t idesc = tc::idesc_bf16(128, NK, 0);
 #pragma unroll
     for (int k = 0; k < 8; ++k)
         tc::mma_bf16(tmem_s, tc::smem_desc(a_smem + k * 256, 128, 2048), tc::smem_desc(b_smem + k * 256, 128, 2048),
@@ -297,23 +329,27 @@ struct TileParams {
 };
 
 // Per-head LSE (log2 units) of every listed (query, candidate leaf):
-// lse[(unit * 32 + slot) * G + head].
-template <int G>
+// lse[(unit * 32 + slot) * G + head]. PAIR: a tile's key is a level-2 node p
+// and its entries are sibling-pair slots i; the 128 keys of leaves 2p and 2p+1
+// are scored by one N = 128 MMA and each non-forced visible leaf's LSE goes to
+// slot 2i or 2i+1.
+template <int G, bool PAIR>
 __global__ void __launch_bounds__(128) leaf_score_kernel(const __nv_bfloat16* __restrict__ Q,
                                                          const __nv_bfloat16* __restrict__ Kmat,
                                                          const int4* __restrict__ tiles,
                                                          const int32_t* __restrict__ ntiles_ptr,
                                                          const uint32_t* __restrict__ entries,
                                                          float* __restrict__ lse, int* __restrict__ err,
-                                                         TileParams p) {
+                                                         TileParams p, int forced_mask) {
+    constexpr int NK = PAIR ? 128 : 64;  // keys per tile
     extern __shared__ __align__(1024) uint8_t dsm[];
     uint8_t* sA = dsm;           // 32 KB gathered query rows
-    uint8_t* sB = dsm + 32768;   // 16 KB key block
+    uint8_t* sB = dsm + 32768;   // NK x 256 B key rows
     __shared__ TileRows tr;
     __shared__ __align__(8) uint64_t mbar;
     __shared__ uint32_t tmem_base;
     const int tid = threadIdx.x, warp = tid >> 5;
-    if (warp == 0) tc::tmem_alloc(&tmem_base, 64);
+    if (warp == 0) tc::tmem_alloc(&tmem_base, NK);
     if (tid == 0) {
         tc::mbar_init(&mbar, 1);
         tc::fence_mbar_init();
@@ -324,28 +360,29 @@ __global__ void __launch_bounds__(128) leaf_score_kernel(const __nv_bfloat16* __
     const uint32_t tmem = tmem_base;
     const uint32_t a_smem = tc::smem_u32(sA), b_smem = tc::smem_u32(sB);
     const int ntiles = min(*ntiles_ptr, p.max_tiles);
+    const int64_t nkeys = PAIR ? (p.M1 + 1) / 2 : p.M1;
     uint32_t phase = 0;
     bool ok;
     for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
         const int4 td = tiles[tile];
-        const int64_t bh = td.x, leaf = td.y;
+        const int64_t bh = td.x, key = td.y;
         const int64_t b = bh / p.Hkv;
         const int kvh = (int)(bh - b * p.Hkv);
-        if (!tile_sane(td, (int64_t)p.B * p.Hkv, p.M1, 128 / G)) {  // self-check: never expected
+        if (!tile_sane(td, (int64_t)p.B * p.Hkv, nkeys, 128 / G)) {  // self-check: never expected
             if (tid == 0) atomicCAS(err, 0, 12);
             continue;
         }
         tile_rows<G>(tr, entries, td.z, td.w, p.N, err, tid);
         __syncthreads();
         gather_q<G>(a_smem, tr, Q, b, kvh, p.Hq, p.N, tid);
-        load_kblock(b_smem, Kmat + bh * p.N * kD, leaf * kBlk, p.N, tid);
+        load_kblock<NK>(b_smem, Kmat + bh * p.N * kD, key * NK, p.N, tid);
         tc::cp_async_commit();
         tc::cp_async_wait_all();
         tc::fence_async_smem();
         __syncthreads();
         if (tid == 0) {
             tc::tc_fence_after();
-            issue_qk(tmem, a_smem, b_smem);
+            issue_qk<NK>(tmem, a_smem, b_smem);
             tc::mma_commit(&mbar);
         }
         // a CTA-uniform verdict: every thread polls, all agree before moving on
@@ -353,24 +390,35 @@ __global__ void __launch_bounds__(128) leaf_score_kernel(const __nv_bfloat16* __
         phase ^= 1;
         if (!ok) break;
         tc::tc_fence_after();
-        float v[64];
-        const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16);
-        tc::tmem_ld32(taddr, v);
-        tc::tmem_ld32(taddr + 32, v + 32);
-        tc::tmem_ld_wait();
         const int t = tr.t[tid];
-        if (t >= 0) {
-            const int nvalid = visible_keys(leaf, t, p.N, p.causal);
-            float m = -INFINITY;
+        const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16);
 #pragma unroll
-            for (int j = 0; j < 64; ++j)
-                if (j < nvalid) m = fmaxf(m, v[j] * p.qscale);
-            float s = 0.f;
+        for (int half = 0; half < NK / 64; ++half) {
+            float v[64];
+            tc::tmem_ld32(taddr + half * 64, v);
+            tc::tmem_ld32(taddr + half * 64 + 32, v + 32);
+            tc::tmem_ld_wait();
+            const int64_t leaf = PAIR ? 2 * key + half : key;
+            int slot = tr.slot[tid];
+            bool write = t >= 0;
+            if (PAIR && write) {
+                slot = 2 * slot + half;
+                const Forced F(t, kBlk, p.causal, forced_mask);
+                write = !F.has((int)leaf, 1);
+            }
+            const int nvalid = write ? visible_keys(leaf, t, p.N, p.causal) : 0;
+            if (write && (!PAIR || nvalid > 0)) {
+                float m = -INFINITY;
 #pragma unroll
-            for (int j = 0; j < 64; ++j)
-                if (j < nvalid) s += exp2f(v[j] * p.qscale - m);
-            const int64_t unit = bh * p.N + t;
-            lse[(unit * kSlots + tr.slot[tid]) * G + (tid % G)] = m + log2f(s);
+                for (int j = 0; j < 64; ++j)
+                    if (j < nvalid) m = fmaxf(m, v[j] * p.qscale);
+                float s = 0.f;
+#pragma unroll
+                for (int j = 0; j < 64; ++j)
+                    if (j < nvalid) s += exp2f(v[j] * p.qscale - m);
+                const int64_t unit = bh * p.N + t;
+                lse[(unit * kSlots + slot) * G + (tid % G)] = m + log2f(s);
+            }
         }
         tc::tc_fence_before();
         __syncthreads();
@@ -378,7 +426,7 @@ __global__ void __launch_bounds__(128) leaf_score_kernel(const __nv_bfloat16* __
     __syncthreads();
     if (warp == 0) {
         tc::tc_fence_after();
-        tc::tmem_dealloc(tmem, 64);
+        tc::tmem_dealloc(tmem, NK);
     }
 }
 
@@ -874,15 +922,24 @@ static cudaError_t zero_counts(const BmShape& s, uint8_t* ws, const BmLayout& L,
 }
 
 // bucket counts of the non-forced entries of `src` must already be in place
-// (stage 1 and Top-K add them as they go); scan them and fill the lists
+// (stage 1 and Top-K add them as they go); scan them and fill the lists.
+// pairs: `src` is the candidate list and the buckets are level-2 nodes.
 static cudaError_t place_tiles(const int32_t* src, int stride, const SelectParams& sp, const BmShape& s,
-                               uint8_t* ws, const BmLayout& L, cudaStream_t st) {
-    const int64_t nb = (int64_t)s.B * s.Hkv * s.M1;
-    bucket_scan_kernel<<<1, 1024, 0, st>>>((const int32_t*)(ws + L.counts), nb, s.M1, 128 / s.G, s.N,
+                               uint8_t* ws, const BmLayout& L, cudaStream_t st, bool pairs = false) {
+    const int64_t nkeys = pairs ? (s.M1 + 1) / 2 : s.M1;
+    const int64_t nb = (int64_t)s.B * s.Hkv * nkeys;
+    bucket_scan_kernel<<<1, 1024, 0, st>>>((const int32_t*)(ws + L.counts), nb, nkeys, 128 / s.G, s.N,
                                            (int32_t*)(ws + L.offsets), (int4*)(ws + L.tiles),
                                            (int32_t*)(ws + L.misc), (int*)(ws + L.misc) + 1);
-    bucket_fill_kernel<<<unit_grid(s), 256, 0, st>>>(src, group_params(stride, sp, s), (const int32_t*)(ws + L.offsets),
-                                                     (int32_t*)(ws + L.cursor), (uint32_t*)(ws + L.entries));
+    GroupParams g = group_params(stride, sp, s);
+    if (pairs) {
+        g.M1 = nkeys;
+        bucket_fill_pairs_kernel<<<unit_grid(s), 256, 0, st>>>(src, g, (const int32_t*)(ws + L.offsets),
+                                                               (int32_t*)(ws + L.cursor), (uint32_t*)(ws + L.entries));
+    } else {
+        bucket_fill_kernel<<<unit_grid(s), 256, 0, st>>>(src, g, (const int32_t*)(ws + L.offsets),
+                                                         (int32_t*)(ws + L.cursor), (uint32_t*)(ws + L.entries));
+    }
     return cudaGetLastError();
 }
 
@@ -903,20 +960,20 @@ static int sm_count() {
     return n;
 }
 
-constexpr size_t kScoreSmem = 32768 + 16384;
 constexpr size_t kAttnSmem = 4 * 16384 + 16384;
 
-template <int G>
+template <int G, bool PAIR>
 static cudaError_t leaf_scores(const void* Q, const void* K, const SelectParams& sp, const BmShape& s, uint8_t* ws,
                                const BmLayout& L, cudaStream_t st) {
     TileParams tp{s.B, s.Hq, s.Hkv, s.N, sp.causal, s.M1, sp.qscale, max_tiles_of(s)};
-    auto kern = leaf_score_kernel<G>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kScoreSmem);
+    constexpr size_t smem = 32768 + (PAIR ? 32768 : 16384);
+    auto kern = leaf_score_kernel<G, PAIR>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    kern<<<sm_count() * 4, 128, kScoreSmem, st>>>((const __nv_bfloat16*)Q, (const __nv_bfloat16*)K,
-                                                  (const int4*)(ws + L.tiles), (const int32_t*)(ws + L.misc),
-                                                  (const uint32_t*)(ws + L.entries), (float*)(ws + L.lse),
-                                                  (int*)(ws + L.misc) + 1, tp);
+    kern<<<sm_count() * (PAIR ? 3 : 4), 128, smem, st>>>((const __nv_bfloat16*)Q, (const __nv_bfloat16*)K,
+                                                          (const int4*)(ws + L.tiles), (const int32_t*)(ws + L.misc),
+                                                          (const uint32_t*)(ws + L.entries), (float*)(ws + L.lse),
+                                                          (int*)(ws + L.misc) + 1, tp, sp.forced_mask);
     return cudaGetLastError();
 }
 
@@ -935,10 +992,10 @@ static cudaError_t select_bm_t(const void* Q, const void* K, const float* pyr, i
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     mark(ev, 2, st);
-    e = place_tiles(cand, kSlots, sp, s, ws, L, st);
+    e = place_tiles(cand, kSlots, sp, s, ws, L, st, /*pairs=*/true);
     if (e != cudaSuccess) return e;
     mark(ev, 3, st);
-    e = leaf_scores<G>(Q, K, sp, s, ws, L, st);
+    e = leaf_scores<G, true>(Q, K, sp, s, ws, L, st);
     if (e != cudaSuccess) return e;
     mark(ev, 4, st);
     e = zero_counts(s, ws, L, st);  // the Top-K counts the kept leaves for the attention grouping
@@ -967,7 +1024,7 @@ static cudaError_t attn_bm_t(const void* Q, const void* K, const void* V, const 
     e = have_z2 ? place_tiles(idx, sp.K, sp, s, ws, L, st) : build_tiles(idx, sp.K, sp, s, ws, L, st);
     if (e != cudaSuccess) return e;
     if (!have_z2) {  // per-head LSE of the listed non-forced leaves, then their part of the normaliser
-        e = leaf_scores<G>(Q, K, sp, s, ws, L, st);
+        e = leaf_scores<G, false>(Q, K, sp, s, ws, L, st);
         if (e != cudaSuccess) return e;
         z2_kernel<G><<<grid_for(units * G, 256), 256, 0, st>>>(idx, (const float*)(ws + L.lse),
                                                                 (float*)(ws + L.z2), units, sp.K, s.N, sp.C,

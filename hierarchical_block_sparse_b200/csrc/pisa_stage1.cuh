@@ -55,9 +55,10 @@ struct Walk4S {
                 off[2 * jj + child] = (int)((ok ? row : 0) * D) + j * 4;
             }
         }
-        float part[8 * G];
+        // two interleaved partial sums per (row, head), packed fp32x2 FMAs
+        float2 acc[8 * G];
 #pragma unroll
-        for (int i = 0; i < 8 * G; ++i) part[i] = 0.f;
+        for (int i = 0; i < 8 * G; ++i) acc[i] = make_float2(0.f, 0.f);
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
             float4 qk[G];
@@ -68,20 +69,18 @@ struct Walk4S {
                 const float4 x = __ldg(reinterpret_cast<const float4*>(child_lvl + off[r] + 16 * k));
 #pragma unroll
                 for (int h = 0; h < G; ++h) {
-                    float a = part[r * G + h];
-                    a = fmaf(qk[h].x, x.x, a);
-                    a = fmaf(qk[h].y, x.y, a);
-                    a = fmaf(qk[h].z, x.z, a);
-                    a = fmaf(qk[h].w, x.w, a);
-                    part[r * G + h] = a;
+                    float2 a = acc[r * G + h];
+                    a = __ffma2_rn(make_float2(qk[h].x, qk[h].y), make_float2(x.x, x.y), a);
+                    a = __ffma2_rn(make_float2(qk[h].z, qk[h].w), make_float2(x.z, x.w), a);
+                    acc[r * G + h] = a;
                 }
             }
         }
+        float part[8 * G];
 #pragma unroll
         for (int r = 0; r < 8; ++r)
 #pragma unroll
-            for (int h = 0; h < G; ++h)
-                if (!okr[r]) part[r * G + h] = 0.f;
+            for (int h = 0; h < G; ++h) part[r * G + h] = okr[r] ? acc[r * G + h].x + acc[r * G + h].y : 0.f;
         constexpr int R = 2 * G;
         {
             const bool hi = (lane & 2) != 0;
