@@ -42,6 +42,8 @@ int check_gpu(const pisa_cfg* c) {
 }
 
 bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+// the block-major stage 1 reads pyramid rows with 256-bit loads
+bool aligned32(const void* p) { return ((uintptr_t)p & 31u) == 0; }
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? PISA_OK : PISA_E_CUDA; }
 
@@ -245,7 +247,7 @@ int pisa_select_ws(const pisa_cfg* cfg, const void* Q, const void* K, const floa
     if (s) return s;
     if (cfg->N == 0) return PISA_OK;
     if (!Q || !K || !pyr || !idx) return PISA_E_INVALID;
-    if (!aligned16(Q) || !aligned16(K) || !aligned16(pyr) || !aligned16(idx)) return PISA_E_ALIGNMENT;
+    if (!aligned16(Q) || !aligned16(K) || !aligned32(pyr) || !aligned16(idx)) return PISA_E_ALIGNMENT;
     s = check_ws(cfg, workspace, workspace_bytes);
     if (s) return s;
     Geom g;
@@ -276,7 +278,7 @@ int pisa_forward_ws_events(const pisa_cfg* cfg, const void* Q, const void* K, co
     if (s) return s;
     if (cfg->N == 0) return PISA_OK;
     if (!Q || !K || !V || !pyr || !idx || !O) return PISA_E_INVALID;
-    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(pyr) || !aligned16(idx) || !aligned16(O))
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned32(pyr) || !aligned16(idx) || !aligned16(O))
         return PISA_E_ALIGNMENT;
     if (n_events < 0 || (n_events > 0 && !events)) return PISA_E_INVALID;
     s = check_ws(cfg, workspace, workspace_bytes);
@@ -347,7 +349,7 @@ const char* pisa_status_string(int status) {
         case PISA_E_INVALID: return "invalid argument";
         case PISA_E_UNSUPPORTED: return "configuration outside the GPU kernels' limits";
         case PISA_E_CUDA: return "CUDA launch or runtime error";
-        case PISA_E_ALIGNMENT: return "tensor pointer not 16-byte aligned";
+        case PISA_E_ALIGNMENT: return "tensor pointer not 16-byte aligned (the pyramid: 32-byte for the block-major calls)";
         case PISA_E_TIMEOUT: return "a tensor-core tile gave up a bounded wait";
         case PISA_E_SCRATCH_LIMIT: return "problem exceeds the fixed scratch of pisa_select_noalloc";
     }

@@ -65,7 +65,8 @@ extern "C" int pisa_select_noalloc(const pisa_cfg* cfg, const void* Q, const voi
     if (need < 0) return (int)need;
     if (cfg->N == 0) return PISA_OK;
     if (!Q || !K || !pyr || !idx) return PISA_E_INVALID;
-    if ((((uintptr_t)Q | (uintptr_t)K | (uintptr_t)pyr | (uintptr_t)idx) & 15u) != 0) return PISA_E_ALIGNMENT;
+    if ((((uintptr_t)Q | (uintptr_t)K | (uintptr_t)idx) & 15u) != 0 || ((uintptr_t)pyr & 31u) != 0)
+        return PISA_E_ALIGNMENT;
     BmShape s;
     s.B = cfg->B; s.Hq = cfg->Hq; s.Hkv = cfg->Hkv; s.N = cfg->N; s.G = cfg->Hq / cfg->Hkv;
     s.M1 = ((int64_t)cfg->N + cfg->C - 1) / cfg->C;

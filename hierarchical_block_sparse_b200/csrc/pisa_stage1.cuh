@@ -4,18 +4,27 @@
 //
 // A scored level has at most 32 candidates (lane c owns candidate c) and needs
 // the dot products of q with both children of each: 64 fp32 summary rows of
-// 128 elements. Lanes are split into 8 groups of 4: group g handles the two
-// children of candidates 4g..4g+3 (8 rows, 1 KB contiguous per candidate);
-// inside a group lane j reads 16-byte chunks j, j+4, ..., j+28 of each row, so
-// every load instruction touches eight half-lines, and keeps the matching 32
-// elements of q in registers. A 2-stage reduce-scatter over the 4 lanes of
-// the group leaves lane 4g+j with both children of candidate 4g+j, so the
-// candidate's LSE over its children needs no further exchange.
+// 128 elements (512 bytes, four 128-byte lines). Lanes are split into 8 groups
+// of 4: group g handles the two children of candidates 4g..4g+3 (8 rows, 1 KB
+// contiguous per candidate); inside a group lane j reads the 32-byte chunks j,
+// j+4, j+8, j+12 of each row with 256-bit loads, so one load instruction
+// covers one whole line of each of 8 rows (the fewest L1 wavefronts for its
+// 1 KB), and keeps the matching 32 elements of q in shared memory. A 2-stage
+// reduce-scatter over the 4 lanes of the group leaves lane 4g+j with both
+// children of candidate 4g+j, so the candidate's LSE over its children needs
+// no further exchange.
 #pragma once
 
 #include "pisa_walk.cuh"
 
 namespace pisa {
+
+// 256-bit read-only global load (sm_100); p must be 32-byte aligned.
+__device__ __forceinline__ void ldg_nc_v8(const float* p, float (&x)[8]) {
+    asm("ld.global.nc.v8.f32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+        : "=f"(x[0]), "=f"(x[1]), "=f"(x[2]), "=f"(x[3]), "=f"(x[4]), "=f"(x[5]), "=f"(x[6]), "=f"(x[7])
+        : "l"(p));
+}
 
 // q is held in shared memory (one 128 x G float slot per warp) and the row loop
 // sits inside the chunk loop: each lane keeps 8 independent row loads in
@@ -24,7 +33,8 @@ template <int G>
 struct Walk4S {
     static_assert(G == 1 || G == 2, "Walk4S serves group sizes 1 and 2");
     static constexpr int D = 128;
-    float* qs;  // this warp's slot: qs[h * 128 + (j + 4k) * 4 + e] (scaled)
+    static constexpr int kChunk = 8;  // floats per lane per load (32 bytes)
+    float* qs;  // this warp's slot: qs[h * 128 + e], scaled, natural order
 
     __device__ __forceinline__ void load_q(const __nv_bfloat16* const* qrow, float scale, int lane) {
 #pragma unroll
@@ -52,7 +62,7 @@ struct Walk4S {
                 const int64_t row = 2 * (int64_t)cc + child;
                 const bool ok = want && row * span_child < n_keys;
                 okr[2 * jj + child] = ok;
-                off[2 * jj + child] = (int)((ok ? row : 0) * D) + j * 4;
+                off[2 * jj + child] = (int)((ok ? row : 0) * D) + j * kChunk;
             }
         }
         // two interleaved partial sums per (row, head), packed fp32x2 FMAs
@@ -60,18 +70,25 @@ struct Walk4S {
 #pragma unroll
         for (int i = 0; i < 8 * G; ++i) acc[i] = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-            float4 qk[G];
+        for (int k = 0; k < D / (4 * kChunk); ++k) {
+            const int e0 = (j + 4 * k) * kChunk;  // first element of this lane's chunk
+            float4 qa[G], qb[G];
 #pragma unroll
-            for (int h = 0; h < G; ++h) qk[h] = *reinterpret_cast<const float4*>(qs + h * 128 + (j + 4 * k) * 4);
+            for (int h = 0; h < G; ++h) {
+                qa[h] = *reinterpret_cast<const float4*>(qs + h * D + e0);
+                qb[h] = *reinterpret_cast<const float4*>(qs + h * D + e0 + 4);
+            }
 #pragma unroll
             for (int r = 0; r < 8; ++r) {
-                const float4 x = __ldg(reinterpret_cast<const float4*>(child_lvl + off[r] + 16 * k));
+                float x[8];
+                ldg_nc_v8(child_lvl + off[r] + 4 * kChunk * k, x);
 #pragma unroll
                 for (int h = 0; h < G; ++h) {
                     float2 a = acc[r * G + h];
-                    a = __ffma2_rn(make_float2(qk[h].x, qk[h].y), make_float2(x.x, x.y), a);
-                    a = __ffma2_rn(make_float2(qk[h].z, qk[h].w), make_float2(x.z, x.w), a);
+                    a = __ffma2_rn(make_float2(qa[h].x, qa[h].y), make_float2(x[0], x[1]), a);
+                    a = __ffma2_rn(make_float2(qa[h].z, qa[h].w), make_float2(x[2], x[3]), a);
+                    a = __ffma2_rn(make_float2(qb[h].x, qb[h].y), make_float2(x[4], x[5]), a);
+                    a = __ffma2_rn(make_float2(qb[h].z, qb[h].w), make_float2(x[6], x[7]), a);
                     acc[r * G + h] = a;
                 }
             }

@@ -58,7 +58,7 @@ enum pisa_status {
     PISA_E_INVALID = -1,      /* null pointer, bad size, inconsistent config */
     PISA_E_UNSUPPORTED = -2,  /* valid for the method, outside the GPU limits */
     PISA_E_CUDA = -3,         /* a CUDA launch or runtime call failed */
-    PISA_E_ALIGNMENT = -4,    /* a tensor pointer is not 16-byte aligned */
+    PISA_E_ALIGNMENT = -4,    /* a tensor pointer is not 16-byte aligned (pyramid of the *_ws calls: 32) */
     PISA_E_TIMEOUT = -5,      /* a kernel gave up a bounded wait (see pisa_workspace_status) */
     PISA_E_SCRATCH_LIMIT = -6 /* problem too large for pisa_select_noalloc's fixed scratch */
 };
@@ -142,7 +142,8 @@ int pisa_bsa_select(const pisa_cfg *cfg, const void *Q, const float *pyr, int32_
  * pisa_sparse_attn up to fp32 rounding.
  * Limits: dtype bf16, d = 128, C = 64, K <= 16, G in {1,2,4,8,16}, N < 2^27,
  * B * Hkv * N * 32 < 2^31, B * Hkv <= 65535. Other shapes return
- * PISA_E_UNSUPPORTED.
+ * PISA_E_UNSUPPORTED. The pyramid pointer must be 32-byte aligned (its rows are
+ * read with 256-bit loads), else PISA_E_ALIGNMENT.
  * Workspace: caller-owned device memory of pisa_workspace_bytes(cfg) bytes,
  * 256-byte aligned; its contents are scratch (overwritten by every call, nothing
  * persists between calls except what pisa_forward_ws passes from its selection

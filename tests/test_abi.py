@@ -124,3 +124,7 @@ def test_workspace_calls_validate_before_launch(lib):
     assert lib.pisa_select_ws(ctypes.byref(cfg), *P, None, need, None) == -1           # no workspace
     assert lib.pisa_select_ws(ctypes.byref(cfg), *P, ctypes.c_void_p(4096 + 16), need, None) == -4  # misaligned
     assert lib.pisa_select_ws(ctypes.byref(cfg), *P, ctypes.c_void_p(8192), need - 1, None) == -1   # too small
+    # the block-major stage 1 reads pyramid rows with 256-bit loads: pyr needs 32 bytes
+    P16 = [ctypes.c_void_p(4096), ctypes.c_void_p(4096), ctypes.c_void_p(4096 + 16), ctypes.c_void_p(4096)]
+    assert lib.pisa_select_ws(ctypes.byref(cfg), *P16, ctypes.c_void_p(8192), need, None) == -4
+    assert lib.pisa_select_noalloc(ctypes.byref(cfg), *P16, None) == -4
