@@ -38,6 +38,7 @@
 namespace pisa {
 
 constexpr int kSlots = 32;   // level-1 candidates per query (2K <= 32)
+constexpr int kPairs = 16;   // bucket slots recorded per query: sibling pairs, or kept leaves (K <= 16)
 constexpr int kBlk = 64;     // leaf size handled by the tensor-core tiles
 constexpr int kD = 128;      // head dimension handled by the tensor-core tiles
 
@@ -56,8 +57,8 @@ constexpr int kD = 128;      // head dimension handled by the tensor-core tiles
 template <int G, class W>
 __global__ void __launch_bounds__(256, PISA_STAGE1_MINBLOCKS) stage1_kernel(const __nv_bfloat16* __restrict__ Q,
                                                      const float* __restrict__ pyr, int32_t* __restrict__ cand_out,
-                                                     int32_t* __restrict__ counts, int64_t M1, int* __restrict__ err,
-                                                     SelectParams p) {
+                                                     int32_t* __restrict__ counts, int32_t* __restrict__ slots,
+                                                     int64_t M1, int* __restrict__ err, SelectParams p) {
     const int lane = threadIdx.x & 31;
     const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     if (t >= p.N) return;
@@ -91,20 +92,26 @@ __global__ void __launch_bounds__(256, PISA_STAGE1_MINBLOCKS) stage1_kernel(cons
             score = w.score_internal(cand, s.vmask & ~fmask, P + p.geom.off[l - 1] * kD,
                                      (int64_t)p.C << (l - 2), p.N, lane);
         int id = cand;
-        const int kept = keep_topk_rank(id, s.forced ? INFINITY : score, s.valid, p.K, lane);
+        const int kept = keep_topk_lane(id, s.forced ? INFINITY : score, s.valid, p.K, lane);
         parent = __shfl_sync(kFull, id, lane >> 1);
         cand = lane < 2 * kept ? 2 * parent + (lane & 1) : -1;
     }
     const LevelState s = level_state(cand, 1, p.C, p.N, t, p.causal, F);
     const bool in_range = cand >= 0 && cand < M1;
     if (s.valid && !in_range && err) atomicCAS(err, 0, 10);  // self-check: never expected
+    // self-check of the lane order the keep relies on: valid candidates ascend
+    const int prev = __shfl_up_sync(kFull, cand, 1);
+    const bool prev_valid = __shfl_up_sync(kFull, s.valid, 1);
+    if (lane > 0 && s.valid && prev_valid && prev >= cand && err) atomicCAS(err, 0, 14);
     const bool ok = s.valid && in_range;
     cand_out[unit * kSlots + lane] = ok ? cand : -1;
     // lanes 2i, 2i+1 hold the two children of one kept level-2 node: the pair
-    // is scored together, so the bucket is that node (counted once per pair)
+    // is scored together, so the bucket is that node (counted once per pair);
+    // the count before this pair's increment is its slot in the bucket
     const bool free_leaf = ok && !s.forced;
     const bool odd_free = __shfl_down_sync(kFull, free_leaf, 1);
-    if ((lane & 1) == 0 && ok && (free_leaf || odd_free)) atomicAdd(&counts[bh * ((M1 + 1) / 2) + (cand >> 1)], 1);
+    if ((lane & 1) == 0 && ok && (free_leaf || odd_free))
+        slots[unit * kPairs + (lane >> 1)] = atomicAdd(&counts[bh * ((M1 + 1) / 2) + (cand >> 1)], 1);
 }
 
 // --------------------------------------------------------------- grouping ----
@@ -126,13 +133,18 @@ __device__ __forceinline__ int free_leaf(const int32_t* src, const GroupParams& 
     return F.has(leaf, 1) ? -1 : leaf;
 }
 
-__global__ void bucket_count_kernel(const int32_t* __restrict__ src, GroupParams g, int32_t* __restrict__ counts) {
+// Counting is also placing: the count a list entry finds in its bucket before
+// its own increment is its slot there, recorded in slots[unit * kPairs + lane]
+// (g.stride <= kPairs), so the fill after the scan needs no atomics.
+__global__ void bucket_count_kernel(const int32_t* __restrict__ src, GroupParams g, int32_t* __restrict__ counts,
+                                    int32_t* __restrict__ slots) {
     const int lane = threadIdx.x & 31;
     const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     if (t >= g.N) return;
     const int64_t bh = blockIdx.y;
-    const int leaf = free_leaf(src, g, bh * g.N + t, t, lane);
-    if (leaf >= 0) atomicAdd(&counts[bh * g.M1 + leaf], 1);
+    const int64_t unit = bh * g.N + t;
+    const int leaf = free_leaf(src, g, unit, t, lane);
+    if (leaf >= 0) slots[unit * kPairs + lane] = atomicAdd(&counts[bh * g.M1 + leaf], 1);
 }
 
 // single CTA: exclusive scan of all bucket counts into entry offsets, and the
@@ -186,24 +198,23 @@ __global__ void __launch_bounds__(1024) bucket_scan_kernel(const int32_t* __rest
 
 // one warp per query position: write (t << 5 | slot) into each bucket
 __global__ void bucket_fill_kernel(const int32_t* __restrict__ src, GroupParams g,
-                                   const int32_t* __restrict__ offsets, int32_t* __restrict__ cursor,
+                                   const int32_t* __restrict__ offsets, const int32_t* __restrict__ slots,
                                    uint32_t* __restrict__ entries) {
     const int lane = threadIdx.x & 31;
     const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     if (t >= g.N) return;
     const int64_t bh = blockIdx.y;
-    const int leaf = free_leaf(src, g, bh * g.N + t, t, lane);
+    const int64_t unit = bh * g.N + t;
+    const int leaf = free_leaf(src, g, unit, t, lane);
     if (leaf < 0) return;
-    const int64_t key = bh * g.M1 + leaf;
-    const int pos = offsets[key] + atomicAdd(&cursor[key], 1);
-    entries[pos] = ((uint32_t)t << 5) | (uint32_t)lane;
+    entries[offsets[bh * g.M1 + leaf] + slots[unit * kPairs + lane]] = ((uint32_t)t << 5) | (uint32_t)lane;
 }
 
 // Sibling pairs of level-1 candidates (slots 2i, 2i+1, children of one kept
 // level-2 node): one entry (t << 5 | i) per pair with at least one non-forced
 // leaf, in the bucket of that level-2 node. One warp per query position.
 __global__ void bucket_fill_pairs_kernel(const int32_t* __restrict__ cand, GroupParams g,
-                                         const int32_t* __restrict__ offsets, int32_t* __restrict__ cursor,
+                                         const int32_t* __restrict__ offsets, const int32_t* __restrict__ slots,
                                          uint32_t* __restrict__ entries) {
     const int lane = threadIdx.x & 31;
     const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
@@ -218,8 +229,7 @@ __global__ void bucket_fill_pairs_kernel(const int32_t* __restrict__ cand, Group
     const bool f0 = !F.has(leaf0, 1), f1 = leaf1 >= 0 && !F.has(leaf1, 1);
     if (!f0 && !f1) return;
     const int64_t key = bh * g.M1 + (leaf0 >> 1);  // g.M1 = level-2 nodes per sequence here
-    const int pos = offsets[key] + atomicAdd(&cursor[key], 1);
-    entries[pos] = ((uint32_t)t << 5) | (uint32_t)lane;
+    entries[offsets[key] + slots[unit * kPairs + lane]] = ((uint32_t)t << 5) | (uint32_t)lane;
 }
 
 // ---------------------------------------------------------- tile plumbing ----
@@ -439,7 +449,8 @@ __global__ void __launch_bounds__(128) leaf_score_kernel(const __nv_bfloat16* __
 template <int G>
 __global__ void __launch_bounds__(256) topk_kernel(const int32_t* __restrict__ cand, const float* __restrict__ lse,
                                                    int32_t* __restrict__ idx, float* __restrict__ z2,
-                                                   int32_t* __restrict__ counts, int64_t M1, SelectParams p) {
+                                                   int32_t* __restrict__ counts, int32_t* __restrict__ slots,
+                                                   int64_t M1, SelectParams p) {
     const int lane = threadIdx.x & 31;
     const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     if (t >= p.N) return;
@@ -464,7 +475,6 @@ __global__ void __launch_bounds__(256) topk_kernel(const int32_t* __restrict__ c
     bool mine = false;
     for (int j = 0; j < kept; ++j) mine |= (__shfl_sync(kFull, id, j) == leaf) && s.valid;
     mine = mine && !s.forced;
-    if (mine) atomicAdd(&counts[bh * M1 + leaf], 1);  // bucket count of the attention grouping
 #pragma unroll
     for (int h = 0; h < G; ++h) {
         const float x = mine ? l2[h] : -INFINITY;
@@ -479,6 +489,9 @@ __global__ void __launch_bounds__(256) topk_kernel(const int32_t* __restrict__ c
     int v = lane < kept ? id : 0x7fffffff;
     warp_sort_asc(v, lane);
     if (lane < p.K) idx[unit * p.K + lane] = v == 0x7fffffff ? -1 : v;
+    // bucket count (and slot) of the attention grouping, by position in idx
+    if (lane < p.K && v != 0x7fffffff && !F.has(v, 1))
+        slots[unit * kPairs + lane] = atomicAdd(&counts[bh * M1 + v], 1);
 }
 
 // ------------------------------------------------------ attention tiles ----
@@ -892,7 +905,7 @@ BmLayout blockmajor_layout(const BmShape& s) {
     L.lse = take(units * kSlots * s.G * 4);
     L.z2 = take(units * s.G * 4);
     L.counts = take(nb * 4);
-    L.cursor = take(nb * 4);
+    L.slots = take(units * kPairs * 4);
     L.offsets = take(nb * 4);
     L.entries = take(units * kSlots * 4);
     L.tiles = take(max_tiles * 16);
@@ -916,13 +929,12 @@ static GroupParams group_params(int stride, const SelectParams& sp, const BmShap
 
 static cudaError_t zero_counts(const BmShape& s, uint8_t* ws, const BmLayout& L, cudaStream_t st) {
     const int64_t nb = (int64_t)s.B * s.Hkv * s.M1;
-    cudaError_t e = cudaMemsetAsync(ws + L.counts, 0, nb * 4, st);
-    if (e != cudaSuccess) return e;
-    return cudaMemsetAsync(ws + L.cursor, 0, nb * 4, st);
+    return cudaMemsetAsync(ws + L.counts, 0, nb * 4, st);
 }
 
-// bucket counts of the non-forced entries of `src` must already be in place
-// (stage 1 and Top-K add them as they go); scan them and fill the lists.
+// bucket counts and slots of the non-forced entries of `src` must already be
+// in place (stage 1 and Top-K record them as they go); scan the counts and
+// scatter the entries to their slots.
 // pairs: `src` is the candidate list and the buckets are level-2 nodes.
 static cudaError_t place_tiles(const int32_t* src, int stride, const SelectParams& sp, const BmShape& s,
                                uint8_t* ws, const BmLayout& L, cudaStream_t st, bool pairs = false) {
@@ -935,10 +947,11 @@ static cudaError_t place_tiles(const int32_t* src, int stride, const SelectParam
     if (pairs) {
         g.M1 = nkeys;
         bucket_fill_pairs_kernel<<<unit_grid(s), 256, 0, st>>>(src, g, (const int32_t*)(ws + L.offsets),
-                                                               (int32_t*)(ws + L.cursor), (uint32_t*)(ws + L.entries));
+                                                               (const int32_t*)(ws + L.slots),
+                                                               (uint32_t*)(ws + L.entries));
     } else {
         bucket_fill_kernel<<<unit_grid(s), 256, 0, st>>>(src, g, (const int32_t*)(ws + L.offsets),
-                                                         (int32_t*)(ws + L.cursor), (uint32_t*)(ws + L.entries));
+                                                         (const int32_t*)(ws + L.slots), (uint32_t*)(ws + L.entries));
     }
     return cudaGetLastError();
 }
@@ -948,7 +961,8 @@ static cudaError_t build_tiles(const int32_t* src, int stride, const SelectParam
                                const BmLayout& L, cudaStream_t st) {
     cudaError_t e = zero_counts(s, ws, L, st);
     if (e != cudaSuccess) return e;
-    bucket_count_kernel<<<unit_grid(s), 256, 0, st>>>(src, group_params(stride, sp, s), (int32_t*)(ws + L.counts));
+    bucket_count_kernel<<<unit_grid(s), 256, 0, st>>>(src, group_params(stride, sp, s), (int32_t*)(ws + L.counts),
+                                                      (int32_t*)(ws + L.slots));
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     return place_tiles(src, stride, sp, s, ws, L, st);
@@ -988,7 +1002,7 @@ static cudaError_t select_bm_t(const void* Q, const void* K, const float* pyr, i
     if (e != cudaSuccess) return e;
     using W = typename std::conditional<(G <= 2), Walk4S<(G <= 2 ? G : 1)>, Walk<__nv_bfloat16, kD, G>>::type;
     stage1_kernel<G, W><<<unit_grid(s), 256, 0, st>>>((const __nv_bfloat16*)Q, pyr, cand, (int32_t*)(ws + L.counts),
-                                                      s.M1, (int*)(ws + L.misc) + 1, sp);
+                                                      (int32_t*)(ws + L.slots), s.M1, (int*)(ws + L.misc) + 1, sp);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     mark(ev, 2, st);
@@ -1001,7 +1015,7 @@ static cudaError_t select_bm_t(const void* Q, const void* K, const float* pyr, i
     e = zero_counts(s, ws, L, st);  // the Top-K counts the kept leaves for the attention grouping
     if (e != cudaSuccess) return e;
     topk_kernel<G><<<unit_grid(s), 256, 0, st>>>(cand, (const float*)(ws + L.lse), idx, (float*)(ws + L.z2),
-                                                  (int32_t*)(ws + L.counts), s.M1, sp);
+                                                  (int32_t*)(ws + L.counts), (int32_t*)(ws + L.slots), s.M1, sp);
     e = cudaGetLastError();
     mark(ev, 5, st);
     return e;

@@ -6,10 +6,11 @@
 // then each ancestor as the mean of its existing children: O(C + L) rows.
 //
 // decode_kernel: the single-stage fused step, one CTA (8 warps) per
-// (b, kv-head). Warp 0 walks the internal levels with the query loaded once;
-// all warps then split the leaf scoring (exact LSE over raw keys) and, after
-// warp 0's final Top-K, split the attention over the kept blocks; partial
-// softmax states are merged through shared memory.
+// (b, kv-head). Warp 0 carries the walk's bookkeeping; at every scored level
+// all warps compute the child dot products together (one round of gathers
+// per level), all warps then split the leaf scoring (exact LSE over raw keys)
+// and, after warp 0's final Top-K, the attention over the kept blocks;
+// partial softmax states are merged through shared memory.
 #include "pisa_internal.h"
 #include "pisa_attn.cuh"
 
@@ -80,18 +81,28 @@ __global__ void __launch_bounds__(128) append_kernel(T* __restrict__ Kc, T* __re
     }
 }
 
+// CTAs per SM the decode kernel is sized for: with G <= 2 four CTAs of 8
+// warps fit (64 registers a thread), so a step of up to 4 * 148 (b, kv-head)
+// units runs in one wave.
+template <int G>
+constexpr int decode_min_blocks() { return G <= 2 ? 4 : (G <= 4 ? 2 : 1); }
+
 template <typename T, int D, int G>
-__global__ void __launch_bounds__(256) decode_kernel(const T* __restrict__ q_new, const T* __restrict__ Kc,
-                                                     const T* __restrict__ Vc, const float* __restrict__ pyr,
-                                                     const int32_t* __restrict__ pos, int32_t* __restrict__ idx,
-                                                     T* __restrict__ out, DecodeParams p) {
+__global__ void __launch_bounds__(256, decode_min_blocks<G>()) decode_kernel(
+    const T* __restrict__ q_new, const T* __restrict__ Kc, const T* __restrict__ Vc, const float* __restrict__ pyr,
+    const int32_t* __restrict__ pos, int32_t* __restrict__ idx, T* __restrict__ out, DecodeParams p) {
     constexpr int VD = D / 32;
     constexpr int NW = 8;
+    constexpr int RB = 32 / G;                  // rows per reduce-scatter batch
+    constexpr int ROWS_W = 64 / NW;             // child rows per warp at a scored level
+    constexpr int NRB = RB < ROWS_W ? RB : ROWS_W;
     extern __shared__ __align__(16) float dsm[];  // [NW][G][D] partial outputs
     __shared__ int s_cand[32];
+    __shared__ float s_dot[64][G];
     __shared__ float s_score[32];
     __shared__ int s_sel[32];
     __shared__ unsigned s_need;
+    __shared__ int s_level;
     __shared__ float s_m[NW][G], s_l[NW][G];
 
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -119,31 +130,93 @@ __global__ void __launch_bounds__(256) decode_kernel(const T* __restrict__ q_new
         w.load_q(qrow, p.qscale, lane);
     }
 
-    if (warp == 0) {
-        int cand = lane == 0 ? 0 : -1;
-        for (int l = p.geom.L; l >= 2; --l) {
-            const LevelState s = level_state(cand, l, p.C, n_keys, t, 1, F);
-            float score = -INFINITY;
-            if (s.n > p.K) {
+    // Internal levels. Warp 0 carries the walk (lane c = candidate c, valid
+    // candidates in ascending node order) and passes alone through the levels
+    // that need no dot products; at a scored level all warps compute the
+    // <= 64 child dots (8 rows each, loads in flight together) into s_dot.
+    int cand = lane == 0 ? 0 : -1;  // warp 0's walk state
+    int l = p.geom.L;
+    for (;;) {
+        if (warp == 0) {
+            unsigned need = 0;
+            for (; l >= 2; --l) {
+                const LevelState s = level_state(cand, l, p.C, n_keys, t, 1, F);
+                if (s.n <= p.K) {
+                    const int parent = compact_by_rank(cand, s.vmask, lane >> 1);
+                    cand = lane < 2 * s.n ? 2 * parent + (lane & 1) : -1;
+                    continue;
+                }
                 const unsigned fmask = __ballot_sync(kFull, s.forced);
-                if (__popc(fmask) < p.K)
-                    score = w.score_internal(cand, s.vmask & ~fmask, P + p.geom.off[l - 1] * D,
-                                             (int64_t)p.C << (l - 2), n_keys, lane);
+                if (__popc(fmask) >= p.K) {  // the forced nodes fill the budget
+                    int id = cand;
+                    const int kept = keep_topk_lane(id, s.forced ? INFINITY : -INFINITY, s.valid, p.K, lane);
+                    const int parent = __shfl_sync(kFull, id, lane >> 1);
+                    cand = lane < 2 * kept ? 2 * parent + (lane & 1) : -1;
+                    continue;
+                }
+                need = s.vmask & ~fmask;
+                break;
+            }
+            s_cand[lane] = cand;
+            if (lane == 0) {
+                s_level = l;
+                s_need = need;
+            }
+        }
+        __syncthreads();
+        const int lv = s_level;
+        if (lv < 2) break;
+        {
+            const unsigned need = s_need;
+            const int64_t span_child = (int64_t)p.C << (lv - 2);
+            const float* child_lvl = P + p.geom.off[lv - 1] * D;
+#pragma unroll
+            for (int r0 = warp * ROWS_W; r0 < warp * ROWS_W + ROWS_W; r0 += NRB) {
+                float v[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) v[i] = 0.f;
+#pragma unroll
+                for (int r = 0; r < NRB; ++r) {
+                    const int rho = r0 + r, c = rho >> 1;
+                    const int64_t child = 2 * (int64_t)s_cand[c] + (rho & 1);
+                    const bool ok = ((need >> c) & 1u) && child * span_child < n_keys;
+                    w.dots_into(v, r, child_lvl + (ok ? child : 0) * D, ok, lane);
+                }
+                const float z = reduce_scatter32(v, lane);  // lane = r * G + h
+                if (lane < NRB * G) s_dot[r0 + lane / G][lane % G] = z;
+            }
+        }
+        __syncthreads();
+        if (warp == 0) {  // scores (Eq.7, summed over the group: Eq.11) and the keep
+            const LevelState s = level_state(cand, l, p.C, n_keys, t, 1, F);
+            const bool mine = (s_need >> lane) & 1u;
+            float score = -INFINITY;
+            if (mine) {
+                const bool has1 = (2 * (int64_t)cand + 1) * ((int64_t)p.C << (l - 2)) < n_keys;
+                score = 0.f;
+#pragma unroll
+                for (int h = 0; h < G; ++h) {
+                    const float z0 = s_dot[2 * lane][h], z1 = has1 ? s_dot[2 * lane + 1][h] : -INFINITY;
+                    const float m = fmaxf(z0, z1);
+                    score += m + log2f(exp2f(z0 - m) + exp2f(z1 - m));
+                }
             }
             int id = cand;
-            const int kept = keep_topk(id, score, s, p.K, lane);
+            const int kept = keep_topk_lane(id, s.forced ? INFINITY : score, s.valid, p.K, lane);
             const int parent = __shfl_sync(kFull, id, lane >> 1);
             cand = lane < 2 * kept ? 2 * parent + (lane & 1) : -1;
+            --l;
         }
+    }
+
+    // leaves: warp 0 flags the candidates to score; exact LSE over raw keys
+    if (warp == 0) {
         const LevelState s = level_state(cand, 1, p.C, n_keys, t, 1, F);
         const unsigned fmask = __ballot_sync(kFull, s.forced);
-        s_cand[lane] = cand;
         s_score[lane] = -INFINITY;
         if (lane == 0) s_need = (s.n > p.K && __popc(fmask) < p.K) ? (s.vmask & ~fmask) : 0u;
     }
     __syncthreads();
-
-    // leaf scores, candidates spread over the warps
     {
         const unsigned need = s_need;
         for (int c = warp; c < 32; c += NW) {
@@ -155,14 +228,16 @@ __global__ void __launch_bounds__(256) decode_kernel(const T* __restrict__ q_new
     }
     __syncthreads();
 
-    if (warp == 0) {
-        const int cand = s_cand[lane];
+    if (warp == 0) {  // final Top-K: kept leaves come out in ascending order
         const LevelState s = level_state(cand, 1, p.C, n_keys, t, 1, F);
-        int id = cand;
-        const int kept = keep_topk(id, s_score[lane], s, p.K, lane);
-        int v = lane < kept ? id : 0x7fffffff;
-        warp_sort_asc(v, lane);
-        const int out_id = v == 0x7fffffff ? -1 : v;
+        int id = cand, kept;
+        if (s.n <= p.K) {
+            id = compact_by_rank(cand, s.vmask, lane);
+            kept = s.n;
+        } else {
+            kept = keep_topk_lane(id, s.forced ? INFINITY : s_score[lane], s.valid, p.K, lane);
+        }
+        const int out_id = lane < kept ? id : -1;
         if (lane < p.K) idx[unit * p.K + lane] = out_id;
         s_sel[lane] = lane < p.K ? out_id : -1;
     }
@@ -178,12 +253,12 @@ __global__ void __launch_bounds__(256) decode_kernel(const T* __restrict__ q_new
         const int64_t hi = min(lo + p.C, n_keys);
         if (lo < hi) acc.block(w, Kh, Vh, lo, hi, lane);
     }
-    float l = acc.lsum;
+    float lsum = acc.lsum;
 #pragma unroll
-    for (int o = G; o < 32; o <<= 1) l += __shfl_xor_sync(kFull, l, o);
+    for (int o = G; o < 32; o <<= 1) lsum += __shfl_xor_sync(kFull, lsum, o);
     if (lane < G) {
         s_m[warp][lane] = acc.m;
-        s_l[warp][lane] = l;
+        s_l[warp][lane] = lsum;
     }
 #pragma unroll
     for (int h = 0; h < G; ++h)

@@ -130,42 +130,4 @@ struct Walk4S {
     }
 };
 
-// Keep-set of a scored level without a sort: every lane counts the lanes that
-// rank before it (higher key, then lower index) with 31 independent shuffles,
-// so the keep decision has no long dependent chain. Keys: +inf forced, the
-// score otherwise, -inf for invalid lanes. Lanes 0..kept-1 of the result hold
-// the kept ids (in lane order of the kept lanes); returns kept.
-__device__ __forceinline__ int keep_topk_rank(int& id, float key, bool valid, int K, int lane) {
-    const int ix = valid ? id : 0x7fffffff;
-    int before = 0;
-#pragma unroll
-    for (int o = 1; o < 32; ++o) {
-        const float ok = __shfl_xor_sync(kFull, key, o);
-        const int oi = __shfl_xor_sync(kFull, ix, o);
-        before += ranks_before(ok, oi, key, ix) ? 1 : 0;
-    }
-    const unsigned kmask = __ballot_sync(kFull, valid && before < K);
-    const int kept = __popc(kmask);
-    int src = 0;
-#pragma unroll
-    for (int step = 16; step >= 1; step >>= 1) {
-        const int probe = src + step;
-        if (probe <= 31 && __popc(kmask & ((1u << probe) - 1u)) <= lane) src = probe;
-    }
-    id = __shfl_sync(kFull, id, src);
-    return kept;
-}
-
-// Lanes 0..n-1 of the result hold the valid candidates in lane order
-// (a gather by rank: the lane holding the r-th set bit of vmask).
-__device__ __forceinline__ int compact_by_rank(int cand, unsigned vmask, int rank) {
-    int src = 0;
-#pragma unroll
-    for (int step = 16; step >= 1; step >>= 1) {
-        const int probe = src + step;
-        if (__popc(vmask & ((1u << probe) - 1u)) <= rank && probe <= 31) src = probe;
-    }
-    return __shfl_sync(kFull, cand, src);
-}
-
 }  // namespace pisa

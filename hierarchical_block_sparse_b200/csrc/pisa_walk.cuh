@@ -170,4 +170,48 @@ __device__ __forceinline__ int keep_topk(int& id, float score, const LevelState&
     return s.n < K ? s.n : K;
 }
 
+// Keep-set of a scored level without a sort: every lane counts the lanes that
+// rank before it (higher key, then lower node index) with 31 independent
+// shuffles, so the keep decision has no long dependent chain. Keys: +inf
+// forced, the score otherwise. The walk keeps its valid candidates in
+// ascending node order across the lanes (the root starts in lane 0, and both
+// the gather by rank and this keep preserve lane order, so the children
+// 2p, 2p + 1 of ascending parents ascend too): "lower index" is "lower lane",
+// and only the key crosses lanes. Invalid lanes send NaN, which ranks before
+// no one. Lanes 0..kept-1 of the result hold the kept ids in lane order;
+// returns kept.
+__device__ __forceinline__ int keep_topk_lane(int& id, float key, bool valid, int K, int lane) {
+    const float kv = valid ? key : __int_as_float(0x7fc00000);
+    int before = 0;
+#pragma unroll
+    for (int o = 1; o < 32; ++o) {
+        const float ok = __shfl_xor_sync(kFull, kv, o);
+        const int hb = o >= 16 ? 4 : o >= 8 ? 3 : o >= 4 ? 2 : o >= 2 ? 1 : 0;
+        const bool lower = (lane >> hb) & 1;  // lane ^ o < lane
+        before += (ok > key || (ok == key && lower)) ? 1 : 0;
+    }
+    const unsigned kmask = __ballot_sync(kFull, valid && before < K);
+    const int kept = __popc(kmask);
+    int src = 0;
+#pragma unroll
+    for (int step = 16; step >= 1; step >>= 1) {
+        const int probe = src + step;
+        if (probe <= 31 && __popc(kmask & ((1u << probe) - 1u)) <= lane) src = probe;
+    }
+    id = __shfl_sync(kFull, id, src);
+    return kept;
+}
+
+// Lanes 0..n-1 of the result hold the valid candidates in lane order
+// (a gather by rank: the lane holding the r-th set bit of vmask).
+__device__ __forceinline__ int compact_by_rank(int cand, unsigned vmask, int rank) {
+    int src = 0;
+#pragma unroll
+    for (int step = 16; step >= 1; step >>= 1) {
+        const int probe = src + step;
+        if (__popc(vmask & ((1u << probe) - 1u)) <= rank && probe <= 31) src = probe;
+    }
+    return __shfl_sync(kFull, cand, src);
+}
+
 }  // namespace pisa

@@ -194,7 +194,7 @@ int pisa_forward_ws_events(const pisa_cfg *cfg, const void *Q, const void *K, co
  * on every GPU that loads the library until the process exits) instead of a
  * caller workspace; it calls no allocating routine.
  * - Problems whose selection scratch exceeds that size return
- *   PISA_E_SCRATCH_LIMIT (about 80 K query units B*Hkv*N for G = 1).
+ *   PISA_E_SCRATCH_LIMIT (about 73 K query units B*Hkv*N for G = 1).
  * - The first call on a device looks up the array's device address (once per
  *   device, that device current); make it before any stream capture.
  * - All calls on a device share the array and it keeps the previous call's
