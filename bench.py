@@ -525,6 +525,9 @@ def main():
 
 
 def bench_decode(w, dev, stream, steps: int = 8, batch: int = 0, cache: int = 0):
+    """Decode: every step appends one token per sequence and selects + attends
+    for it (pisa_decode_step, one launch). Also times the same step as the two
+    separate calls (pisa_pyramid_append, then pisa_decode)."""
     import torch
     from hierarchical_block_sparse_b200 import pisa
     from hierarchical_block_sparse_b200.workloads import decode_cache, decode_step_inputs
@@ -539,18 +542,24 @@ def bench_decode(w, dev, stream, steps: int = 8, batch: int = 0, cache: int = 0)
     pyr = torch.empty((B, w.Hkv, pisa.pisa_pyramid_rows(cfg), w.d), dtype=torch.float32, device=dev)
     pos = torch.full((B,), prefix, dtype=torch.int32, device=dev)
     pisa.pisa_build_pyramid_prefix(cfg, Kc, pos, pyr)
-    ins = [tuple(x.to(dev) for x in decode_step_inputs(w, s)) for s in range(steps + 3)]
+    ins = [tuple(x.to(dev) for x in decode_step_inputs(w, s)) for s in range(2 * steps + 3)]
     idx = torch.empty((B, w.Hkv, w.K), dtype=torch.int32, device=dev)
     o = torch.empty((B, w.Hq, w.d), dtype=Kc.dtype, device=dev)
     for s in range(3):
         q, k, v = ins[s]
-        pisa.pisa_pyramid_append(cfg, Kc, Vc, pyr, k, v, pos)
-        pisa.pisa_decode(cfg, q, Kc, Vc, pyr, pos, idx, o)
+        pisa.pisa_decode_step(cfg, q, k, v, Kc, Vc, pyr, pos, idx, o)
         pos += 1
     torch.cuda.synchronize()
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    evf = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
     for s in range(steps):
         q, k, v = ins[3 + s]
+        evf[s][0].record(stream)
+        pisa.pisa_decode_step(cfg, q, k, v, Kc, Vc, pyr, pos, idx, o)
+        evf[s][1].record(stream)
+        pos += 1
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    for s in range(steps):
+        q, k, v = ins[3 + steps + s]
         ev[s][0].record(stream)
         pisa.pisa_pyramid_append(cfg, Kc, Vc, pyr, k, v, pos)
         ev[s][1].record(stream)
@@ -558,23 +567,34 @@ def bench_decode(w, dev, stream, steps: int = 8, batch: int = 0, cache: int = 0)
         ev[s][2].record(stream)
         pos += 1
     torch.cuda.synchronize()
+    fused = float(np.mean([e[0].elapsed_time(e[1]) for e in evf])) * 1e3
     app = float(np.mean([e[0].elapsed_time(e[1]) for e in ev])) * 1e3
     dec = float(np.mean([e[1].elapsed_time(e[2]) for e in ev])) * 1e3
-    # gathered bytes per step (per sequence and KV head): the scored internal
-    # children summaries, the scored leaves' raw keys and the attended K and V rows
+    # compulsory bytes per step (per sequence and KV head): the scored levels'
+    # child summaries (fp32), the raw keys of every level-1 candidate (scored or
+    # forced), the attended values, the new q/k/v rows and the updated leaf
+    # and ancestor summaries. The kernel also reads the attended keys a second
+    # time (gathered bytes).
     internal, leafkeys, attended = walk_counts(prefix + 8, w.C, w.K, w.forced_mask)
     tlast = prefix + 4
     G = w.Hq // w.Hkv
     e = 2 if w.dtype == "bf16" else 4
-    per_unit = internal[tlast] * w.d * 4 + leafkeys[tlast] * w.d * e + 2 * attended[tlast] * w.d * e + \
-        (G * 2 * w.d * e)
+    L = 1
+    m = -(-cap // w.C)
+    while m > 1:
+        m = -(-m // 2)
+        L += 1
+    per_unit = internal[tlast] * w.d * 4 + (leafkeys[tlast] + walk_counts.forced_keys[tlast]) * w.d * e + \
+        attended[tlast] * w.d * e + (G + 2) * w.d * e + L * w.d * 4
     step_bytes = per_unit * B * w.Hkv
-    us = app + dec
+    gathered = step_bytes + attended[tlast] * w.d * e * B * w.Hkv
     pk = peaks()
     del Kc, Vc, pyr
-    return {"batch": B, "cache_keys": prefix, "us_per_step": us, "append_us": app, "decode_kernel_us": dec,
-            "tokens_per_s": B / (us / 1e6), "gathered_bytes_per_step": int(step_bytes),
-            "hbm_roofline_frac": step_bytes / (dec / 1e6) / (pk["hbm_gbs"] * 1e9)}
+    return {"batch": B, "cache_keys": prefix, "call": "pisa_decode_step", "us_per_step": fused,
+            "tokens_per_s": B / (fused / 1e6), "compulsory_bytes_per_step": int(step_bytes),
+            "gathered_bytes_per_step": int(gathered),
+            "hbm_roofline_frac": step_bytes / (fused / 1e6) / (pk["hbm_gbs"] * 1e9),
+            "split_calls_us": {"pisa_pyramid_append": app, "pisa_decode": dec, "total": app + dec}}
 
 
 def reference_arm(args, w, config, metric, unit):

@@ -339,8 +339,25 @@ int pisa_decode(const pisa_cfg* cfg, const void* q_new, const void* Kc, const vo
         return PISA_E_ALIGNMENT;
     Geom g;
     make_geom(cfg->N, cfg->C, &g);
-    return cuda_status(launch_decode(cfg->dtype, cfg->d, q_new, Kc, Vc, pyr, pos, idx, o, decode_params(cfg, g),
+    return cuda_status(launch_decode(cfg->dtype, cfg->d, q_new, const_cast<void*>(Kc), const_cast<void*>(Vc),
+                                     const_cast<float*>(pyr), pos, idx, o, nullptr, nullptr, decode_params(cfg, g),
                                      (cudaStream_t)stream));
+}
+
+int pisa_decode_step(const pisa_cfg* cfg, const void* q_new, const void* k_new, const void* v_new, void* Kc,
+                     void* Vc, float* pyr, const int32_t* pos, int32_t* idx, void* o, void* stream) {
+    int s = check_gpu(cfg);
+    if (s) return s;
+    if (cfg->causal != 1) return PISA_E_INVALID;
+    if (cfg->N == 0) return PISA_OK;
+    if (!q_new || !k_new || !v_new || !Kc || !Vc || !pyr || !pos || !idx || !o) return PISA_E_INVALID;
+    if (!aligned16(q_new) || !aligned16(k_new) || !aligned16(v_new) || !aligned16(Kc) || !aligned16(Vc) ||
+        !aligned16(pyr) || !aligned16(o))
+        return PISA_E_ALIGNMENT;
+    Geom g;
+    make_geom(cfg->N, cfg->C, &g);
+    return cuda_status(launch_decode(cfg->dtype, cfg->d, q_new, Kc, Vc, pyr, pos, idx, o, k_new, v_new,
+                                     decode_params(cfg, g), (cudaStream_t)stream));
 }
 
 const char* pisa_status_string(int status) {

@@ -62,7 +62,8 @@ cudaError_t launch_bsa(int dtype, int d, const void* Q, const float* pyr, int32_
                        cudaStream_t st);
 cudaError_t launch_append(int dtype, int d, void* Kc, void* Vc, float* pyr, const void* k_new, const void* v_new,
                           const int32_t* pos, const DecodeParams& p, cudaStream_t st);
-cudaError_t launch_decode(int dtype, int d, const void* q_new, const void* Kc, const void* Vc, const float* pyr,
-                          const int32_t* pos, int32_t* idx, void* o, const DecodeParams& p, cudaStream_t st);
+cudaError_t launch_decode(int dtype, int d, const void* q_new, void* Kc, void* Vc, float* pyr, const int32_t* pos,
+                          int32_t* idx, void* o, const void* k_new, const void* v_new, const DecodeParams& p,
+                          cudaStream_t st);
 
 }  // namespace pisa

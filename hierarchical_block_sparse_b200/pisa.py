@@ -81,6 +81,7 @@ def load(path: str | None = None):
             "pisa_build_pyramid_prefix": (ctypes.c_int, [cfgp, P, P, P, P]),
             "pisa_pyramid_append": (ctypes.c_int, [cfgp, P, P, P, P, P, P, P]),
             "pisa_decode": (ctypes.c_int, [cfgp, P, P, P, P, P, P, P, P]),
+            "pisa_decode_step": (ctypes.c_int, [cfgp, P, P, P, P, P, P, P, P, P, P]),
             "pisa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
             "pisa_version": (ctypes.c_char_p, []),
         }
@@ -242,6 +243,12 @@ def pisa_pyramid_append(cfg, Kc, Vc, pyr, k_new, v_new, pos):
 def pisa_decode(cfg, q_new, Kc, Vc, pyr, pos, idx, o):
     _check("pisa_decode", load().pisa_decode(ctypes.byref(cfg), _ptr(q_new), _ptr(Kc), _ptr(Vc), _ptr(pyr),
                                              _ptr(pos), _ptr(idx), _ptr(o), _stream()))
+
+
+def pisa_decode_step(cfg, q_new, k_new, v_new, Kc, Vc, pyr, pos, idx, o):
+    _check("pisa_decode_step", load().pisa_decode_step(ctypes.byref(cfg), _ptr(q_new), _ptr(k_new), _ptr(v_new),
+                                                       _ptr(Kc), _ptr(Vc), _ptr(pyr), _ptr(pos), _ptr(idx), _ptr(o),
+                                                       _stream()))
 
 
 def pisa_status_string(status: int) -> str:

@@ -231,6 +231,17 @@ int pisa_pyramid_append(const pisa_cfg *cfg, void *Kc, void *Vc, float *pyr,
 int pisa_decode(const pisa_cfg *cfg, const void *q_new, const void *Kc, const void *Vc,
                 const float *pyr, const int32_t *pos, int32_t *idx, void *o, void *stream);
 
+/* pisa_pyramid_append followed by pisa_decode, as one kernel launch: the whole
+ * decode step of the close reading's §5.3 (append the token, update the leaf
+ * and its ancestors, then select and attend for the new query). Same
+ * arguments, layouts and results as the two calls in sequence (up to fp32
+ * summation order in the updated summaries). The append reuses the step's
+ * shared memory and overlaps its first walk levels, which never read the
+ * rows it rewrites (the new token's leaf and its ancestors are forced nodes). */
+int pisa_decode_step(const pisa_cfg *cfg, const void *q_new, const void *k_new, const void *v_new,
+                     void *Kc, void *Vc, float *pyr, const int32_t *pos, int32_t *idx, void *o,
+                     void *stream);
+
 /* ---- misc --------------------------------------------------------------------- */
 
 /* Static English text for a status code (never NULL). */

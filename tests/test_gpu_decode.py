@@ -57,15 +57,28 @@ def _check_seq(w, cap, Khost, Vhost, pyr_gpu, n, q, idx_g, o_g, check_pyr=True):
     return exempt
 
 
-@pytest.mark.parametrize("G", [1, 2])
-def test_decode_steps_small(G):
-    w = Workload("dec_small", 120, B=1, Hq=2 * G, Hkv=2, N=0, d=128, C=64, K=8, decode_batch=3)
-    cap = 4096
+# (G, d, C, K, dtype, cap, prefixes): the decode kernel streams leaf blocks in
+# tiles of 16 KB of rows, so these cover a leaf in one tile, a leaf in two
+# scoring tiles (fp32 at d = 128; C = 128), several leaves' worth of rows per
+# tile (d = 64, small C), and group sizes up to 8.
+DECODE_SHAPES = [
+    (1, 128, 64, 8, "bf16", 4096, [1000, 2048, 3071]),
+    (2, 128, 64, 8, "bf16", 4096, [1000, 2048, 3071]),
+    (1, 64, 16, 4, "f32", 1024, [100, 512, 990]),
+    (1, 128, 64, 8, "f32", 4096, [700, 2048, 4000]),
+    (4, 64, 32, 8, "bf16", 2048, [333, 1024, 2000]),
+    (8, 128, 128, 4, "bf16", 4096, [1500, 2600, 4050]),
+]
+
+
+@pytest.mark.parametrize("fused", [False, True], ids=["append+decode", "decode_step"])
+@pytest.mark.parametrize("G,d,C,K,dtype,cap,prefix", DECODE_SHAPES)
+def test_decode_steps_small(G, d, C, K, dtype, cap, prefix, fused):
+    w = Workload("dec_small", 120, B=1, Hq=2 * G, Hkv=2, N=0, d=d, C=C, K=K, decode_batch=3, dtype=dtype)
     dev = torch.device("cuda", 0)
-    prefix = [1000, 2048, 3071]
-    Kc, Vc, Kp, Vp = decode_cache(w, cap, 3100, dev)
-    Khost = [decode_rows(Kp, s, 3100) for s in range(3)]
-    Vhost = [decode_rows(Vp, s, 3100) for s in range(3)]
+    Kc, Vc, Kp, Vp = decode_cache(w, cap, max(prefix) + 29, dev)
+    Khost = [decode_rows(Kp, s, max(prefix) + 29) for s in range(3)]
+    Vhost = [decode_rows(Vp, s, max(prefix) + 29) for s in range(3)]
     for s in range(3):  # zero the rows past each sequence's prefix
         Kc[s, :, prefix[s]:] = 0
         Vc[s, :, prefix[s]:] = 0
@@ -82,8 +95,11 @@ def test_decode_steps_small(G):
         q, k, v = decode_step_inputs(w, step, B=3)
         idx = torch.full((3, w.Hkv, w.K), -7, dtype=torch.int32, device=dev)
         o = torch.empty((3, w.Hq, w.d), dtype=q.dtype, device=dev)
-        pisa.pisa_pyramid_append(cfg, Kc, Vc, pyr, k.to(dev), v.to(dev), pos)
-        pisa.pisa_decode(cfg, q.to(dev), Kc, Vc, pyr, pos, idx, o)
+        if fused:  # one launch: append, then select and attend
+            pisa.pisa_decode_step(cfg, q.to(dev), k.to(dev), v.to(dev), Kc, Vc, pyr, pos, idx, o)
+        else:
+            pisa.pisa_pyramid_append(cfg, Kc, Vc, pyr, k.to(dev), v.to(dev), pos)
+            pisa.pisa_decode(cfg, q.to(dev), Kc, Vc, pyr, pos, idx, o)
         torch.cuda.synchronize()
         for s in range(3):
             n = int(pos[s])
@@ -119,7 +135,7 @@ def test_decode_out_of_range_positions():
 
 
 def test_decode_full_size_sampled():
-    # 64 sequences x 8 heads against 262144-key caches (bench launch shape)
+    # 64 sequences x 8 heads against 262144-key caches (the bench's fused step)
     w = WORKLOADS["mha8_n256k"]
     prefix = w.N
     cap = prefix + 64
@@ -134,8 +150,7 @@ def test_decode_full_size_sampled():
     idx = torch.full((B, w.Hkv, w.K), -7, dtype=torch.int32, device=dev)
     o = torch.empty((B, w.Hq, w.d), dtype=q.dtype, device=dev)
     pos = lens.clone()
-    pisa.pisa_pyramid_append(cfg, Kc, Vc, pyr, k.to(dev), v.to(dev), pos)
-    pisa.pisa_decode(cfg, q.to(dev), Kc, Vc, pyr, pos, idx, o)
+    pisa.pisa_decode_step(cfg, q.to(dev), k.to(dev), v.to(dev), Kc, Vc, pyr, pos, idx, o)  # bench launch
     torch.cuda.synchronize()
     assert int((idx == -7).sum()) == 0
     for s in (0, 17, 63):
