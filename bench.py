@@ -145,17 +145,18 @@ def source_sha(files):
     return h.hexdigest()[:16]
 
 
+_CS = "hierarchical_block_sparse_b200/csrc/"
+_BM = [_CS + "blockmajor.cu", _CS + "pisa_internal.h"]
 KERNEL_SOURCES = {
-    "stage1": ["hierarchical_block_sparse_b200/csrc/blockmajor.cu", "hierarchical_block_sparse_b200/csrc/pisa_walk.cuh",
-               "hierarchical_block_sparse_b200/csrc/pisa_device.cuh"],
-    "leaf_scores": ["hierarchical_block_sparse_b200/csrc/blockmajor.cu", "hierarchical_block_sparse_b200/csrc/tc.cuh"],
-    "attn_tiles": ["hierarchical_block_sparse_b200/csrc/blockmajor.cu", "hierarchical_block_sparse_b200/csrc/tc.cuh"],
-    "forced_tiles": ["hierarchical_block_sparse_b200/csrc/blockmajor.cu", "hierarchical_block_sparse_b200/csrc/tc.cuh"],
-    "pool": ["hierarchical_block_sparse_b200/csrc/pool.cu", "hierarchical_block_sparse_b200/csrc/pisa_device.cuh"],
-    "select": ["hierarchical_block_sparse_b200/csrc/select.cu", "hierarchical_block_sparse_b200/csrc/pisa_walk.cuh",
-               "hierarchical_block_sparse_b200/csrc/pisa_device.cuh"],
-    "attn": ["hierarchical_block_sparse_b200/csrc/attn.cu", "hierarchical_block_sparse_b200/csrc/pisa_attn.cuh",
-             "hierarchical_block_sparse_b200/csrc/pisa_walk.cuh", "hierarchical_block_sparse_b200/csrc/pisa_device.cuh"],
+    "stage1": _BM + [_CS + "pisa_stage1.cuh", _CS + "pisa_walk.cuh", _CS + "pisa_device.cuh"],
+    "leaf_scores": _BM + [_CS + "tc.cuh"],
+    "attn_tiles": _BM + [_CS + "tc.cuh"],
+    "forced_tiles": _BM + [_CS + "tc.cuh"],
+    "topk": _BM + [_CS + "pisa_walk.cuh", _CS + "pisa_device.cuh"],
+    "pool": [_CS + "pool.cu", _CS + "pisa_device.cuh"],
+    "select": [_CS + "select.cu", _CS + "pisa_walk.cuh", _CS + "pisa_device.cuh"],
+    "attn": [_CS + "attn.cu", _CS + "pisa_attn.cuh", _CS + "pisa_walk.cuh", _CS + "pisa_device.cuh"],
+    "decode": [_CS + "decode.cu", _CS + "tc.cuh", _CS + "pisa_walk.cuh", _CS + "pisa_device.cuh"],
 }
 
 

@@ -48,6 +48,9 @@ constexpr int kD = 128;      // head dimension handled by the tensor-core tiles
 // the 32-slot reduce-scatter walker otherwise. Levels with at most K
 // candidates keep them all (gather by rank); scored levels keep the forced
 // nodes and the best by (score, lower index) through an all-pairs rank.
+#ifndef PISA_STAGE1_CARVEOUT
+#define PISA_STAGE1_CARVEOUT (-1)  // percent of the shared-memory maximum; -1: the driver's choice
+#endif
 #ifndef PISA_STAGE1_MINBLOCKS
 #define PISA_STAGE1_MINBLOCKS 4  // 64 registers: 32 warps per SM hide the gathers' latency
 #endif
@@ -1001,6 +1004,12 @@ static cudaError_t select_bm_t(const void* Q, const void* K, const float* pyr, i
     e = zero_counts(s, ws, L, st);
     if (e != cudaSuccess) return e;
     using W = typename std::conditional<(G <= 2), Walk4S<(G <= 2 ? G : 1)>, Walk<__nv_bfloat16, kD, G>>::type;
+#if PISA_STAGE1_CARVEOUT >= 0
+    // the walk lives on L1 hits of pyramid rows and needs little shared memory
+    e = cudaFuncSetAttribute(stage1_kernel<G, W>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             PISA_STAGE1_CARVEOUT);
+    if (e != cudaSuccess) return e;
+#endif
     stage1_kernel<G, W><<<unit_grid(s), 256, 0, st>>>((const __nv_bfloat16*)Q, pyr, cand, (int32_t*)(ws + L.counts),
                                                       (int32_t*)(ws + L.slots), s.M1, (int*)(ws + L.misc) + 1, sp);
     e = cudaGetLastError();
