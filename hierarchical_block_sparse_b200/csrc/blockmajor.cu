@@ -41,6 +41,7 @@ constexpr int kSlots = 32;   // level-1 candidates per query (2K <= 32)
 constexpr int kPairs = 16;   // bucket slots recorded per query: sibling pairs, or kept leaves (K <= 16)
 constexpr int kBlk = 64;     // leaf size handled by the tensor-core tiles
 constexpr int kD = 128;      // head dimension handled by the tensor-core tiles
+constexpr int kORowStride = kD * 4 + 16;  // staged fp32 output row: 16-byte pad keeps the row writes conflict-free
 
 // ------------------------------------------------------------------ stage 1 ----
 
@@ -604,23 +605,34 @@ __global__ void __launch_bounds__(128) attn_tile_kernel(const __nv_bfloat16* __r
         if (!ok) break;
         tc::tc_fence_after();
         {
+            // Row tid of the output tile is staged in shared memory (the tile's
+            // buffers are free once the PV product has landed) and added to the
+            // accumulator with one 512-byte bulk reduction: whole-line
+            // operations at L2 instead of 32 scattered 16-byte ones.
             const int t = tr.t[tid];
-            float* dst = t >= 0 ? oacc + (((b * p.Hq + (int64_t)kvh * G + (tid % G)) * p.N) + t) * kD : nullptr;
             const uint32_t taddr = tmem_o + ((uint32_t)(warp * 32) << 16);
+            uint8_t* srow = dsm + tid * kORowStride;
 #pragma unroll
             for (int part = 0; part < 4; ++part) {
                 float v[32];
                 tc::tmem_ld32(taddr + part * 32, v);
                 tc::tmem_ld_wait();
-                if (dst) {
 #pragma unroll
-                    for (int q = 0; q < 32; q += 4) tc::red_add_v4(dst + part * 32 + q, v[q], v[q + 1], v[q + 2], v[q + 3]);
-                }
+                for (int q = 0; q < 32; q += 4)
+                    *reinterpret_cast<float4*>(srow + (part * 32 + q) * 4) = make_float4(v[q], v[q + 1], v[q + 2], v[q + 3]);
+            }
+            if (t >= 0) {
+                tc::fence_async_smem();
+                tc::bulk_reduce_add_f32(oacc + (((b * p.Hq + (int64_t)kvh * G + (tid % G)) * p.N) + t) * kD,
+                                        tc::smem_u32(srow), kD * 4);
+                tc::bulk_commit();
             }
         }
         tc::tc_fence_before();
+        tc::bulk_wait_read_all();  // the staged row has been read: the buffers may be refilled
         __syncthreads();
     }
+    tc::bulk_wait_all();
     __syncthreads();
     if (warp == 0) {
         tc::tc_fence_after();
@@ -978,6 +990,7 @@ static int sm_count() {
 }
 
 constexpr size_t kAttnSmem = 4 * 16384 + 16384;
+static_assert(128 * kORowStride <= kAttnSmem, "the staged output tile fits in the attention tile's buffers");
 
 template <int G, bool PAIR>
 static cudaError_t leaf_scores(const void* Q, const void* K, const SelectParams& sp, const BmShape& s, uint8_t* ws,
