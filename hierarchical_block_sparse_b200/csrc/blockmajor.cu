@@ -854,10 +854,12 @@ __global__ void __launch_bounds__(128) forced_tile_kernel(const __nv_bfloat16* _
             tc::tc_fence_after();
         }
         if (!ok) break;
-        // initial value of the output accumulator for these rows
+        // initial value of the output accumulator for these rows: row tid is
+        // staged in the tile's (now free) shared memory and stored with one
+        // 512-byte bulk copy
         {
-            float* dst = row_ok ? oacc + (((b * p.Hq + (int64_t)kvh * G + (tid % G)) * p.N) + t) * kD : nullptr;
             const uint32_t taddr = tmem_o + ((uint32_t)(warp * 32) << 16);
+            uint8_t* srow = dsm + tid * kORowStride;
 #pragma unroll
             for (int part = 0; part < 4; ++part) {
                 float v[32];
@@ -868,16 +870,22 @@ __global__ void __launch_bounds__(128) forced_tile_kernel(const __nv_bfloat16* _
 #pragma unroll
                     for (int q = 0; q < 32; ++q) v[q] = 0.f;
                 }
-                if (dst) {
 #pragma unroll
-                    for (int q = 0; q < 32; q += 4)
-                        *reinterpret_cast<float4*>(dst + part * 32 + q) = make_float4(v[q], v[q + 1], v[q + 2], v[q + 3]);
-                }
+                for (int q = 0; q < 32; q += 4)
+                    *reinterpret_cast<float4*>(srow + (part * 32 + q) * 4) = make_float4(v[q], v[q + 1], v[q + 2], v[q + 3]);
+            }
+            if (row_ok) {
+                tc::fence_async_smem();
+                tc::bulk_store(oacc + (((b * p.Hq + (int64_t)kvh * G + (tid % G)) * p.N) + t) * kD, tc::smem_u32(srow),
+                               kD * 4);
+                tc::bulk_commit();
             }
         }
         tc::tc_fence_before();
+        tc::bulk_wait_read_all();  // the staged row has been read: the buffers may be refilled
         __syncthreads();
     }
+    tc::bulk_wait_all();
     __syncthreads();
     if (warp == 0) {
         tc::tc_fence_after();
