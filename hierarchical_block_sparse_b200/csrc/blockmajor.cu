@@ -446,56 +446,79 @@ __global__ void __launch_bounds__(128) leaf_score_kernel(const __nv_bfloat16* __
 
 // ----------------------------------------------------------- final Top-K ----
 
-// One warp per (b, kv-head, t): lane = candidate slot. Keeps forced + best by
-// the LSE summed over the group (ties: lower leaf), writes idx sorted and the
+// One warp per kTopkQ consecutive positions of one (b, kv-head); lane =
+// candidate slot. Keeps forced + best by the LSE summed over the group (ties:
+// lower leaf: valid candidates arrive in ascending order, so the lane order is
+// the index order and the kept leaves come out sorted), writes idx and the
 // per-head partial normaliser z2[unit * G + h] = log2 sum 2^lse over the kept
-// leaves that are not forced (forced_tile_kernel adds the forced ones).
+// leaves that are not forced (forced_tile_kernel adds the forced ones). The
+// slot-returning atomics that place each kept free leaf in its attention
+// bucket are issued for all of the warp's positions together, so their round
+// trips overlap.
+constexpr int kTopkQ = 4;
+
 template <int G>
 __global__ void __launch_bounds__(256) topk_kernel(const int32_t* __restrict__ cand, const float* __restrict__ lse,
                                                    int32_t* __restrict__ idx, float* __restrict__ z2,
                                                    int32_t* __restrict__ counts, int32_t* __restrict__ slots,
                                                    int64_t M1, SelectParams p) {
     const int lane = threadIdx.x & 31;
-    const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-    if (t >= p.N) return;
+    const int t0 = (blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * kTopkQ;
+    if (t0 >= p.N) return;
     const int64_t bh = blockIdx.y;
-    const int64_t unit = bh * p.N + t;
-    const Forced F(t, p.C, p.causal, p.forced_mask);
-    const int leaf = cand[unit * kSlots + lane];
-    float l2[G];
-    float score = 0.f;
+    int out_leaf[kTopkQ];  // lane < K: the lane-th kept leaf that needs a bucket slot, else -1
 #pragma unroll
-    for (int h = 0; h < G; ++h) {
-        l2[h] = leaf >= 0 ? lse[(unit * kSlots + lane) * G + h] : -INFINITY;
-        score += l2[h];
+    for (int i = 0; i < kTopkQ; ++i) {
+        out_leaf[i] = -1;
+        const int t = t0 + i;
+        if (t >= p.N) continue;
+        const int64_t unit = bh * p.N + t;
+        const Forced F(t, p.C, p.causal, p.forced_mask);
+        const int leaf = cand[unit * kSlots + lane];
+        float l2[G];
+        float score = 0.f;
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+            l2[h] = leaf >= 0 ? lse[(unit * kSlots + lane) * G + h] : -INFINITY;
+            score += l2[h];
+        }
+        const bool valid = leaf >= 0;
+        const bool forced = valid && F.has(leaf, 1);
+        const unsigned vmask = __ballot_sync(kFull, valid);
+        int id = leaf;
+        unsigned kmask;
+        int kept;
+        if (__popc(vmask) <= p.K) {
+            kmask = vmask;
+            kept = __popc(vmask);
+            id = compact_by_rank(leaf, vmask, lane);
+        } else {
+            kept = keep_topk_lane(id, forced ? INFINITY : score, valid, p.K, lane, &kmask);
+        }
+        const bool mine = ((kmask >> lane) & 1u) && !forced;
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+            const float x = mine ? l2[h] : -INFINITY;
+            float m = x;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, o));
+            float e = mine ? exp2f(x - m) : 0.f;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) e += __shfl_xor_sync(kFull, e, o);
+            if (lane == 0) z2[unit * G + h] = m + log2f(e);
+        }
+        const int v = lane < kept ? id : -1;
+        if (lane < p.K) idx[unit * p.K + lane] = v;
+        if (lane < p.K && v >= 0 && !F.has(v, 1)) out_leaf[i] = v;
     }
-    LevelState s;
-    s.valid = leaf >= 0;
-    s.forced = s.valid && F.has(leaf, 1);
-    s.vmask = __ballot_sync(kFull, s.valid);
-    s.n = __popc(s.vmask);
-    int id = leaf;
-    const int kept = keep_topk(id, s.valid ? score : -INFINITY, s, p.K, lane);
-    bool mine = false;
-    for (int j = 0; j < kept; ++j) mine |= (__shfl_sync(kFull, id, j) == leaf) && s.valid;
-    mine = mine && !s.forced;
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-        const float x = mine ? l2[h] : -INFINITY;
-        float m = x;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, o));
-        float e = mine ? exp2f(x - m) : 0.f;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) e += __shfl_xor_sync(kFull, e, o);
-        if (lane == 0) z2[unit * G + h] = m + log2f(e);
-    }
-    int v = lane < kept ? id : 0x7fffffff;
-    warp_sort_asc(v, lane);
-    if (lane < p.K) idx[unit * p.K + lane] = v == 0x7fffffff ? -1 : v;
     // bucket count (and slot) of the attention grouping, by position in idx
-    if (lane < p.K && v != 0x7fffffff && !F.has(v, 1))
-        slots[unit * kPairs + lane] = atomicAdd(&counts[bh * M1 + v], 1);
+    int slot[kTopkQ];
+#pragma unroll
+    for (int i = 0; i < kTopkQ; ++i)
+        slot[i] = out_leaf[i] >= 0 ? atomicAdd(&counts[bh * M1 + out_leaf[i]], 1) : 0;
+#pragma unroll
+    for (int i = 0; i < kTopkQ; ++i)
+        if (out_leaf[i] >= 0) slots[(bh * p.N + t0 + i) * kPairs + lane] = slot[i];
 }
 
 // ------------------------------------------------------ attention tiles ----
@@ -514,12 +537,14 @@ __global__ void __launch_bounds__(128) attn_tile_kernel(const __nv_bfloat16* __r
     uint8_t* sA = dsm;                 // 32 KB gathered Q rows
     uint8_t* sK = dsm + 32768;         // 16 KB key block
     uint8_t* sV = dsm + 49152;         // 16 KB value block (MN-major)
-    uint8_t* sP = dsm + 65536;         // 16 KB probabilities (K-major)
+    uint8_t* sP = sK;                  // 16 KB probabilities (K-major), over the keys once S has landed
     __shared__ TileRows tr;
     __shared__ __align__(8) uint64_t mbar;
     __shared__ uint32_t tmem_base;
     const int tid = threadIdx.x, warp = tid >> 5;
-    if (warp == 0) tc::tmem_alloc(&tmem_base, 256);
+    // S (64 columns) and O (128) share one 128-column allocation: S is read
+    // into registers before the PV product starts, and O starts fresh per tile
+    if (warp == 0) tc::tmem_alloc(&tmem_base, 128);
     if (tid == 0) {
         tc::mbar_init(&mbar, 1);
         tc::fence_mbar_init();
@@ -527,7 +552,7 @@ __global__ void __launch_bounds__(128) attn_tile_kernel(const __nv_bfloat16* __r
     tc::tc_fence_before();
     __syncthreads();
     tc::tc_fence_after();
-    const uint32_t tmem_s = tmem_base, tmem_o = tmem_base + 128;
+    const uint32_t tmem_s = tmem_base, tmem_o = tmem_base;
     const uint32_t a_smem = tc::smem_u32(sA), k_smem = tc::smem_u32(sK), v_smem = tc::smem_u32(sV),
                    p_smem = tc::smem_u32(sP);
     const int ntiles = min(*ntiles_ptr, p.max_tiles);
@@ -636,7 +661,7 @@ __global__ void __launch_bounds__(128) attn_tile_kernel(const __nv_bfloat16* __r
     __syncthreads();
     if (warp == 0) {
         tc::tc_fence_after();
-        tc::tmem_dealloc(tmem_base, 256);
+        tc::tmem_dealloc(tmem_base, 128);
     }
 }
 
@@ -709,7 +734,7 @@ __global__ void __launch_bounds__(128) forced_tile_kernel(const __nv_bfloat16* _
     uint8_t* sA = dsm;          // 32 KB query rows
     uint8_t* sK = dsm + 32768;  // 16 KB key block
     uint8_t* sV = dsm + 49152;  // 16 KB value block (MN-major)
-    uint8_t* sP = dsm + 65536;  // 16 KB probabilities
+    uint8_t* sP = sK;           // 16 KB probabilities, over the keys once S has landed
     __shared__ TileRows tr;
     __shared__ __align__(8) uint64_t mbar;
     __shared__ uint32_t tmem_base;
@@ -997,8 +1022,11 @@ static int sm_count() {
     return n;
 }
 
-constexpr size_t kAttnSmem = 4 * 16384 + 16384;
+// Q 32 KB + K (then P) 16 KB + V 16 KB, rounded up so that the staged output
+// tile fits: three CTAs per SM
+constexpr size_t kAttnSmem = 72 * 1024;
 static_assert(128 * kORowStride <= kAttnSmem, "the staged output tile fits in the attention tile's buffers");
+constexpr int kAttnCtasPerSm = 3;
 
 template <int G, bool PAIR>
 static cudaError_t leaf_scores(const void* Q, const void* K, const SelectParams& sp, const BmShape& s, uint8_t* ws,
@@ -1044,8 +1072,9 @@ static cudaError_t select_bm_t(const void* Q, const void* K, const float* pyr, i
     mark(ev, 4, st);
     e = zero_counts(s, ws, L, st);  // the Top-K counts the kept leaves for the attention grouping
     if (e != cudaSuccess) return e;
-    topk_kernel<G><<<unit_grid(s), 256, 0, st>>>(cand, (const float*)(ws + L.lse), idx, (float*)(ws + L.z2),
-                                                  (int32_t*)(ws + L.counts), (int32_t*)(ws + L.slots), s.M1, sp);
+    const dim3 topk_grid((unsigned)((s.N + 8 * kTopkQ - 1) / (8 * kTopkQ)), (unsigned)(s.B * s.Hkv));
+    topk_kernel<G><<<topk_grid, 256, 0, st>>>(cand, (const float*)(ws + L.lse), idx, (float*)(ws + L.z2),
+                                              (int32_t*)(ws + L.counts), (int32_t*)(ws + L.slots), s.M1, sp);
     e = cudaGetLastError();
     mark(ev, 5, st);
     return e;
@@ -1084,7 +1113,9 @@ static cudaError_t attn_bm_t(const void* Q, const void* K, const void* V, const 
         e = cudaFuncSetAttribute(fk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kAttnSmem);
         if (e != cudaSuccess) return e;
         const int64_t ntiles = (int64_t)s.B * s.Hkv * fp.tiles_per_head;
-        const int grid = (int)(ntiles < (int64_t)sm_count() * 2 ? ntiles : (int64_t)sm_count() * 2);
+        // 256 TMEM columns each (O accumulates over the leaves while S is recomputed): two per SM
+        const int64_t slots = (int64_t)sm_count() * 2;
+        const int grid = (int)(ntiles < slots ? ntiles : slots);
         fk<<<grid, 128, kAttnSmem, st>>>((const __nv_bfloat16*)Q, (const __nv_bfloat16*)K, (const __nv_bfloat16*)V,
                                          idx, (float*)(ws + L.z2), oacc, (int*)(ws + L.misc) + 1, fp);
         e = cudaGetLastError();
@@ -1095,7 +1126,7 @@ static cudaError_t attn_bm_t(const void* Q, const void* K, const void* V, const 
     auto kern = attn_tile_kernel<G>;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kAttnSmem);
     if (e != cudaSuccess) return e;
-    kern<<<sm_count() * 2, 128, kAttnSmem, st>>>((const __nv_bfloat16*)Q, (const __nv_bfloat16*)K,
+    kern<<<sm_count() * kAttnCtasPerSm, 128, kAttnSmem, st>>>((const __nv_bfloat16*)Q, (const __nv_bfloat16*)K,
                                                  (const __nv_bfloat16*)V, (const int4*)(ws + L.tiles),
                                                  (const int32_t*)(ws + L.misc), (const uint32_t*)(ws + L.entries),
                                                  (const float*)(ws + L.z2), oacc, (int*)(ws + L.misc) + 1, tp);

@@ -50,21 +50,24 @@ struct Walk4S {
     __device__ __forceinline__ float score_internal(int cand, unsigned need, const float* child_lvl,
                                                     int64_t span_child, int64_t n_keys, int lane) const {
         const int g = lane >> 2, j = lane & 3;
-        int off[8];    // row offsets (floats) of the 8 rows, chunk j
-        bool okr[8];
+        int cbase[4];      // first-child row offset (floats) of the group's 4 candidates, chunk j
+        unsigned okm = 0;  // bit r: row r of the group exists and is wanted
 #pragma unroll
         for (int jj = 0; jj < 4; ++jj) {
             const int c = 4 * g + jj;
             const int cc = __shfl_sync(kFull, cand, c);
             const bool want = (need >> c) & 1u;
-#pragma unroll
-            for (int child = 0; child < 2; ++child) {
-                const int64_t row = 2 * (int64_t)cc + child;
-                const bool ok = want && row * span_child < n_keys;
-                okr[2 * jj + child] = ok;
-                off[2 * jj + child] = (int)((ok ? row : 0) * D) + j * kChunk;
-            }
+            const int64_t row0 = 2 * (int64_t)cc;
+            const bool ok0 = want && row0 * span_child < n_keys;
+            const bool ok1 = want && (row0 + 1) * span_child < n_keys;
+            okm |= (ok0 ? 1u : 0u) << (2 * jj);
+            okm |= (ok1 ? 1u : 0u) << (2 * jj + 1);
+            cbase[jj] = (int)((ok0 ? row0 : 0) * D) + j * kChunk;
         }
+        // row r of the group: child r & 1 of candidate r >> 1 (a row that does
+        // not exist reads an existing one; its dot is discarded)
+        auto row_off = [&](int r) { return cbase[r >> 1] + ((((okm >> r) & 1u) && (r & 1)) ? D : 0); };
+        auto row_ok = [&](int r) { return ((okm >> r) & 1u) != 0; };
         // two interleaved partial sums per (row, head), packed fp32x2 FMAs
         float2 acc[8 * G];
 #pragma unroll
@@ -81,7 +84,7 @@ struct Walk4S {
 #pragma unroll
             for (int r = 0; r < 8; ++r) {
                 float x[8];
-                ldg_nc_v8(child_lvl + off[r] + 4 * kChunk * k, x);
+                ldg_nc_v8(child_lvl + row_off(r) + 4 * kChunk * k, x);
 #pragma unroll
                 for (int h = 0; h < G; ++h) {
                     float2 a = acc[r * G + h];
@@ -97,7 +100,7 @@ struct Walk4S {
 #pragma unroll
         for (int r = 0; r < 8; ++r)
 #pragma unroll
-            for (int h = 0; h < G; ++h) part[r * G + h] = okr[r] ? acc[r * G + h].x + acc[r * G + h].y : 0.f;
+            for (int h = 0; h < G; ++h) part[r * G + h] = row_ok(r) ? acc[r * G + h].x + acc[r * G + h].y : 0.f;
         constexpr int R = 2 * G;
         {
             const bool hi = (lane & 2) != 0;

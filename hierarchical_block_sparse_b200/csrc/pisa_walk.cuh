@@ -179,8 +179,9 @@ __device__ __forceinline__ int keep_topk(int& id, float score, const LevelState&
 // 2p, 2p + 1 of ascending parents ascend too): "lower index" is "lower lane",
 // and only the key crosses lanes. Invalid lanes send NaN, which ranks before
 // no one. Lanes 0..kept-1 of the result hold the kept ids in lane order;
-// returns kept.
-__device__ __forceinline__ int keep_topk_lane(int& id, float key, bool valid, int K, int lane) {
+// returns kept (and, if asked, the mask of kept candidate lanes).
+__device__ __forceinline__ int keep_topk_lane(int& id, float key, bool valid, int K, int lane,
+                                              unsigned* kmask_out = nullptr) {
     const float kv = valid ? key : __int_as_float(0x7fc00000);
     int before = 0;
 #pragma unroll
@@ -191,6 +192,7 @@ __device__ __forceinline__ int keep_topk_lane(int& id, float key, bool valid, in
         before += (ok > key || (ok == key && lower)) ? 1 : 0;
     }
     const unsigned kmask = __ballot_sync(kFull, valid && before < K);
+    if (kmask_out) *kmask_out = kmask;  // bit c: candidate lane c is kept
     const int kept = __popc(kmask);
     int src = 0;
 #pragma unroll
