@@ -151,53 +151,108 @@ __global__ void bucket_count_kernel(const int32_t* __restrict__ src, GroupParams
     if (leaf >= 0) slots[unit * kPairs + lane] = atomicAdd(&counts[bh * g.M1 + leaf], 1);
 }
 
-// single CTA: exclusive scan of all bucket counts into entry offsets, and the
-// tile list (b*Hkv + kvh, leaf, first entry, entries) of every bucket.
-__global__ void __launch_bounds__(1024) bucket_scan_kernel(const int32_t* __restrict__ counts, int64_t nbuckets,
-                                                           int64_t M1, int per_tile, int N, int32_t* __restrict__ offsets,
-                                                           int4* __restrict__ tiles, int32_t* __restrict__ ntiles,
-                                                           int* __restrict__ err) {
-    __shared__ long long s_e[1024], s_t[1024];
-    const int tid = threadIdx.x;
-    const int64_t per = (nbuckets + 1023) / 1024;
-    const int64_t lo = tid * per, hi = min(lo + per, nbuckets);
-    // self-check: a bucket holds at most one entry per query position
-    auto count_of = [&](int64_t i) {
-        const int c = counts[i];
-        if (c < 0 || c > N) {
-            atomicCAS(err, 0, 11);
-            return 0;
+// Exclusive scan of the bucket counts into entry offsets, and the tile list
+// (b*Hkv + kvh, leaf, first entry, entries) of every bucket, in two passes
+// over blocks of kScanBlock buckets: per-block totals, then each block adds
+// the totals of the blocks before it and scans its own buckets.
+constexpr int kScanBlock = 1024;
+
+// self-check: a bucket holds at most one entry per query position
+__device__ __forceinline__ int bucket_count(const int32_t* counts, int64_t i, int64_t nbuckets, int N, int* err) {
+    if (i >= nbuckets) return 0;
+    const int c = counts[i];
+    if (c < 0 || c > N) {
+        if (err) atomicCAS(err, 0, 11);
+        return 0;
+    }
+    return c;
+}
+
+// inclusive scan of (a, b) over the block's 1024 threads
+__device__ __forceinline__ void block_scan2(long long& a, long long& b, long long* s_a, long long* s_b) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const long long xa = __shfl_up_sync(kFull, a, o), xb = __shfl_up_sync(kFull, b, o);
+        if (lane >= o) {
+            a += xa;
+            b += xb;
         }
-        return c;
-    };
-    long long e = 0, tt = 0;
-    for (int64_t i = lo; i < hi; ++i) {
-        const int c = count_of(i);
-        e += c;
-        tt += (c + per_tile - 1) / per_tile;
     }
-    s_e[tid] = e;
-    s_t[tid] = tt;
+    if (lane == 31) {
+        s_a[warp] = a;
+        s_b[warp] = b;
+    }
     __syncthreads();
-    for (int off = 1; off < 1024; off <<= 1) {  // inclusive Hillis-Steele scan
-        long long ve = tid >= off ? s_e[tid - off] : 0, vt = tid >= off ? s_t[tid - off] : 0;
-        __syncthreads();
-        s_e[tid] += ve;
-        s_t[tid] += vt;
-        __syncthreads();
+    if (warp == 0) {
+        long long wa = s_a[lane], wb = s_b[lane];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const long long xa = __shfl_up_sync(kFull, wa, o), xb = __shfl_up_sync(kFull, wb, o);
+            if (lane >= o) {
+                wa += xa;
+                wb += xb;
+            }
+        }
+        s_a[lane] = wa;  // inclusive totals of warps 0..lane
+        s_b[lane] = wb;
     }
-    long long be = s_e[tid] - e, bt = s_t[tid] - tt;
-    for (int64_t i = lo; i < hi; ++i) {
-        const int c = count_of(i);
+    __syncthreads();
+    if (warp > 0) {
+        a += s_a[warp - 1];
+        b += s_b[warp - 1];
+    }
+}
+
+__global__ void __launch_bounds__(kScanBlock) bucket_total_kernel(const int32_t* __restrict__ counts,
+                                                                 int64_t nbuckets, int per_tile, int N,
+                                                                 longlong2* __restrict__ bsum, int* __restrict__ err) {
+    __shared__ long long s_a[32], s_b[32];
+    const int c = bucket_count(counts, (int64_t)blockIdx.x * kScanBlock + threadIdx.x, nbuckets, N, err);
+    long long e = c, t = (c + per_tile - 1) / per_tile;
+    block_scan2(e, t, s_a, s_b);
+    if (threadIdx.x == kScanBlock - 1) bsum[blockIdx.x] = make_longlong2(e, t);
+}
+
+__global__ void __launch_bounds__(kScanBlock) bucket_place_kernel(const int32_t* __restrict__ counts,
+                                                                 int64_t nbuckets, int64_t M1, int per_tile, int N,
+                                                                 const longlong2* __restrict__ bsum,
+                                                                 int32_t* __restrict__ offsets,
+                                                                 int4* __restrict__ tiles,
+                                                                 int32_t* __restrict__ ntiles) {
+    __shared__ long long s_a[32], s_b[32];
+    __shared__ long long s_pre[2];
+    // entries and tiles of the blocks before this one
+    long long pe = 0, pt = 0;
+    for (int j = threadIdx.x; j < (int)blockIdx.x; j += kScanBlock) {
+        pe += bsum[j].x;
+        pt += bsum[j].y;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        pe += __shfl_xor_sync(kFull, pe, o);
+        pt += __shfl_xor_sync(kFull, pt, o);
+    }
+    if (threadIdx.x == 0) s_pre[0] = s_pre[1] = 0;
+    __syncthreads();
+    if ((threadIdx.x & 31) == 0) {
+        atomicAdd(reinterpret_cast<unsigned long long*>(&s_pre[0]), (unsigned long long)pe);
+        atomicAdd(reinterpret_cast<unsigned long long*>(&s_pre[1]), (unsigned long long)pt);
+    }
+    __syncthreads();
+    const int64_t i = (int64_t)blockIdx.x * kScanBlock + threadIdx.x;
+    const int c = bucket_count(counts, i, nbuckets, N, nullptr);
+    const int nt = (c + per_tile - 1) / per_tile;
+    long long e = c, t = nt;
+    block_scan2(e, t, s_a, s_b);
+    const long long be = s_pre[0] + e - c, bt = s_pre[1] + t - nt;  // exclusive
+    if (i < nbuckets) {
         offsets[i] = (int32_t)be;
-        const int nt = (c + per_tile - 1) / per_tile;
         for (int j = 0; j < nt; ++j)
             tiles[bt + j] = make_int4((int)(i / M1), (int)(i % M1), (int)(be + (int64_t)j * per_tile),
                                       min(per_tile, c - j * per_tile));
-        be += c;
-        bt += nt;
     }
-    if (tid == 1023) *ntiles = (int32_t)s_t[1023];
+    if (blockIdx.x == gridDim.x - 1 && threadIdx.x == kScanBlock - 1) *ntiles = (int32_t)(s_pre[1] + t);
 }
 
 // one warp per query position: write (t << 5 | slot) into each bucket
@@ -467,6 +522,16 @@ __global__ void __launch_bounds__(256) topk_kernel(const int32_t* __restrict__ c
     if (t0 >= p.N) return;
     const int64_t bh = blockIdx.y;
     int out_leaf[kTopkQ];  // lane < K: the lane-th kept leaf that needs a bucket slot, else -1
+    // all positions' candidates and LSEs are loaded first (independent requests in flight)
+    int leaves[kTopkQ];
+    float l2s[kTopkQ][G];
+#pragma unroll
+    for (int i = 0; i < kTopkQ; ++i) {
+        const int64_t unit = bh * p.N + t0 + i;
+        leaves[i] = t0 + i < p.N ? cand[unit * kSlots + lane] : -1;
+#pragma unroll
+        for (int h = 0; h < G; ++h) l2s[i][h] = t0 + i < p.N ? lse[(unit * kSlots + lane) * G + h] : -INFINITY;
+    }
 #pragma unroll
     for (int i = 0; i < kTopkQ; ++i) {
         out_leaf[i] = -1;
@@ -474,12 +539,12 @@ __global__ void __launch_bounds__(256) topk_kernel(const int32_t* __restrict__ c
         if (t >= p.N) continue;
         const int64_t unit = bh * p.N + t;
         const Forced F(t, p.C, p.causal, p.forced_mask);
-        const int leaf = cand[unit * kSlots + lane];
+        const int leaf = leaves[i];
         float l2[G];
         float score = 0.f;
 #pragma unroll
         for (int h = 0; h < G; ++h) {
-            l2[h] = leaf >= 0 ? lse[(unit * kSlots + lane) * G + h] : -INFINITY;
+            l2[h] = leaf >= 0 ? l2s[i][h] : -INFINITY;
             score += l2[h];
         }
         const bool valid = leaf >= 0;
@@ -957,6 +1022,7 @@ BmLayout blockmajor_layout(const BmShape& s) {
     L.offsets = take(nb * 4);
     L.entries = take(units * kSlots * 4);
     L.tiles = take(max_tiles * 16);
+    L.bsum = take(((nb + kScanBlock - 1) / kScanBlock) * 16);
     L.misc = take(256);  // [0] tile count, [1] error word
     L.oacc = take((int64_t)s.B * s.Hq * s.N * kD * 4);
     L.total = off;
@@ -988,9 +1054,12 @@ static cudaError_t place_tiles(const int32_t* src, int stride, const SelectParam
                                uint8_t* ws, const BmLayout& L, cudaStream_t st, bool pairs = false) {
     const int64_t nkeys = pairs ? (s.M1 + 1) / 2 : s.M1;
     const int64_t nb = (int64_t)s.B * s.Hkv * nkeys;
-    bucket_scan_kernel<<<1, 1024, 0, st>>>((const int32_t*)(ws + L.counts), nb, nkeys, 128 / s.G, s.N,
-                                           (int32_t*)(ws + L.offsets), (int4*)(ws + L.tiles),
-                                           (int32_t*)(ws + L.misc), (int*)(ws + L.misc) + 1);
+    const unsigned nblk = (unsigned)((nb + kScanBlock - 1) / kScanBlock);
+    bucket_total_kernel<<<nblk, kScanBlock, 0, st>>>((const int32_t*)(ws + L.counts), nb, 128 / s.G, s.N,
+                                                     (longlong2*)(ws + L.bsum), (int*)(ws + L.misc) + 1);
+    bucket_place_kernel<<<nblk, kScanBlock, 0, st>>>((const int32_t*)(ws + L.counts), nb, nkeys, 128 / s.G, s.N,
+                                                     (const longlong2*)(ws + L.bsum), (int32_t*)(ws + L.offsets),
+                                                     (int4*)(ws + L.tiles), (int32_t*)(ws + L.misc));
     GroupParams g = group_params(stride, sp, s);
     if (pairs) {
         g.M1 = nkeys;

@@ -40,7 +40,7 @@ struct BmShape {
     int64_t rows;  // pyramid rows per (b, kv-head)
 };
 struct BmLayout {  // byte offsets of the workspace regions
-    size_t cand, lse, z2, counts, slots, offsets, entries, tiles, misc, oacc, total;
+    size_t cand, lse, z2, counts, slots, offsets, entries, tiles, bsum, misc, oacc, total;
 };
 struct PhaseEvents {  // optional caller events recorded at phase boundaries
     void* const* events;
