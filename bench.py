@@ -235,6 +235,29 @@ class ClockSampler:
 
 # ------------------------------------------------------------ cpu baseline ----
 
+# ------------------------------------------------------------ replicas ----
+
+def replica_seed(base_seed: int, rank: int) -> int:
+    """Each rank runs its own seeded copy of the workload (weak scaling)."""
+    return base_seed + rank
+
+
+def max_over_ranks(ms: float, dist, device) -> float:
+    """The job's time is the slowest rank's: all-reduce MAX of a per-rank time
+    (any backend: `device` is cuda for NCCL, cpu for gloo)."""
+    if dist is None:
+        return ms
+    import torch
+    tt = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+    return float(tt.item())
+
+
+def job_tokens_per_s(tokens_per_rank: int, world: int, ms_per_step: float) -> float:
+    """Whole-job throughput: the tokens all ranks processed over the max-rank time."""
+    return tokens_per_rank * world / (ms_per_step / 1e3)
+
+
 def oracle_prefill_sample(w, Q, K, V, rows_per_head: int, rng_seed: int = 0):
     """Time the oracle (fp64, OpenMP) on: the full pyramid of every KV head and
     selection + attention for `rows_per_head` sampled query rows of every head.
@@ -336,7 +359,7 @@ def main():
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
 
-    Q, K, V, meta = make_inputs(w, seed=w.seed + rank)
+    Q, K, V, meta = make_inputs(w, seed=replica_seed(w.seed, rank))
     Qd, Kd, Vd = Q.to(dev), K.to(dev), V.to(dev)
     cfg = pisa.cfg_for(Qd, Kd, C=w.C, K_=w.K, causal=w.causal, forced_mask=w.forced_mask)
     pyr, idx, O = pisa.alloc_outputs(cfg, dev, Qd.dtype)
@@ -377,13 +400,10 @@ def main():
     total_ms = evs[0][0].elapsed_time(evs[-1][nph])
     phase_ms = {name: float(np.mean([e[i].elapsed_time(e[i + 1]) for e in evs]))
                 for i, name in enumerate(pisa.PHASES)}
-    if dist:
-        tt = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        total_ms = float(tt.item())
+    total_ms = max_over_ranks(total_ms, dist, dev)
     ms_per_step = total_ms / args.steps
     tokens = w.B * w.N * world
-    value = tokens / (ms_per_step / 1e3)
+    value = job_tokens_per_s(w.B * w.N, world, ms_per_step)
 
     alg = algorithmic(w, w.N)
     pk = peaks()
@@ -475,11 +495,8 @@ def main():
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / n_e2e
-    if dist:
-        tt = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
-    out["e2e"] = {"value": tokens / (e2e_ms / 1e3), "unit": unit,
+    e2e_ms = max_over_ranks(e2e_ms, dist, dev)
+    out["e2e"] = {"value": job_tokens_per_s(w.B * w.N, world, e2e_ms), "unit": unit,
                   "h2d_bytes_per_step": int(Qh.nbytes + Kh.nbytes + Vh.nbytes),
                   "d2h_bytes_per_step": int(Oh.nbytes + Ih.nbytes), "ms_per_step": e2e_ms}
     del Qh, Kh, Vh, Oh, Ih
