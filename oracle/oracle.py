@@ -63,10 +63,10 @@ def _load():
         lib.oracle_build_pyramid.restype = None
         lib.oracle_pyramid_append.argtypes = [i64, i64, c_int, c_int, c_int, P, P]
         lib.oracle_pyramid_append.restype = None
-        lib.oracle_node_score.argtypes = [c_int, i64, i64, c_int, c_int, c_int, P, P, P, c_int, i64]
+        lib.oracle_node_score.argtypes = [c_int, i64, i64, c_int, c_int, c_int, P, P, P, c_int, i64, c_int]
         lib.oracle_node_score.restype = ctypes.c_double
         lib.oracle_select_rows.argtypes = [c_int, i64, i64, c_int, c_int, c_int, c_int, c_int, c_int,
-                                           P, P, i64, P, P, P, P, P]
+                                           P, P, i64, P, P, P, P, P, c_int]
         lib.oracle_select_rows.restype = None
         lib.oracle_flat_rows.argtypes = [c_int, c_int, i64, i64, c_int, c_int, c_int, c_int, c_int, c_int,
                                          P, P, i64, P, P, P, P]
@@ -137,22 +137,27 @@ def pyramid_append(P: np.ndarray, Kh: np.ndarray, n: int, C: int, g: int, N_layo
     _load().oracle_pyramid_append(int(n), int(N_layout), Kh.shape[-1], C, g, _p(Kh), _p(P))
 
 
+VARIANTS = {"lse": 0, "pisa1": 1, "pisa2": 2}
+
+
 def node_score(qg: np.ndarray, Kh: np.ndarray, P: np.ndarray, level: int, node: int, C: int,
-               g: int = 2, N: int | None = None, N_layout: int | None = None) -> float:
-    """Eq.(7) (+ Eq.11 sum over the G rows of qg [G, d]) for one node."""
+               g: int = 2, N: int | None = None, N_layout: int | None = None, variant: int = 0) -> float:
+    """Eq.(7) (+ Eq.11 sum over the G rows of qg [G, d]) for one node; variant
+    1 / 2 scores by the PISA-1 / PISA-2 ablation (Eq.8-9) instead."""
     qg = np.ascontiguousarray(np.atleast_2d(qg), dtype=np.float64)
     Kh = np.ascontiguousarray(Kh, dtype=np.float64)
     N = Kh.shape[0] if N is None else N
     N_layout = N if N_layout is None else N_layout
     return float(_load().oracle_node_score(qg.shape[0], N, N_layout, qg.shape[1], C, g,
                                            _p(Kh), _p(np.ascontiguousarray(P)), _p(qg),
-                                           int(level), int(node)))
+                                           int(level), int(node), int(variant)))
 
 
 def select_rows(Qrows: np.ndarray, t: np.ndarray, Kh: np.ndarray, P: np.ndarray, *, C: int, K: int,
                 g: int = 2, causal: bool = True, forced_mask: int = 7, N: int | None = None,
-                N_layout: int | None = None, want_counts: bool = False):
-    """Pyramid walk for query rows of one KV head.
+                N_layout: int | None = None, want_counts: bool = False, variant: int = 0):
+    """Pyramid walk for query rows of one KV head (node score: variant 0 the
+    Eq.7 LSE, 1 PISA-1, 2 PISA-2).
 
     Qrows: [n, G, d] (G query heads of the group), t: [n] positions.
     Returns (idx [n, K] int32, gap [n] float64[, counts [n, MAX_LEVELS, 2] int32]).
@@ -170,7 +175,7 @@ def select_rows(Qrows: np.ndarray, t: np.ndarray, Kh: np.ndarray, P: np.ndarray,
     gap = np.zeros(n, np.float64)
     counts = np.zeros((n, MAX_LEVELS, 2), np.int32) if want_counts else None
     _load().oracle_select_rows(G, N, N_layout, d, C, K, g, int(causal), int(forced_mask),
-                               _p(Kh), _p(P), n, _p(t), _p(Qrows), _p(idx), _p(gap), _p(counts))
+                               _p(Kh), _p(P), n, _p(t), _p(Qrows), _p(idx), _p(gap), _p(counts), int(variant))
     return (idx, gap, counts) if want_counts else (idx, gap)
 
 

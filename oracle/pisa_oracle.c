@@ -18,6 +18,9 @@
  *   Eq.(6)  |I| <= K, |A| <= g K                                      (§04 4.2)
  *   Eq.(7)  s^{(l)}_{t,i} = log sum_{r in Ch(i)} exp(q . kbar^{(l-1)}_r / sqrt d)
  *           (at l = 1 the children are the raw keys)                  (§04 4.3)
+ *   Eq.(8)-(9) the Taylor view of Eq.(7) and its ablations: PISA-1 scores a
+ *           node by the mean of its children's logits, PISA-2 by that mean
+ *           plus half their variance                                  (§04 4.3)
  *   Eq.(11) GQA: the node score is the SUM over the group's query heads
  *           of each head's Eq.(7) score; the group shares the choice  (§04 4.4)
  *   §5.3    forced blocks: the first, previous and current leaf and their
@@ -181,16 +184,35 @@ static double lse(const double *z, int n)
     return m + log(s);
 }
 
+/* Score of a node from its children's logits z[0..n) (n >= 1):
+ *   variant 0: Eq.(7), log sum_r exp(z_r);
+ *   variant 1 (PISA-1, Eq.8 truncated): the mean logit;
+ *   variant 2 (PISA-2, Eq.9): the mean logit plus half the population variance
+ *   of the logits (the second cumulant; divide by n). */
+static double child_score(const double *z, int n, int variant)
+{
+    if (variant == 0) return lse(z, n);
+    double m = 0.0;
+    for (int i = 0; i < n; ++i) m += z[i];
+    m /= (double)n;
+    if (variant == 1) return m;
+    double v = 0.0;
+    for (int i = 0; i < n; ++i) v += (z[i] - m) * (z[i] - m);
+    return m + 0.5 * v / (double)n;
+}
+
 typedef struct {
     int G, d, C, g;
     int64_t N;              /* keys that exist */
     const int64_t *M, *off; /* layout geometry */
     const double *Kh, *P;   /* raw keys [>=N, d]; pyramid */
+    int variant;            /* node score: 0 Eq.(7) LSE, 1 PISA-1, 2 PISA-2 */
 } ctx_t;
 
-/* Eq.(7) for one query head, summed over the G heads of the group (Eq.11).
- * Level l >= 2: LSE over the existing child summaries at level l-1.
- * Level 1: LSE over the raw keys of the leaf (exact leaf LSE). */
+/* Eq.(7) (or its PISA-1 / PISA-2 ablation) for one query head, summed over
+ * the G heads of the group (Eq.11).
+ * Level l >= 2: over the existing child summaries at level l-1.
+ * Level 1: over the raw keys of the leaf (the exact leaf LSE for Eq.7). */
 static double node_score(const ctx_t *c, const double *qg, int l, int64_t i)
 {
     double inv = 1.0 / sqrt((double)c->d);
@@ -202,7 +224,7 @@ static double node_score(const ctx_t *c, const double *qg, int l, int64_t i)
         for (int h = 0; h < c->G; ++h) {
             for (int64_t j = lo; j < hi; ++j)
                 z[j - lo] = dot(qg + (int64_t)h * c->d, c->Kh + j * c->d, c->d) * inv;
-            total += lse(z, n);
+            total += n > 0 ? child_score(z, n, c->variant) : -INFINITY;
         }
         free(z);
     } else {
@@ -214,7 +236,7 @@ static double node_score(const ctx_t *c, const double *qg, int l, int64_t i)
             int n = 0;
             for (int64_t r = r0; r < r1; ++r)
                 z[n++] = dot(qg + (int64_t)h * c->d, c->P + (c->off[l - 1] + r) * c->d, c->d) * inv;
-            total += lse(z, n);
+            total += n > 0 ? child_score(z, n, c->variant) : -INFINITY;
         }
     }
     return total;
@@ -222,12 +244,12 @@ static double node_score(const ctx_t *c, const double *qg, int l, int64_t i)
 
 double oracle_node_score(int G, int64_t N, int64_t N_layout, int d, int C, int g,
                          const double *Kh, const double *P, const double *qg,
-                         int level, int64_t node)
+                         int level, int64_t node, int variant)
 {
     int64_t M[OR_MAX_LEVELS + 1], off[OR_MAX_LEVELS + 1];
     int L = oracle_geometry(N_layout, C, g, M, off);
     if (L <= 0 || level < 1 || level > L) return NAN;
-    ctx_t c = {G, d, C, g, N, M, off, Kh, P};
+    ctx_t c = {G, d, C, g, N, M, off, Kh, P, variant};
     return node_score(&c, qg, level, node);
 }
 
@@ -372,12 +394,12 @@ static void walk_one(const ctx_t *c, int L, int K, int causal, int mask,
 void oracle_select_rows(int G, int64_t N, int64_t N_layout, int d, int C, int K, int g,
                         int causal, int forced_mask, const double *Kh, const double *P,
                         int64_t n, const int64_t *t, const double *Qrows,
-                        int32_t *idx, double *gap, int32_t *counts)
+                        int32_t *idx, double *gap, int32_t *counts, int variant)
 {
     int64_t M[OR_MAX_LEVELS + 1], off[OR_MAX_LEVELS + 1];
     int L = oracle_geometry(N_layout, C, g, M, off);
     if (L <= 0) return;
-    ctx_t c = {G, d, C, g, N, M, off, Kh, P};
+    ctx_t c = {G, d, C, g, N, M, off, Kh, P, variant};
 #pragma omp parallel for schedule(dynamic, 4)
     for (int64_t u = 0; u < n; ++u)
         walk_one(&c, L, K, causal, forced_mask, t[u], Qrows + u * G * d, idx + u * K,
@@ -435,7 +457,7 @@ void oracle_flat_rows(int kind, int G, int64_t N, int64_t N_layout, int d, int C
     int64_t M[OR_MAX_LEVELS + 1], off[OR_MAX_LEVELS + 1];
     int L = oracle_geometry(N_layout, C, g, M, off);
     if (L <= 0) return;
-    ctx_t c = {G, d, C, g, N, M, off, Kh, P};
+    ctx_t c = {G, d, C, g, N, M, off, Kh, P, 0};
 #pragma omp parallel for schedule(dynamic, 4)
     for (int64_t u = 0; u < n; ++u)
         flat_one(&c, kind, K, causal, forced_mask, t[u], Qrows + u * G * d, idx + u * K,
