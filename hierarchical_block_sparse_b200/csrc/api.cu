@@ -20,6 +20,7 @@ int check_cfg(const pisa_cfg* c) {
     if (c->causal != 0 && c->causal != 1) return PISA_E_INVALID;
     if (c->forced_mask < 0 || c->forced_mask > 7) return PISA_E_INVALID;
     if (c->dtype != PISA_DTYPE_F32 && c->dtype != PISA_DTYPE_BF16) return PISA_E_INVALID;
+    if (c->score_variant < PISA_SCORE_LSE || c->score_variant > PISA_SCORE_MEAN_VAR) return PISA_E_INVALID;
     const int forced = c->forced_mask | (c->causal ? 4 : 0);
     const int nf = (forced & 1) + ((forced >> 1) & 1) + ((forced >> 2) & 1);
     if (c->K < nf) return PISA_E_INVALID;  // forced leaves count against K (Eq.6)
@@ -68,6 +69,7 @@ SelectParams select_params(const pisa_cfg* c, const Geom& g) {
     p.causal = c->causal; p.forced_mask = c->forced_mask;
     p.qscale = (float)(1.4426950408889634 / sqrt((double)c->d));
     p.geom = g;
+    p.variant = c->score_variant;
     return p;
 }
 
@@ -98,6 +100,7 @@ BmShape bm_shape(const pisa_cfg* c) {
     Geom g;
     make_geom(c->N, c->C, &g);
     s.rows = g.rows;
+    s.variant = c->score_variant;
     return s;
 }
 
@@ -114,6 +117,7 @@ DecodeParams decode_params(const pisa_cfg* c, const Geom& g) {
     p.forced_mask = c->forced_mask;
     p.qscale = (float)(1.4426950408889634 / sqrt((double)c->d));
     p.geom = g;
+    p.variant = c->score_variant;
     return p;
 }
 

@@ -94,7 +94,7 @@ __global__ void __launch_bounds__(256, PISA_STAGE1_MINBLOCKS) stage1_kernel(cons
         const unsigned fmask = __ballot_sync(kFull, s.forced);
         if (__popc(fmask) < p.K)
             score = w.score_internal(cand, s.vmask & ~fmask, P + p.geom.off[l - 1] * kD,
-                                     (int64_t)p.C << (l - 2), p.N, lane);
+                                     (int64_t)p.C << (l - 2), p.N, lane, p.variant);
         int id = cand;
         const int kept = keep_topk_lane(id, s.forced ? INFINITY : score, s.valid, p.K, lane);
         parent = __shfl_sync(kFull, id, lane >> 1);
@@ -395,6 +395,7 @@ struct TileParams {
     int64_t M1;
     float qscale;  // log2(e) / sqrt(d)
     int max_tiles;  // capacity of the tile list
+    int variant;    // enum pisa_score (leaf scoring: PISA-1 / PISA-2 ranking scores when nonzero)
 };
 
 // Per-head LSE (log2 units) of every listed (query, candidate leaf):
@@ -408,8 +409,8 @@ __global__ void __launch_bounds__(128) leaf_score_kernel(const __nv_bfloat16* __
                                                          const int4* __restrict__ tiles,
                                                          const int32_t* __restrict__ ntiles_ptr,
                                                          const uint32_t* __restrict__ entries,
-                                                         float* __restrict__ lse, int* __restrict__ err,
-                                                         TileParams p, int forced_mask) {
+                                                         float* __restrict__ lse, float* __restrict__ vscore,
+                                                         int* __restrict__ err, TileParams p, int forced_mask) {
     constexpr int NK = PAIR ? 128 : 64;  // keys per tile
     extern __shared__ __align__(1024) uint8_t dsm[];
     uint8_t* sA = dsm;           // 32 KB gathered query rows
@@ -487,6 +488,20 @@ __global__ void __launch_bounds__(128) leaf_score_kernel(const __nv_bfloat16* __
                     if (j < nvalid) s += exp2f(v[j] * p.qscale - m);
                 const int64_t unit = bh * p.N + t;
                 lse[(unit * kSlots + slot) * G + (tid % G)] = m + log2f(s);
+                if (vscore) {  // PISA-1 / PISA-2 ranking score: two-pass mean and variance of the logits
+                    float sum = 0.f;
+#pragma unroll
+                    for (int j = 0; j < 64; ++j)
+                        if (j < nvalid) sum += v[j];
+                    const float mean = sum / (float)nvalid;
+                    float m2 = 0.f;
+#pragma unroll
+                    for (int j = 0; j < 64; ++j)
+                        if (j < nvalid) m2 += (v[j] - mean) * (v[j] - mean);
+                    const float mean2 = mean * p.qscale, var2 = m2 / (float)nvalid * p.qscale * p.qscale;
+                    vscore[(unit * kSlots + slot) * G + (tid % G)] =
+                        p.variant == 1 ? mean2 : mean2 + kHalfLn2 * var2;
+                }
             }
         }
         tc::tc_fence_before();
@@ -514,6 +529,7 @@ constexpr int kTopkQ = 4;
 
 template <int G>
 __global__ void __launch_bounds__(256) topk_kernel(const int32_t* __restrict__ cand, const float* __restrict__ lse,
+                                                   const float* __restrict__ vscore,
                                                    int32_t* __restrict__ idx, float* __restrict__ z2,
                                                    int32_t* __restrict__ counts, int32_t* __restrict__ slots,
                                                    int64_t M1, SelectParams p) {
@@ -524,13 +540,18 @@ __global__ void __launch_bounds__(256) topk_kernel(const int32_t* __restrict__ c
     int out_leaf[kTopkQ];  // lane < K: the lane-th kept leaf that needs a bucket slot, else -1
     // all positions' candidates and LSEs are loaded first (independent requests in flight)
     int leaves[kTopkQ];
-    float l2s[kTopkQ][G];
+    float l2s[kTopkQ][G], rank_score[kTopkQ];
 #pragma unroll
     for (int i = 0; i < kTopkQ; ++i) {
         const int64_t unit = bh * p.N + t0 + i;
         leaves[i] = t0 + i < p.N ? cand[unit * kSlots + lane] : -1;
+        rank_score[i] = 0.f;
 #pragma unroll
-        for (int h = 0; h < G; ++h) l2s[i][h] = t0 + i < p.N ? lse[(unit * kSlots + lane) * G + h] : -INFINITY;
+        for (int h = 0; h < G; ++h) {
+            l2s[i][h] = t0 + i < p.N ? lse[(unit * kSlots + lane) * G + h] : -INFINITY;
+            // ranking: the Eq.(7) LSE, or the PISA-1 / PISA-2 score, summed over the group (Eq.11)
+            rank_score[i] += vscore ? (t0 + i < p.N ? vscore[(unit * kSlots + lane) * G + h] : -INFINITY) : l2s[i][h];
+        }
     }
 #pragma unroll
     for (int i = 0; i < kTopkQ; ++i) {
@@ -541,12 +562,9 @@ __global__ void __launch_bounds__(256) topk_kernel(const int32_t* __restrict__ c
         const Forced F(t, p.C, p.causal, p.forced_mask);
         const int leaf = leaves[i];
         float l2[G];
-        float score = 0.f;
 #pragma unroll
-        for (int h = 0; h < G; ++h) {
-            l2[h] = leaf >= 0 ? l2s[i][h] : -INFINITY;
-            score += l2[h];
-        }
+        for (int h = 0; h < G; ++h) l2[h] = leaf >= 0 ? l2s[i][h] : -INFINITY;
+        const float score = leaf >= 0 ? rank_score[i] : -INFINITY;
         const bool valid = leaf >= 0;
         const bool forced = valid && F.has(leaf, 1);
         const unsigned vmask = __ballot_sync(kFull, valid);
@@ -1016,6 +1034,7 @@ BmLayout blockmajor_layout(const BmShape& s) {
     };
     L.cand = take(units * kSlots * 4);
     L.lse = take(units * kSlots * s.G * 4);
+    L.vscore = take(s.variant ? units * kSlots * s.G * 4 : 0);  // PISA-1 / PISA-2 ranking scores
     L.z2 = take(units * s.G * 4);
     L.counts = take(nb * 4);
     L.slots = take(units * kPairs * 4);
@@ -1100,7 +1119,7 @@ constexpr int kAttnCtasPerSm = 3;
 template <int G, bool PAIR>
 static cudaError_t leaf_scores(const void* Q, const void* K, const SelectParams& sp, const BmShape& s, uint8_t* ws,
                                const BmLayout& L, cudaStream_t st) {
-    TileParams tp{s.B, s.Hq, s.Hkv, s.N, sp.causal, s.M1, sp.qscale, max_tiles_of(s)};
+    TileParams tp{s.B, s.Hq, s.Hkv, s.N, sp.causal, s.M1, sp.qscale, max_tiles_of(s), sp.variant};
     constexpr size_t smem = 32768 + (PAIR ? 32768 : 16384);
     auto kern = leaf_score_kernel<G, PAIR>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -1108,6 +1127,7 @@ static cudaError_t leaf_scores(const void* Q, const void* K, const SelectParams&
     kern<<<sm_count() * (PAIR ? 3 : 4), 128, smem, st>>>((const __nv_bfloat16*)Q, (const __nv_bfloat16*)K,
                                                           (const int4*)(ws + L.tiles), (const int32_t*)(ws + L.misc),
                                                           (const uint32_t*)(ws + L.entries), (float*)(ws + L.lse),
+                                                          (PAIR && sp.variant) ? (float*)(ws + L.vscore) : nullptr,
                                                           (int*)(ws + L.misc) + 1, tp, sp.forced_mask);
     return cudaGetLastError();
 }
@@ -1142,7 +1162,9 @@ static cudaError_t select_bm_t(const void* Q, const void* K, const float* pyr, i
     e = zero_counts(s, ws, L, st);  // the Top-K counts the kept leaves for the attention grouping
     if (e != cudaSuccess) return e;
     const dim3 topk_grid((unsigned)((s.N + 8 * kTopkQ - 1) / (8 * kTopkQ)), (unsigned)(s.B * s.Hkv));
-    topk_kernel<G><<<topk_grid, 256, 0, st>>>(cand, (const float*)(ws + L.lse), idx, (float*)(ws + L.z2),
+    topk_kernel<G><<<topk_grid, 256, 0, st>>>(cand, (const float*)(ws + L.lse),
+                                              sp.variant ? (const float*)(ws + L.vscore) : nullptr, idx,
+                                              (float*)(ws + L.z2),
                                               (int32_t*)(ws + L.counts), (int32_t*)(ws + L.slots), s.M1, sp);
     e = cudaGetLastError();
     mark(ev, 5, st);
@@ -1191,7 +1213,7 @@ static cudaError_t attn_bm_t(const void* Q, const void* K, const void* V, const 
         if (e != cudaSuccess) return e;
     }
     mark(ev, 7, st);
-    TileParams tp{s.B, s.Hq, s.Hkv, s.N, sp.causal, s.M1, sp.qscale, max_tiles_of(s)};
+    TileParams tp{s.B, s.Hq, s.Hkv, s.N, sp.causal, s.M1, sp.qscale, max_tiles_of(s), sp.variant};
     auto kern = attn_tile_kernel<G>;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kAttnSmem);
     if (e != cudaSuccess) return e;

@@ -210,9 +210,16 @@ __global__ void __launch_bounds__(256, decode_min_blocks<G>()) decode_kernel(
     __shared__ unsigned s_need;
     __shared__ int s_level, s_nlist;
     __shared__ float s_Z[G];
-    __shared__ float s_pm[32][NW][G], s_ps[32][NW][G];  // per-warp LSE states of the listed leaves
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    // per-warp states of the listed leaves, after the pipeline stages: the LSE
+    // (max, sum) and, for the PISA-1 / PISA-2 ranking, the logits' moments
+    using Part = float[32][NW][G];
+    Part& s_pm = *reinterpret_cast<Part*>(dsm + kDecStages * kDecStageBytes);
+    Part& s_ps = *reinterpret_cast<Part*>(dsm + kDecStages * kDecStageBytes + sizeof(Part));
+    Part& s_vn = *reinterpret_cast<Part*>(dsm + kDecStages * kDecStageBytes + 2 * sizeof(Part));
+    Part& s_vmean = *reinterpret_cast<Part*>(dsm + kDecStages * kDecStageBytes + 3 * sizeof(Part));
+    Part& s_vm2 = *reinterpret_cast<Part*>(dsm + kDecStages * kDecStageBytes + 4 * sizeof(Part));
     const int64_t unit = blockIdx.x;  // b * Hkv + kvh
     const int64_t b = unit / p.Hkv;
     const int kvh = (int)(unit - b * p.Hkv);
@@ -325,11 +332,8 @@ __global__ void __launch_bounds__(256, decode_min_blocks<G>()) decode_kernel(
                 const bool has1 = (2 * (int64_t)cand + 1) * ((int64_t)p.C << (l - 2)) < n_keys;
                 score = 0.f;
 #pragma unroll
-                for (int h = 0; h < G; ++h) {
-                    const float z0 = s_dot[2 * lane][h], z1 = has1 ? s_dot[2 * lane + 1][h] : -INFINITY;
-                    const float m = fmaxf(z0, z1);
-                    score += m + log2f(exp2f(z0 - m) + exp2f(z1 - m));
-                }
+                for (int h = 0; h < G; ++h)
+                    score += pair_score(s_dot[2 * lane][h], has1 ? s_dot[2 * lane + 1][h] : -INFINITY, p.variant);
             }
             int id = cand;
             const int kept = keep_topk_lane(id, s.forced ? INFINITY : score, s.valid, p.K, lane);
@@ -425,25 +429,56 @@ __global__ void __launch_bounds__(256, decode_min_blocks<G>()) decode_kernel(
                     s_pm[j][warp][h] = mm;
                     s_ps[j][warp][h] = ss;
                 }
+                if (p.variant) {  // moments of this warp's logits (two passes), merged likewise
+                    const bool live = z != -INFINITY && sl == 0;
+                    float cnt = live ? 1.f : 0.f, sum = live ? z : 0.f;
+#pragma unroll
+                    for (int o = TPR; o < 32; o <<= 1) {
+                        cnt += __shfl_xor_sync(kFull, cnt, o);
+                        sum += __shfl_xor_sync(kFull, sum, o);
+                    }
+                    const float mean = cnt > 0.f ? sum / cnt : 0.f;
+                    float dev = live ? (z - mean) * (z - mean) : 0.f;
+#pragma unroll
+                    for (int o = TPR; o < 32; o <<= 1) dev += __shfl_xor_sync(kFull, dev, o);
+                    if (lane == 0) {
+                        Moments mo;
+                        if (tile % tpl != 0) {
+                            mo.n = s_vn[j][warp][h];
+                            mo.mean = s_vmean[j][warp][h];
+                            mo.m2 = s_vm2[j][warp][h];
+                        }
+                        mo.merge(cnt, mean, dev);
+                        s_vn[j][warp][h] = mo.n;
+                        s_vmean[j][warp][h] = mo.mean;
+                        s_vm2[j][warp][h] = mo.m2;
+                    }
+                }
             }
         }
         tc::cp_async_wait_all();
         __syncthreads();
-        if (tid < nlist * G) {  // leaf LSE per head
+        if (tid < nlist * G) {  // leaf LSE per head (and the PISA-1 / PISA-2 score in s_dot)
             const int j = tid / G, h = tid - j * G;
             float m = -INFINITY, sm = 0.f;
 #pragma unroll
             for (int ww = 0; ww < NW; ++ww) lse_merge(m, sm, s_pm[j][ww][h], s_ps[j][ww][h]);
             s_lse[s_slot[j]][h] = m + log2f(sm);
+            if (p.variant) {
+                Moments mo;
+#pragma unroll
+                for (int ww = 0; ww < NW; ++ww) mo.merge(s_vn[j][ww][h], s_vmean[j][ww][h], s_vm2[j][ww][h]);
+                s_dot[s_slot[j]][h] = mo.score(p.variant);
+            }
         }
     }
     __syncthreads();
 
     if (warp == 0) {  // final Top-K (kept leaves come out in ascending order), then Z per head
         const LevelState s = level_state(cand, 1, p.C, n_keys, t, 1, F);
-        float score = 0.f;
+        float score = 0.f;  // ranking: the LSE or the PISA-1 / PISA-2 score, summed over the group (Eq.11)
 #pragma unroll
-        for (int h = 0; h < G; ++h) score += s.valid ? s_lse[lane][h] : 0.f;  // Eq.(11)
+        for (int h = 0; h < G; ++h) score += s.valid ? (p.variant ? s_dot[lane][h] : s_lse[lane][h]) : 0.f;
         int id = cand, kept;
         unsigned kmask;
         if (s.n <= p.K) {
@@ -621,7 +656,8 @@ static cudaError_t launch_decode_t(const void* q, void* Kc, void* Vc, float* pyr
                                    void* o, const void* k_new, const void* v_new, const DecodeParams& p,
                                    cudaStream_t st) {
     const size_t out_bytes = sizeof(float) * 8 * G * (D + 1);
-    const size_t stage_bytes = (size_t)kDecStages * kDecStageBytes;
+    // pipeline stages + five per-warp arrays [32][8][G] of leaf states
+    const size_t stage_bytes = (size_t)kDecStages * kDecStageBytes + 5 * sizeof(float) * 32 * 8 * G;
     const size_t smem = out_bytes > stage_bytes ? out_bytes : stage_bytes;
     auto kern = decode_kernel<T, D, G>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

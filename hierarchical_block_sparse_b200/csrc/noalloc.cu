@@ -73,6 +73,7 @@ extern "C" int pisa_select_noalloc(const pisa_cfg* cfg, const void* Q, const voi
     Geom g;
     make_geom(cfg->N, cfg->C, &g);
     s.rows = g.rows;
+    s.variant = cfg->score_variant;
     const BmLayout L = blockmajor_layout(s);
     // the selection uses every region except the attention accumulator, which is last
     if (L.oacc > kScratchBytes) return PISA_E_SCRATCH_LIMIT;
@@ -83,6 +84,7 @@ extern "C" int pisa_select_noalloc(const pisa_cfg* cfg, const void* Q, const voi
     sp.causal = cfg->causal; sp.forced_mask = cfg->forced_mask;
     sp.qscale = (float)(1.4426950408889634 / sqrt((double)cfg->d));
     sp.geom = g;
+    sp.variant = cfg->score_variant;
     const cudaError_t e = launch_select_bm(Q, K, pyr, idx, sp, s, ws, nullptr, (cudaStream_t)stream);
     return e == cudaSuccess ? PISA_OK : PISA_E_CUDA;
 }

@@ -145,6 +145,56 @@ __device__ __forceinline__ float reduce_scatter32(float (&v)[32], int lane) {
     return v[0];
 }
 
+// ---- node scores from the children's logits (close reading §04 4.3) ------------
+// Logits are in log2 units on the GPU (z2 = z * log2(e)). Eq.(7): LSE; PISA-1:
+// the mean; PISA-2: mean + var / 2 in nats, which is mean2 + var2 * ln(2) / 2
+// in log2 units (a positive multiple: every ranking is preserved).
+constexpr float kHalfLn2 = 0.34657359027997264f;
+
+// score of a node from the logits of its (up to) two children; a missing
+// child is -inf. Symmetric in (a, b).
+__device__ __forceinline__ float pair_score(float a, float b, int variant) {
+    if (a == -INFINITY) return b;
+    if (b == -INFINITY) return a;
+    if (variant == 0) {
+        const float m = fmaxf(a, b);
+        return m + log2f(exp2f(a - m) + exp2f(b - m));
+    }
+    const float mean = 0.5f * (a + b);
+    if (variant == 1) return mean;
+    const float h = 0.5f * (a - b);
+    return mean + kHalfLn2 * h * h;
+}
+
+// count, mean and sum of squared deviations of a set of logits (mergeable)
+struct Moments {
+    float n = 0.f, mean = 0.f, m2 = 0.f;
+    __device__ __forceinline__ void add(float x) {
+        n += 1.f;
+        const float d = x - mean;
+        mean += d / n;
+        m2 += d * (x - mean);
+    }
+    __device__ __forceinline__ void merge(float nb, float meanb, float m2b) {
+        if (nb == 0.f) return;
+        if (n == 0.f) {
+            n = nb;
+            mean = meanb;
+            m2 = m2b;
+            return;
+        }
+        const float nn = n + nb, d = meanb - mean;
+        mean += d * (nb / nn);
+        m2 += m2b + d * d * (n * nb / nn);
+        n = nn;
+    }
+    // PISA-1 / PISA-2 score (variant 1 / 2)
+    __device__ __forceinline__ float score(int variant) const {
+        if (n == 0.f) return -INFINITY;
+        return variant == 1 ? mean : mean + kHalfLn2 * (m2 / n);
+    }
+};
+
 // ---- warp bitonic sorts -----------------------------------------------------------
 
 // (ka, ia) ranks before (kb, ib): larger key first, then lower index.

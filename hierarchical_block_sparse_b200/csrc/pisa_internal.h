@@ -20,6 +20,7 @@ struct SelectParams {
     int B, Hq, Hkv, N, C, K, causal, forced_mask;
     float qscale;  // log2(e) / sqrt(d)
     Geom geom;
+    int variant;   // enum pisa_score
 };
 
 struct AttnParams {
@@ -31,6 +32,7 @@ struct DecodeParams {
     int B, Hq, Hkv, N, C, K, forced_mask;
     float qscale;  // log2(e) / sqrt(d)
     Geom geom;     // layout for the capacity N
+    int variant;   // enum pisa_score
 };
 
 // block-major tensor-core path (bf16, d = 128, C = 64)
@@ -38,9 +40,10 @@ struct BmShape {
     int B, Hq, Hkv, N, G;
     int64_t M1;    // leaves per sequence
     int64_t rows;  // pyramid rows per (b, kv-head)
+    int variant;   // enum pisa_score (the ranking scores need their own region unless 0)
 };
 struct BmLayout {  // byte offsets of the workspace regions
-    size_t cand, lse, z2, counts, slots, offsets, entries, tiles, bsum, misc, oacc, total;
+    size_t cand, lse, vscore, z2, counts, slots, offsets, entries, tiles, bsum, misc, oacc, total;
 };
 struct PhaseEvents {  // optional caller events recorded at phase boundaries
     void* const* events;

@@ -48,7 +48,8 @@ struct Walk4S {
     }
 
     __device__ __forceinline__ float score_internal(int cand, unsigned need, const float* child_lvl,
-                                                    int64_t span_child, int64_t n_keys, int lane) const {
+                                                    int64_t span_child, int64_t n_keys, int lane,
+                                                    int variant = 0) const {
         const int g = lane >> 2, j = lane & 3;
         int cbase[4];      // first-child row offset (floats) of the group's 4 candidates, chunk j
         unsigned okm = 0;  // bit r: row r of the group exists and is wanted
@@ -124,11 +125,7 @@ struct Walk4S {
         const bool has1 = (2 * (int64_t)cand + 1) * span_child < n_keys;
         float score = 0.f;
 #pragma unroll
-        for (int h = 0; h < G; ++h) {
-            const float z0 = part[h], z1 = has1 ? part[G + h] : -INFINITY;
-            const float m = fmaxf(z0, z1);
-            score += (m == -INFINITY) ? -INFINITY : m + log2f(exp2f(z0 - m) + exp2f(z1 - m));
-        }
+        for (int h = 0; h < G; ++h) score += pair_score(part[h], has1 ? part[G + h] : -INFINITY, variant);
         return mine ? score : -INFINITY;
     }
 };

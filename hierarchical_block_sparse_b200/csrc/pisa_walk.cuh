@@ -55,7 +55,7 @@ struct Walk {
     // head's pyramid; children with first token >= n_keys do not exist.
     __device__ __forceinline__ float score_internal(int cand, unsigned need, const float* child_lvl,
                                                     int64_t span_child, int64_t n_keys,
-                                                    int lane) const {
+                                                    int lane, int variant = 0) const {
         float my = -INFINITY;
         constexpr int CPB = RB / 2;  // candidates finished per batch
         for (int bi = 0; bi < 32 / CPB; ++bi) {
@@ -77,10 +77,9 @@ struct Walk {
                 const bool ok = ((need >> c) & 1u) && (int64_t)child * span_child < n_keys;
                 if (!ok) z = -INFINITY;
             }
-            // LSE over the two children of the same head: partner lane is lane ^ G
+            // score over the two children of the same head: partner lane is lane ^ G
             const float z2 = __shfl_xor_sync(kFull, z, G);
-            const float m = fmaxf(z, z2);
-            float s = (m == -INFINITY) ? -INFINITY : m + log2f(exp2f(z - m) + exp2f(z2 - m));
+            float s = pair_score(z, z2, variant);
 #pragma unroll
             for (int o = 1; o < G; o <<= 1) s += __shfl_xor_sync(kFull, s, o);
             // candidate c of this batch sits in lanes [(c - bi*CPB) * 2G, +2G)
@@ -94,16 +93,43 @@ struct Walk {
     // Eq.(7) at the leaves: exact LSE over each flagged candidate's raw keys
     // [leaf*C, min(leaf*C + C, n_keys)), summed over the G heads.
     __device__ __forceinline__ float score_leaves(int cand, unsigned need, const T* Kh, int C,
-                                                  int64_t n_keys, int lane) const {
+                                                  int64_t n_keys, int lane, int variant = 0) const {
         float my = -INFINITY;
         while (need) {
             const int c = __ffs(need) - 1;
             need &= need - 1;
             const int leaf = __shfl_sync(kFull, cand, c);
-            const float s = leaf_lse(Kh, (int64_t)leaf * C, min((int64_t)leaf * C + C, n_keys), lane);
+            const int64_t lo = (int64_t)leaf * C, hi = min((int64_t)leaf * C + C, n_keys);
+            const float s = variant == 0 ? leaf_lse(Kh, lo, hi, lane) : leaf_moments_score(Kh, lo, hi, lane, variant);
             if (lane == c) my = s;
         }
         return my;
+    }
+
+    // PISA-1 / PISA-2 score over the raw keys [lo, hi), summed over the G heads
+    __device__ __forceinline__ float leaf_moments_score(const T* Kh, int64_t lo, int64_t hi, int lane,
+                                                        int variant) const {
+        Moments mo;  // head lane % G
+        for (int64_t r0 = lo; r0 < hi; r0 += RB) {
+            float v[32];
+#pragma unroll
+            for (int r = 0; r < RB; ++r) {
+                const int64_t row = r0 + r;
+                dots_into(v, r, Kh + row * D, row < hi, lane);
+            }
+            const float z = reduce_scatter32(v, lane);
+            if (r0 + lane / G < hi) mo.add(z);
+        }
+#pragma unroll
+        for (int o = G; o < 32; o <<= 1) {
+            const float nb = __shfl_xor_sync(kFull, mo.n, o), mb = __shfl_xor_sync(kFull, mo.mean, o),
+                        m2b = __shfl_xor_sync(kFull, mo.m2, o);
+            mo.merge(nb, mb, m2b);
+        }
+        float r = mo.score(variant);
+#pragma unroll
+        for (int o = 1; o < G; o <<= 1) r += __shfl_xor_sync(kFull, r, o);
+        return r;
     }
 
     // sum over heads of log2-sum-exp2 of the scaled dots with rows [lo, hi)

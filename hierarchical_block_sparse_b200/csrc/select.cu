@@ -44,9 +44,9 @@ __global__ void __launch_bounds__(256) select_kernel(const T* __restrict__ Q, co
                 const unsigned need = s.vmask & ~fmask;
                 if (l >= 2)
                     score = w.score_internal(cand, need, P + p.geom.off[l - 1] * D,
-                                             (int64_t)p.C << (l - 2), p.N, lane);
+                                             (int64_t)p.C << (l - 2), p.N, lane, p.variant);
                 else
-                    score = w.score_leaves(cand, need, Kh, p.C, p.N, lane);
+                    score = w.score_leaves(cand, need, Kh, p.C, p.N, lane, p.variant);
             }
         }
         int id = cand;

@@ -31,7 +31,7 @@ class PisaError(RuntimeError):
 
 class PisaCfg(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in
-                ("B", "Hq", "Hkv", "N", "d", "C", "K", "g", "causal", "forced_mask", "dtype")]
+                ("B", "Hq", "Hkv", "N", "d", "C", "K", "g", "causal", "forced_mask", "dtype", "score_variant")]
 
 
 _lock = threading.Lock()
@@ -93,17 +93,20 @@ def load(path: str | None = None):
         return lib
 
 
+PISA_SCORE_LSE, PISA_SCORE_MEAN, PISA_SCORE_MEAN_VAR = 0, 1, 2
+
+
 def make_cfg(*, B: int, Hq: int, Hkv: int, N: int, d: int, C: int, K: int, g: int = 2, causal: bool = True,
-             forced_mask: int = 7, dtype=torch.bfloat16) -> PisaCfg:
+             forced_mask: int = 7, dtype=torch.bfloat16, score_variant: int = PISA_SCORE_LSE) -> PisaCfg:
     dt = {torch.bfloat16: PISA_DTYPE_BF16, torch.float32: PISA_DTYPE_F32}.get(dtype, dtype)
-    return PisaCfg(B, Hq, Hkv, N, d, C, K, g, int(causal), forced_mask, int(dt))
+    return PisaCfg(B, Hq, Hkv, N, d, C, K, g, int(causal), forced_mask, int(dt), int(score_variant))
 
 
 def cfg_for(Q: torch.Tensor, K: torch.Tensor, *, C: int, K_: int, causal: bool = True, forced_mask: int = 7,
-            g: int = 2) -> PisaCfg:
+            g: int = 2, score_variant: int = PISA_SCORE_LSE) -> PisaCfg:
     B, Hq, N, d = Q.shape
     return make_cfg(B=B, Hq=Hq, Hkv=K.shape[1], N=N, d=d, C=C, K=K_, g=g, causal=causal,
-                    forced_mask=forced_mask, dtype=Q.dtype)
+                    forced_mask=forced_mask, dtype=Q.dtype, score_variant=score_variant)
 
 
 def _ptr(t: torch.Tensor | None):

@@ -53,6 +53,16 @@ extern "C" {
 
 enum pisa_dtype { PISA_DTYPE_F32 = 0, PISA_DTYPE_BF16 = 1 };
 
+/* Node score used for ranking (close reading §04 4.3). From the children's
+ * logits z_r = q . kbar_r / sqrt(d) (raw keys at the leaves), summed over a
+ * GQA group (Eq.11):
+ *   PISA_SCORE_LSE      Eq.(7): log sum_r exp(z_r) (the method; default);
+ *   PISA_SCORE_MEAN     PISA-1, Eq.(8) truncated: the mean of the z_r;
+ *   PISA_SCORE_MEAN_VAR PISA-2, Eq.(9): the mean plus half the population
+ *                       variance of the z_r.
+ * Only the ranking changes: attention always uses the exact softmax. */
+enum pisa_score { PISA_SCORE_LSE = 0, PISA_SCORE_MEAN = 1, PISA_SCORE_MEAN_VAR = 2 };
+
 enum pisa_status {
     PISA_OK = 0,
     PISA_E_INVALID = -1,      /* null pointer, bad size, inconsistent config */
@@ -76,6 +86,7 @@ typedef struct pisa_cfg {
     int32_t causal;       /* 1: causal mask and causal eligibility; 0: none */
     int32_t forced_mask;  /* bit0 first, bit1 previous, bit2 current leaf */
     int32_t dtype;        /* enum pisa_dtype of Q, K, V, O and the decode caches */
+    int32_t score_variant; /* enum pisa_score: how a node is ranked from its children */
 } pisa_cfg;
 
 /* ---- geometry (close reading §04 4.1, Eq.(3)) -------------------------------

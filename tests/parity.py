@@ -27,13 +27,14 @@ def tdtype(w):
     return torch.bfloat16 if w.dtype == "bf16" else torch.float32
 
 
-def gpu_prefill(w, Q, K, V, bsa: bool = False, ws: bool = False):
+def gpu_prefill(w, Q, K, V, bsa: bool = False, ws: bool = False, variant: int = 0):
     """Run pisa_forward (or, with ws=True, the block-major pisa_forward_ws) and
-    optionally pisa_bsa_select on cuda:0; returns GPU tensors."""
+    optionally pisa_bsa_select on cuda:0; returns GPU tensors. variant: the
+    node score (0 Eq.7 LSE, 1 PISA-1, 2 PISA-2)."""
     dev = torch.device("cuda", 0)
     Qd, Kd, Vd = Q.to(dev), K.to(dev), V.to(dev)
     cfg = pisa.make_cfg(B=w.B, Hq=w.Hq, Hkv=w.Hkv, N=Q.shape[2], d=w.d, C=w.C, K=w.K, g=w.g, causal=w.causal,
-                        forced_mask=w.forced_mask, dtype=Q.dtype)
+                        forced_mask=w.forced_mask, dtype=Q.dtype, score_variant=variant)
     pyr, idx, O = pisa.alloc_outputs(cfg, dev, Q.dtype)
     idx.fill_(-7)
     if ws:
@@ -95,7 +96,7 @@ def compare_indices(gpu_rows, ora_rows, gaps, t, w, N, what="select"):
     return len(t), exempt, same
 
 
-def check_head(w, Q, K, V, res, b, kvh, rows, check_bsa=False):
+def check_head(w, Q, K, V, res, b, kvh, rows, check_bsa=False, variant=0):
     """Check pyramid, selection and attention of one (b, kv-head) on query rows `rows`."""
     N = Q.shape[2]
     G = w.Hq // w.Hkv
@@ -108,7 +109,7 @@ def check_head(w, Q, K, V, res, b, kvh, rows, check_bsa=False):
     tt = torch.as_tensor(t)
     Qg = oracle.to_f64(Q[b, kvh * G:(kvh + 1) * G][:, tt]).transpose(1, 0, 2).copy()  # [n, G, d]
     idx_o, gap = oracle.select_rows(Qg, t, Kh, P, C=w.C, K=w.K, g=w.g, causal=w.causal,
-                                    forced_mask=w.forced_mask)
+                                    forced_mask=w.forced_mask, variant=variant)
     idx_g = res["idx"][b, kvh][tt.to(res["idx"].device)].cpu().numpy()
     n, ex, same = compare_indices(idx_g, idx_o, gap, t, w, N)
     # attention on the GPU's own indices, every head of the group

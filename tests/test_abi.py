@@ -68,6 +68,15 @@ def test_invalid_configs_are_rejected_before_launch(lib, field, value, status):
     assert _call_select(lib, cfg) == status
 
 
+def test_score_variant_is_validated(lib):
+    for v in (0, 1, 2):
+        cfg = pisa.make_cfg(B=1, Hq=2, Hkv=2, N=1000, d=128, C=64, K=8, score_variant=v)
+        assert lib.pisa_num_levels(ctypes.byref(cfg)) > 0
+    for v in (-1, 3):
+        cfg = pisa.make_cfg(B=1, Hq=2, Hkv=2, N=1000, d=128, C=64, K=8, score_variant=v)
+        assert lib.pisa_num_levels(ctypes.byref(cfg)) == -1
+
+
 def test_group_size_limits(lib):
     cfg = pisa.make_cfg(B=1, Hq=6, Hkv=2, N=256, d=128, C=16, K=4)   # G = 3
     assert _call_select(lib, cfg) == -2

@@ -21,12 +21,13 @@ def _cuda():
     pisa.load()
 
 
-def _cfg(w, B, cap):
+def _cfg(w, B, cap, variant=0):
     return pisa.make_cfg(B=B, Hq=w.Hq, Hkv=w.Hkv, N=cap, d=w.d, C=w.C, K=w.K, causal=True,
-                         forced_mask=w.forced_mask, dtype=torch.bfloat16 if w.dtype == "bf16" else torch.float32)
+                         forced_mask=w.forced_mask, dtype=torch.bfloat16 if w.dtype == "bf16" else torch.float32,
+                         score_variant=variant)
 
 
-def _check_seq(w, cap, Khost, Vhost, pyr_gpu, n, q, idx_g, o_g, check_pyr=True):
+def _check_seq(w, cap, Khost, Vhost, pyr_gpu, n, q, idx_g, o_g, check_pyr=True, variant=0):
     """One sequence after its token at position n was appended."""
     G = w.Hq // w.Hkv
     worst, exempt = 0.0, 0
@@ -43,7 +44,7 @@ def _check_seq(w, cap, Khost, Vhost, pyr_gpu, n, q, idx_g, o_g, check_pyr=True):
                                            rtol=1e-5, atol=2e-6)
         qg = oracle.to_f64(q[h * G:(h + 1) * G])[None]
         want, gap = oracle.select_rows(qg, np.array([n]), Kh, P, C=w.C, K=w.K, N=n + 1, N_layout=cap,
-                                       forced_mask=w.forced_mask)
+                                       forced_mask=w.forced_mask, variant=variant)
         got = idx_g[h].cpu().numpy()
         parity.check_row_valid(got, n, n + 1, w.C, w.K, True, w.forced_mask)
         if gap[0] >= parity.TIE_BAND:
