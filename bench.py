@@ -310,6 +310,7 @@ def main():
     ap.add_argument("--workload", default="mha8_n256k")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-bsa", action="store_true")
+    ap.add_argument("--no-variants", action="store_true", help="skip timing the PISA-1 / PISA-2 scores")
     ap.add_argument("--no-per-query", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=16.0)
@@ -471,35 +472,55 @@ def main():
         torch.cuda.synchronize()
         out["per_query_path_ms_per_step"] = e0.elapsed_time(e1)
 
-    # ---- end to end through the public API: pinned host -> device -> host ----
+    # ---- end to end through the C ABI with host buffers: pinned host -> device -> host ----
+    # pisa_forward_host copies the step's Q, K, V in, runs the step and copies
+    # idx and O out, all on one stream. Two sets of device buffers on two
+    # streams take alternate steps, so one step's copies overlap the other's
+    # kernels; every step's copies are inside the timed region.
     Qh, Kh, Vh = Q.pin_memory(), K.pin_memory(), V.pin_memory()
-    Oh = torch.empty(O.shape, dtype=O.dtype, pin_memory=True)
-    Ih = torch.empty(idx.shape, dtype=idx.dtype, pin_memory=True)
+    slots = []
+    for i in range(2):
+        if i == 0:
+            sQ, sK, sV, spyr, sidx, sO, swork = Qd, Kd, Vd, pyr, idx, O, work
+        else:
+            sQ, sK, sV = torch.empty_like(Qd), torch.empty_like(Kd), torch.empty_like(Vd)
+            spyr, sidx, sO = torch.empty_like(pyr), torch.empty_like(idx), torch.empty_like(O)
+            swork = pisa.alloc_workspace(cfg, dev)
+        slots.append({"dev": (sQ, sK, sV, spyr, sidx, sO, swork), "stream": torch.cuda.Stream(dev),
+                      "Oh": torch.empty(O.shape, dtype=O.dtype, pin_memory=True),
+                      "Ih": torch.empty(idx.shape, dtype=idx.dtype, pin_memory=True)})
 
-    def e2e_step():
-        Qd.copy_(Qh, non_blocking=True)
-        Kd.copy_(Kh, non_blocking=True)
-        Vd.copy_(Vh, non_blocking=True)
-        pisa.pisa_forward_ws(cfg, Qd, Kd, Vd, pyr, idx, O, work)
-        Oh.copy_(O, non_blocking=True)
-        Ih.copy_(idx, non_blocking=True)
+    def e2e_step(i):
+        sl = slots[i % 2]
+        sQ, sK, sV, spyr, sidx, sO, swork = sl["dev"]
+        with torch.cuda.stream(sl["stream"]):
+            pisa.pisa_forward_host(cfg, Qh, Kh, Vh, sl["Ih"], sl["Oh"], sQ, sK, sV, spyr, sidx, sO, swork)
 
-    for _ in range(2):
-        e2e_step()
+    def e2e_run(n):
+        start = torch.cuda.Event(enable_timing=True)
+        start.record(stream)
+        for sl in slots:
+            sl["stream"].wait_event(start)
+        for i in range(n):
+            e2e_step(i)
+        for sl in slots:
+            stream.wait_stream(sl["stream"])
+        end = torch.cuda.Event(enable_timing=True)
+        end.record(stream)
+        return start, end
+
+    e2e_run(2)
     torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    n_e2e = max(3, min(args.steps, 5))
-    e0.record(stream)
-    for _ in range(n_e2e):
-        e2e_step()
-    e1.record(stream)
+    n_e2e = max(4, min(args.steps, 6))
+    e0, e1 = e2e_run(n_e2e)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / n_e2e
     e2e_ms = max_over_ranks(e2e_ms, dist, dev)
     out["e2e"] = {"value": job_tokens_per_s(w.B * w.N, world, e2e_ms), "unit": unit,
                   "h2d_bytes_per_step": int(Qh.nbytes + Kh.nbytes + Vh.nbytes),
-                  "d2h_bytes_per_step": int(Oh.nbytes + Ih.nbytes), "ms_per_step": e2e_ms}
-    del Qh, Kh, Vh, Oh, Ih
+                  "d2h_bytes_per_step": int(O.nbytes + idx.nbytes), "ms_per_step": e2e_ms,
+                  "call": "pisa_forward_host", "pipelining": "2 buffer sets on 2 streams, alternate steps"}
+    del Qh, Kh, Vh, slots
 
     # ---- flat BSA selection, the quadratic comparison ----
     if not args.no_bsa:
@@ -517,6 +538,30 @@ def main():
         out["bsa_kernel"] = "per-query CUDA-core flat scan (bsa_kernel)"
         out["pisa_vs_bsa_selection_speedup"] = out["bsa_selection_ms"] / sel_total
         del bidx
+
+    # ---- the same step ranking by the PISA-1 / PISA-2 scores (Eq.8-9 ablations) ----
+    if not args.no_variants:
+        vout = {}
+        for vname, v in (("pisa1_mean", pisa.PISA_SCORE_MEAN), ("pisa2_mean_var", pisa.PISA_SCORE_MEAN_VAR)):
+            vcfg = pisa.cfg_for(Qd, Kd, C=w.C, K_=w.K, causal=w.causal, forced_mask=w.forced_mask, score_variant=v)
+            vwork = pisa.alloc_workspace(vcfg, dev)
+            for _ in range(2):
+                pisa.pisa_forward_ws(vcfg, Qd, Kd, Vd, pyr, idx, O, vwork)
+            torch.cuda.synchronize()
+            vev = [[torch.cuda.Event(enable_timing=True) for _ in range(nph + 1)] for _ in range(3)]
+            for e in vev:
+                for x in e:
+                    x.record(stream)
+            torch.cuda.synchronize()
+            for e in vev:
+                pisa.pisa_forward_ws_events(vcfg, Qd, Kd, Vd, pyr, idx, O, vwork, e)
+            torch.cuda.synchronize()
+            vms = max_over_ranks(vev[0][0].elapsed_time(vev[-1][nph]) / len(vev), dist, dev)
+            vout[vname] = {"ms_per_step": vms, "tokens_per_s": job_tokens_per_s(w.B * w.N, world, vms),
+                           "phase_ms": {name: float(np.mean([e[i].elapsed_time(e[i + 1]) for e in vev]))
+                                        for i, name in enumerate(pisa.PHASES)}}
+            del vwork
+        out["score_variants"] = vout
 
     # ---- decode: 64 sequences, one new token each, against 256K-key caches ----
     if not args.no_decode and w.decode_batch:

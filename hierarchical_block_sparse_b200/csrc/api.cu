@@ -302,6 +302,31 @@ int pisa_forward_ws_events(const pisa_cfg* cfg, const void* Q, const void* K, co
     return cuda_status(launch_attn_bm(Q, K, V, idx, O, sp, sh, workspace, true, &ev, st));
 }
 
+int pisa_forward_host(const pisa_cfg* cfg, const void* Q_host, const void* K_host, const void* V_host,
+                      int32_t* idx_host, void* O_host, void* Q, void* K, void* V, float* pyr, int32_t* idx,
+                      void* O, void* workspace, size_t workspace_bytes, void* stream) {
+    int s = check_bm(cfg);
+    if (s) return s;
+    if (cfg->N == 0) return PISA_OK;
+    if (!Q_host || !K_host || !V_host || !idx_host || !O_host) return PISA_E_INVALID;
+    const size_t es = cfg->dtype == PISA_DTYPE_BF16 ? 2 : 4;
+    const size_t q_bytes = (size_t)cfg->B * cfg->Hq * cfg->N * cfg->d * es;
+    const size_t kv_bytes = (size_t)cfg->B * cfg->Hkv * cfg->N * cfg->d * es;
+    const size_t idx_bytes = (size_t)cfg->B * cfg->Hkv * cfg->N * cfg->K * sizeof(int32_t);
+    cudaStream_t st = (cudaStream_t)stream;
+    if (!Q || !K || !V) return PISA_E_INVALID;
+    if (cudaMemcpyAsync(Q, Q_host, q_bytes, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+        cudaMemcpyAsync(K, K_host, kv_bytes, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+        cudaMemcpyAsync(V, V_host, kv_bytes, cudaMemcpyHostToDevice, st) != cudaSuccess)
+        return PISA_E_CUDA;
+    s = pisa_forward_ws(cfg, Q, K, V, pyr, idx, O, workspace, workspace_bytes, stream);
+    if (s) return s;
+    if (cudaMemcpyAsync(idx_host, idx, idx_bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+        cudaMemcpyAsync(O_host, O, q_bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+        return PISA_E_CUDA;
+    return PISA_OK;
+}
+
 int pisa_forward_ws(const pisa_cfg* cfg, const void* Q, const void* K, const void* V, float* pyr, int32_t* idx,
                     void* O, void* workspace, size_t workspace_bytes, void* stream) {
     return pisa_forward_ws_events(cfg, Q, K, V, pyr, idx, O, workspace, workspace_bytes, nullptr, 0, stream);

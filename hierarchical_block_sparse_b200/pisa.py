@@ -75,6 +75,7 @@ def load(path: str | None = None):
             "pisa_select_ws": (ctypes.c_int, [cfgp, P, P, P, P, P, ctypes.c_size_t, P]),
             "pisa_sparse_attn_ws": (ctypes.c_int, [cfgp, P, P, P, P, P, P, ctypes.c_size_t, P]),
             "pisa_forward_ws": (ctypes.c_int, [cfgp, P, P, P, P, P, P, P, ctypes.c_size_t, P]),
+            "pisa_forward_host": (ctypes.c_int, [cfgp, P, P, P, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]),
             "pisa_forward_ws_events": (ctypes.c_int, [cfgp, P, P, P, P, P, P, P, ctypes.c_size_t,
                                                       ctypes.POINTER(ctypes.c_void_p), ctypes.c_int, P]),
             "pisa_select_noalloc": (ctypes.c_int, [cfgp, P, P, P, P, P]),
@@ -114,6 +115,14 @@ def _ptr(t: torch.Tensor | None):
         return None
     if not t.is_cuda:
         raise ValueError("tensors must live on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _host_ptr(t: torch.Tensor):
+    if t.is_cuda:
+        raise ValueError("host buffers must live in host memory")
     if not t.is_contiguous():
         raise ValueError("tensors must be contiguous")
     return ctypes.c_void_p(t.data_ptr())
@@ -205,6 +214,14 @@ def pisa_sparse_attn_ws(cfg, Q, K, V, idx, O, ws):
 def pisa_forward_ws(cfg, Q, K, V, pyr, idx, O, ws):
     _check("pisa_forward_ws", load().pisa_forward_ws(ctypes.byref(cfg), _ptr(Q), _ptr(K), _ptr(V), _ptr(pyr),
                                                      _ptr(idx), _ptr(O), _ptr(ws), ws.numel(), _stream()))
+
+
+def pisa_forward_host(cfg, Q_host, K_host, V_host, idx_host, O_host, Q, K, V, pyr, idx, O, ws):
+    """pisa_forward_ws from host buffers (pinned for asynchronous copies) on the current stream."""
+    _check("pisa_forward_host", load().pisa_forward_host(
+        ctypes.byref(cfg), _host_ptr(Q_host), _host_ptr(K_host), _host_ptr(V_host), _host_ptr(idx_host),
+        _host_ptr(O_host), _ptr(Q), _ptr(K), _ptr(V), _ptr(pyr), _ptr(idx), _ptr(O), _ptr(ws), ws.numel(),
+        _stream()))
 
 
 def pisa_select_noalloc(cfg, Q, K, pyr, idx):

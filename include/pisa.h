@@ -183,6 +183,19 @@ int pisa_sparse_attn_ws(const pisa_cfg *cfg, const void *Q, const void *K, const
 int pisa_forward_ws(const pisa_cfg *cfg, const void *Q, const void *K, const void *V, float *pyr, int32_t *idx,
                     void *O, void *workspace, size_t workspace_bytes, void *stream);
 
+/* pisa_forward_ws from and to HOST memory: copies Q_host, K_host, V_host
+ * (layouts as above) into the caller's device buffers Q, K, V, runs
+ * pisa_forward_ws, and copies idx and O back into idx_host and O_host, all
+ * enqueued on `stream` (one cudaMemcpyAsync per tensor). The host buffers
+ * should be page-locked (cudaHostAlloc / pinned) for the copies to be
+ * asynchronous; the call returns before they complete. Callers that keep two
+ * sets of device buffers on two streams overlap one step's copies with the
+ * other step's kernels. Same limits and errors as pisa_forward_ws; null host
+ * pointers give PISA_E_INVALID. */
+int pisa_forward_host(const pisa_cfg *cfg, const void *Q_host, const void *K_host, const void *V_host,
+                      int32_t *idx_host, void *O_host, void *Q, void *K, void *V, float *pyr, int32_t *idx,
+                      void *O, void *workspace, size_t workspace_bytes, void *stream);
+
 /* pisa_forward_ws that also records caller-created CUDA events (cudaEvent_t
  * passed as void*, NULL entries skipped) on `stream` at its phase boundaries,
  * for per-phase timing with cudaEventElapsedTime. Index i marks the start of

@@ -106,3 +106,22 @@ def test_workspace_errors():
     with pytest.raises(pisa.PisaError):
         pisa.pisa_workspace_bytes(bad)
     _ = w
+
+
+def test_forward_host_equals_forward_ws():
+    # pisa_forward_host: the same step from pinned host buffers, copies on the stream
+    w = SMALL["bm_ragged"]
+    Q, K, V, _ = make_inputs(w)
+    res = parity.gpu_prefill(w, Q, K, V, ws=True)
+    dev = torch.device("cuda", 0)
+    cfg = res["cfg"]
+    Qd, Kd, Vd = torch.empty_like(Q, device=dev), torch.empty_like(K, device=dev), torch.empty_like(V, device=dev)
+    pyr, idx, O = pisa.alloc_outputs(cfg, dev, Q.dtype)
+    work = pisa.alloc_workspace(cfg, dev)
+    Ih = torch.full(idx.shape, -7, dtype=idx.dtype).pin_memory()
+    Oh = torch.zeros(O.shape, dtype=O.dtype).pin_memory()
+    pisa.pisa_forward_host(cfg, Q.pin_memory(), K.pin_memory(), V.pin_memory(), Ih, Oh, Qd, Kd, Vd, pyr, idx, O,
+                           work)
+    torch.cuda.synchronize()
+    assert torch.equal(Ih, res["idx"].cpu())
+    assert torch.equal(Oh, res["O"].cpu())
