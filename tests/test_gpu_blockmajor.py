@@ -124,4 +124,6 @@ def test_forward_host_equals_forward_ws():
                            work)
     torch.cuda.synchronize()
     assert torch.equal(Ih, res["idx"].cpu())
-    assert torch.equal(Oh, res["O"].cpu())
+    # the attention tiles add fp32 partial outputs in an order that varies from
+    # run to run, so O agrees to rounding, not bit for bit
+    assert float((Oh.float() - res["O"].float().cpu()).abs().max()) <= parity.O_TOL[w.dtype]
