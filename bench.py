@@ -138,21 +138,33 @@ def algorithmic(w, N: int):
     }
 
 
-def source_sha(files):
+def source_sha(parts):
+    """Hash of a kernel's sources: whole files, or (file, section) pairs for the
+    section of a file that starts at a "// ---- <section> ----" marker line and
+    ends at the next marker."""
     h = hashlib.sha256()
-    for f in files:
-        h.update(open(os.path.join(ROOT, f), "rb").read())
+    for part in parts:
+        f, section = (part, None) if isinstance(part, str) else part
+        text = open(os.path.join(ROOT, f), encoding="utf-8").read()
+        if section is not None:
+            lines = text.splitlines(keepends=True)
+            marks = [i for i, ln in enumerate(lines) if ln.startswith("// ---") and ln.rstrip().endswith("----")]
+            start = next(i for i in marks if section in lines[i])
+            end = next((i for i in marks if i > start), len(lines))
+            text = "".join(lines[start:end])
+        h.update(text.encode())
     return h.hexdigest()[:16]
 
 
 _CS = "hierarchical_block_sparse_b200/csrc/"
-_BM = [_CS + "blockmajor.cu", _CS + "pisa_internal.h"]
+_BMF = _CS + "blockmajor.cu"
+_TILE = [(_BMF, "tile plumbing"), _CS + "tc.cuh", _CS + "pisa_internal.h"]
 KERNEL_SOURCES = {
-    "stage1": _BM + [_CS + "pisa_stage1.cuh", _CS + "pisa_walk.cuh", _CS + "pisa_device.cuh"],
-    "leaf_scores": _BM + [_CS + "tc.cuh"],
-    "attn_tiles": _BM + [_CS + "tc.cuh"],
-    "forced_tiles": _BM + [_CS + "tc.cuh"],
-    "topk": _BM + [_CS + "pisa_walk.cuh", _CS + "pisa_device.cuh"],
+    "stage1": [(_BMF, "stage 1"), _CS + "pisa_stage1.cuh", _CS + "pisa_walk.cuh", _CS + "pisa_device.cuh"],
+    "leaf_scores": [(_BMF, "stage 2: leaf LSEs")] + _TILE,
+    "topk": [(_BMF, "final Top-K"), _CS + "pisa_walk.cuh", _CS + "pisa_device.cuh"],
+    "attn_tiles": [(_BMF, "attention tiles")] + _TILE,
+    "forced_tiles": [(_BMF, "forced leaves, dense")] + _TILE,
     "pool": [_CS + "pool.cu", _CS + "pisa_device.cuh"],
     "select": [_CS + "select.cu", _CS + "pisa_walk.cuh", _CS + "pisa_device.cuh"],
     "attn": [_CS + "attn.cu", _CS + "pisa_attn.cuh", _CS + "pisa_walk.cuh", _CS + "pisa_device.cuh"],

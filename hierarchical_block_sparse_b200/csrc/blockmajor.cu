@@ -403,7 +403,7 @@ struct TileParams {
 // and its entries are sibling-pair slots i; the 128 keys of leaves 2p and 2p+1
 // are scored by one N = 128 MMA and each non-forced visible leaf's LSE goes to
 // slot 2i or 2i+1.
-template <int G, bool PAIR>
+template <int G, bool PAIR, bool VSCORE = false>
 __global__ void __launch_bounds__(128) leaf_score_kernel(const __nv_bfloat16* __restrict__ Q,
                                                          const __nv_bfloat16* __restrict__ Kmat,
                                                          const int4* __restrict__ tiles,
@@ -488,7 +488,7 @@ __global__ void __launch_bounds__(128) leaf_score_kernel(const __nv_bfloat16* __
                     if (j < nvalid) s += exp2f(v[j] * p.qscale - m);
                 const int64_t unit = bh * p.N + t;
                 lse[(unit * kSlots + slot) * G + (tid % G)] = m + log2f(s);
-                if (vscore) {  // PISA-1 / PISA-2 ranking score: two-pass mean and variance of the logits
+                if constexpr (VSCORE) {  // PISA-1 / PISA-2 ranking score: two-pass mean and variance of the logits
                     float sum = 0.f;
 #pragma unroll
                     for (int j = 0; j < 64; ++j)
@@ -1116,20 +1116,30 @@ constexpr size_t kAttnSmem = 72 * 1024;
 static_assert(128 * kORowStride <= kAttnSmem, "the staged output tile fits in the attention tile's buffers");
 constexpr int kAttnCtasPerSm = 3;
 
-template <int G, bool PAIR>
-static cudaError_t leaf_scores(const void* Q, const void* K, const SelectParams& sp, const BmShape& s, uint8_t* ws,
-                               const BmLayout& L, cudaStream_t st) {
+template <int G, bool PAIR, bool VSCORE>
+static cudaError_t leaf_scores_t(const void* Q, const void* K, const SelectParams& sp, const BmShape& s, uint8_t* ws,
+                                 const BmLayout& L, cudaStream_t st) {
     TileParams tp{s.B, s.Hq, s.Hkv, s.N, sp.causal, s.M1, sp.qscale, max_tiles_of(s), sp.variant};
     constexpr size_t smem = 32768 + (PAIR ? 32768 : 16384);
-    auto kern = leaf_score_kernel<G, PAIR>;
+    auto kern = leaf_score_kernel<G, PAIR, VSCORE>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     kern<<<sm_count() * (PAIR ? 3 : 4), 128, smem, st>>>((const __nv_bfloat16*)Q, (const __nv_bfloat16*)K,
                                                           (const int4*)(ws + L.tiles), (const int32_t*)(ws + L.misc),
                                                           (const uint32_t*)(ws + L.entries), (float*)(ws + L.lse),
-                                                          (PAIR && sp.variant) ? (float*)(ws + L.vscore) : nullptr,
+                                                          VSCORE ? (float*)(ws + L.vscore) : nullptr,
                                                           (int*)(ws + L.misc) + 1, tp, sp.forced_mask);
     return cudaGetLastError();
+}
+
+// leaf LSEs (and, for the sibling-pair ranking pass with a PISA-1 / PISA-2
+// score, the ranking scores: a separate instantiation, so the default pass
+// keeps its registers)
+template <int G, bool PAIR>
+static cudaError_t leaf_scores(const void* Q, const void* K, const SelectParams& sp, const BmShape& s, uint8_t* ws,
+                               const BmLayout& L, cudaStream_t st) {
+    if (PAIR && sp.variant) return leaf_scores_t<G, PAIR, true>(Q, K, sp, s, ws, L, st);
+    return leaf_scores_t<G, PAIR, false>(Q, K, sp, s, ws, L, st);
 }
 
 template <int G>
