@@ -343,6 +343,26 @@ int pisa_build_pyramid_prefix(const pisa_cfg* cfg, const void* Kc, const int32_t
     return cuda_status(launch_pool(cfg->dtype, cfg->d, Kc, pyr, pool_params(cfg, g, len), (cudaStream_t)stream));
 }
 
+int pisa_pyramid_grow(const pisa_cfg* cfg_old, const float* pyr_old, const pisa_cfg* cfg_new, float* pyr_new,
+                      void* stream) {
+    int s = check_gpu(cfg_old);
+    if (s) return s;
+    s = check_gpu(cfg_new);
+    if (s) return s;
+    if (cfg_old->B != cfg_new->B || cfg_old->Hq != cfg_new->Hq || cfg_old->Hkv != cfg_new->Hkv ||
+        cfg_old->d != cfg_new->d || cfg_old->C != cfg_new->C || cfg_old->g != cfg_new->g ||
+        cfg_old->dtype != cfg_new->dtype || cfg_new->N < cfg_old->N)
+        return PISA_E_INVALID;
+    if (cfg_old->N == 0) return PISA_OK;
+    if (!pyr_old || !pyr_new || pyr_old == pyr_new) return PISA_E_INVALID;
+    if (!aligned16(pyr_old) || !aligned16(pyr_new)) return PISA_E_ALIGNMENT;
+    Geom go, gn;
+    make_geom(cfg_old->N, cfg_old->C, &go);
+    make_geom(cfg_new->N, cfg_new->C, &gn);
+    return cuda_status(launch_pyramid_grow(pyr_old, pyr_new, (int64_t)cfg_new->B * cfg_new->Hkv, cfg_new->d, go, gn,
+                                           (cudaStream_t)stream));
+}
+
 int pisa_pyramid_append(const pisa_cfg* cfg, void* Kc, void* Vc, float* pyr, const void* k_new, const void* v_new,
                         const int32_t* pos, void* stream) {
     int s = check_gpu(cfg);

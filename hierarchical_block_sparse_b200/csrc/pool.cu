@@ -131,6 +131,37 @@ static cudaError_t launch_pool_t(const void* K, float* pyr, const PoolParams& p,
     return e;
 }
 
+// Pyramid cache growth (close reading §5.3, decode cache: the capacity grows by
+// a fixed ratio). Row r of the new layout (level l, node i) takes old row
+// (l, i) when that node exists in the old layout; node 0 of a level above the
+// old root takes the old root (its second child starts past the old capacity,
+// so at any length the old layout can hold it is the mean of one node: the
+// old root); every other row is zero until tokens reach it. One warp per row.
+__global__ void __launch_bounds__(256) pyramid_grow_kernel(const float* __restrict__ old_pyr,
+                                                           float* __restrict__ new_pyr, int64_t units, int d,
+                                                           Geom go, Geom gn) {
+    const int lane = threadIdx.x & 31;
+    const int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (row >= units * gn.rows) return;
+    const int64_t u = row / gn.rows, r = row - u * gn.rows;
+    int l = 1;
+    while (l < gn.L && r >= gn.off[l + 1]) ++l;
+    const int64_t i = r - gn.off[l];
+    int64_t src = -1;
+    if (l <= go.L && i < go.M[l]) src = go.off[l] + i;
+    else if (l > go.L && i == 0) src = go.off[go.L];
+    const float* from = old_pyr + (u * go.rows + (src < 0 ? 0 : src)) * d;
+    float* to = new_pyr + row * d;
+    for (int e = lane; e < d; e += 32) to[e] = src >= 0 ? from[e] : 0.f;
+}
+
+cudaError_t launch_pyramid_grow(const float* old_pyr, float* new_pyr, int64_t units, int d, const Geom& go,
+                                const Geom& gn, cudaStream_t st) {
+    const int64_t rows = units * gn.rows;
+    pyramid_grow_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(old_pyr, new_pyr, units, d, go, gn);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_pool(int dtype, int d, const void* K, float* pyr, const PoolParams& p, cudaStream_t st) {
     if (dtype == 1) {
         if (d == 128) return launch_pool_t<__nv_bfloat16, 128>(K, pyr, p, st);

@@ -81,6 +81,7 @@ def load(path: str | None = None):
             "pisa_select_noalloc": (ctypes.c_int, [cfgp, P, P, P, P, P]),
             "pisa_build_pyramid_prefix": (ctypes.c_int, [cfgp, P, P, P, P]),
             "pisa_pyramid_append": (ctypes.c_int, [cfgp, P, P, P, P, P, P, P]),
+            "pisa_pyramid_grow": (ctypes.c_int, [cfgp, P, cfgp, P, P]),
             "pisa_decode": (ctypes.c_int, [cfgp, P, P, P, P, P, P, P, P]),
             "pisa_decode_step": (ctypes.c_int, [cfgp, P, P, P, P, P, P, P, P, P, P]),
             "pisa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -258,6 +259,11 @@ def pisa_build_pyramid_prefix(cfg, Kc, length, pyr):
 def pisa_pyramid_append(cfg, Kc, Vc, pyr, k_new, v_new, pos):
     _check("pisa_pyramid_append", load().pisa_pyramid_append(ctypes.byref(cfg), _ptr(Kc), _ptr(Vc), _ptr(pyr),
                                                              _ptr(k_new), _ptr(v_new), _ptr(pos), _stream()))
+
+
+def pisa_pyramid_grow(cfg_old, pyr_old, cfg_new, pyr_new):
+    _check("pisa_pyramid_grow", load().pisa_pyramid_grow(ctypes.byref(cfg_old), _ptr(pyr_old), ctypes.byref(cfg_new),
+                                                         _ptr(pyr_new), _stream()))
 
 
 def pisa_decode(cfg, q_new, Kc, Vc, pyr, pos, idx, o):

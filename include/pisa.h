@@ -240,6 +240,19 @@ int pisa_select_noalloc(const pisa_cfg *cfg, const void *Q, const void *K, const
 int pisa_build_pyramid_prefix(const pisa_cfg *cfg, const void *Kc, const int32_t *len,
                               float *pyr, void *stream);
 
+/* Grow a decode pyramid cache (close reading §5.3: the cache's capacity grows
+ * by a fixed ratio as tokens arrive; the caller picks the new capacity, e.g.
+ * twice the old one). pyr_old is laid out for cfg_old->N, pyr_new (a separate
+ * caller buffer of pisa_pyramid_rows(cfg_new) rows per (b, kv-head)) for
+ * cfg_new->N >= cfg_old->N; every other cfg field must match. Every summary of
+ * the old pyramid, for any lengths up to the old capacity, lands where the
+ * new layout keeps it (the levels added above the old root repeat the old
+ * root); rows past the old capacity are zeroed. The caller copies its K/V
+ * cache rows into caches of the new capacity itself. Mismatched configs, a
+ * smaller new capacity or pyr_new == pyr_old give PISA_E_INVALID. */
+int pisa_pyramid_grow(const pisa_cfg *cfg_old, const float *pyr_old, const pisa_cfg *cfg_new, float *pyr_new,
+                      void *stream);
+
 /* Append one token per sequence: k_new, v_new [B, Hkv, d] are written to cache
  * row pos[b]; the leaf holding pos[b] and each of its ancestors is recomputed
  * as the mean of what exists at length pos[b] + 1 (O(C + L) work per head). */

@@ -32,7 +32,7 @@ MAX_LEVELS = 64
 
 __all__ = [
     "build_oracle", "geometry", "total_nodes", "build_pyramid", "pyramid_append",
-    "select_rows", "flat_rows", "attn_rows", "node_score", "threads",
+    "select_rows", "flat_rows", "attn_rows", "attn_backward_rows", "node_score", "threads",
     "to_f64", "MAX_LEVELS",
 ]
 
@@ -220,3 +220,51 @@ def attn_rows(Qrows: np.ndarray, t: np.ndarray, Kh: np.ndarray, Vh: np.ndarray, 
     _load().oracle_attn_rows(N, d, C, K, int(causal), _p(Kh), _p(Vh), n, _p(t), _p(Qrows),
                              _p(idx), _p(O), _p(lse))
     return (O, lse) if want_lse else O
+
+
+def attn_backward_rows(Qg: np.ndarray, Kh: np.ndarray, Vh: np.ndarray, idx: np.ndarray, dOg: np.ndarray, *,
+                       C: int, causal: bool = True):
+    """Backward of Eq.(2) over fixed selected leaves (close reading §5.3: the
+    gradient flows only through the selected attention entries), for one KV
+    head and its G query heads, every position 0..N-1.
+
+    Qg, dOg: [G, N, d]; Kh, Vh: [N, d]; idx: [N, K] selected leaves (-1 pads).
+    Per query row: s = q k_J / sqrt(d) over the keys J of its leaves (j <= t
+    when causal), p = softmax(s), o = p V_J; then dV_J += p dO, dp = V_J dO,
+    ds = p (dp - dO . o), dq = ds K_J / sqrt(d), dK_J += ds q / sqrt(d).
+    Returns (dQ [G, N, d], dK [N, d], dV [N, d]) in float64 (plain numpy, a
+    loop over rows: small cases only)."""
+    Qg = np.asarray(Qg, np.float64)
+    dOg = np.asarray(dOg, np.float64)
+    Kh = np.asarray(Kh, np.float64)
+    Vh = np.asarray(Vh, np.float64)
+    G, N, d = Qg.shape
+    inv = 1.0 / np.sqrt(d)
+    dQ = np.zeros_like(Qg)
+    dK = np.zeros_like(Kh)
+    dV = np.zeros_like(Vh)
+    for t in range(N):
+        J = []
+        for leaf in idx[t]:
+            if leaf < 0:
+                continue
+            hi = min((int(leaf) + 1) * C, N)
+            if causal:
+                hi = min(hi, t + 1)
+            J.extend(range(int(leaf) * C, hi))
+        J = np.array(sorted(J), np.int64)
+        if J.size == 0:
+            continue
+        KJ, VJ = Kh[J], Vh[J]
+        for h in range(G):
+            s = KJ @ Qg[h, t] * inv
+            p = np.exp(s - s.max())
+            p /= p.sum()
+            o = p @ VJ
+            do = dOg[h, t]
+            dV[J] += np.outer(p, do)
+            dp = VJ @ do
+            ds = p * (dp - do @ o)
+            dQ[h, t] = ds @ KJ * inv
+            dK[J] += np.outer(ds, Qg[h, t]) * inv
+    return dQ, dK, dV

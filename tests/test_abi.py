@@ -68,6 +68,19 @@ def test_invalid_configs_are_rejected_before_launch(lib, field, value, status):
     assert _call_select(lib, cfg) == status
 
 
+def test_pyramid_grow_validates_before_launch(lib):
+    old = pisa.make_cfg(B=2, Hq=2, Hkv=2, N=2048, d=128, C=64, K=8)
+    P = ctypes.c_void_p(4096)
+    for field, value in (("N", 1024), ("C", 32), ("Hkv", 1), ("d", 64)):
+        new = pisa.make_cfg(B=2, Hq=2, Hkv=2, N=4096, d=128, C=64, K=8)
+        setattr(new, field, value)
+        assert lib.pisa_pyramid_grow(ctypes.byref(old), P, ctypes.byref(new), ctypes.c_void_p(8192), None) == -1
+    new = pisa.make_cfg(B=2, Hq=2, Hkv=2, N=4096, d=128, C=64, K=8)
+    assert lib.pisa_pyramid_grow(ctypes.byref(old), P, ctypes.byref(new), P, None) == -1          # in place
+    assert lib.pisa_pyramid_grow(ctypes.byref(old), None, ctypes.byref(new), P, None) == -1       # null
+    assert lib.pisa_pyramid_grow(ctypes.byref(old), ctypes.c_void_p(4104), ctypes.byref(new), P, None) == -4
+
+
 def test_score_variant_is_validated(lib):
     for v in (0, 1, 2):
         cfg = pisa.make_cfg(B=1, Hq=2, Hkv=2, N=1000, d=128, C=64, K=8, score_variant=v)

@@ -158,3 +158,54 @@ def test_decode_full_size_sampled():
         Kh = torch.cat([decode_rows(Kp, s, prefix), k[s][:, None]], 1)
         Vh = torch.cat([decode_rows(Vp, s, prefix), v[s][:, None]], 1)
         _check_seq(w, cap, Kh, Vh, pyr[s], prefix, q[s], idx[s], o[s], check_pyr=(s == 0))
+
+
+def test_pyramid_grow_then_decode_past_the_old_capacity():
+    # the decode cache outgrows its capacity: the pyramid is re-laid out for
+    # twice the capacity (pisa_pyramid_grow), the caller copies its K/V rows,
+    # and decoding continues past the old capacity
+    w = Workload("dec_grow", 122, B=1, Hq=2, Hkv=2, N=0, d=128, C=64, K=8, decode_batch=2)
+    cap_old, cap_new = 2048, 4096
+    lens = [1500, 2045]
+    dev = torch.device("cuda", 0)
+    Kc, Vc, Kp, Vp = decode_cache(w, cap_old, 2047, dev)
+    Khost = [decode_rows(Kp, s, 2047) for s in range(2)]
+    Vhost = [decode_rows(Vp, s, 2047) for s in range(2)]
+    for s in range(2):
+        Kc[s, :, lens[s]:] = 0
+        Vc[s, :, lens[s]:] = 0
+    cfg_old, cfg_new = _cfg(w, 2, cap_old), _cfg(w, 2, cap_new)
+    pyr_old = torch.zeros((2, w.Hkv, pisa.pisa_pyramid_rows(cfg_old), w.d), dtype=torch.float32, device=dev)
+    pos = torch.tensor(lens, dtype=torch.int32, device=dev)
+    pisa.pisa_build_pyramid_prefix(cfg_old, Kc, pos, pyr_old)
+    pyr = torch.full((2, w.Hkv, pisa.pisa_pyramid_rows(cfg_new), w.d), float("nan"), dtype=torch.float32, device=dev)
+    pisa.pisa_pyramid_grow(cfg_old, pyr_old, cfg_new, pyr)
+    torch.cuda.synchronize()
+    L, _, off = oracle.geometry(cap_new, w.C)
+    for s in range(2):  # the grown layout holds the same summaries as a rebuild for cap_new
+        for h in range(w.Hkv):
+            Kh = oracle.to_f64(Khost[s][h, : lens[s]])
+            P = oracle.build_pyramid(Kh, w.C, N=lens[s], N_layout=cap_new)
+            gp = oracle.to_f64(pyr[s, h])
+            for lvl in range(1, L + 1):
+                live = -(-lens[s] // (w.C * 2 ** (lvl - 1)))
+                np.testing.assert_allclose(gp[off[lvl]:off[lvl] + live], P[off[lvl]:off[lvl] + live],
+                                           rtol=1e-5, atol=2e-6)
+    Kc2 = torch.zeros((2, w.Hkv, cap_new, w.d), dtype=Kc.dtype, device=dev)
+    Vc2 = torch.zeros_like(Kc2)
+    Kc2[:, :, :cap_old] = Kc
+    Vc2[:, :, :cap_old] = Vc
+    for step in range(6):  # sequence 1 crosses position 2048
+        q, k, v = decode_step_inputs(w, step, B=2)
+        idx = torch.full((2, w.Hkv, w.K), -7, dtype=torch.int32, device=dev)
+        o = torch.empty((2, w.Hq, w.d), dtype=q.dtype, device=dev)
+        pisa.pisa_decode_step(cfg_new, q.to(dev), k.to(dev), v.to(dev), Kc2, Vc2, pyr, pos, idx, o)
+        torch.cuda.synchronize()
+        for s in range(2):
+            n = int(pos[s])
+            Kh = torch.cat([Khost[s][:, :n], k[s][:, None]], 1)
+            Vh = torch.cat([Vhost[s][:, :n], v[s][:, None]], 1)
+            Khost[s], Vhost[s] = Kh, Vh
+            _check_seq(w, cap_new, Kh, Vh, pyr[s], n, q[s], idx[s], o[s])
+        pos += 1
+    assert int(pos[1]) > cap_old
