@@ -323,6 +323,7 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-bsa", action="store_true")
     ap.add_argument("--no-variants", action="store_true", help="skip timing the PISA-1 / PISA-2 scores")
+    ap.add_argument("--no-backward", action="store_true", help="skip timing the attention backward")
     ap.add_argument("--no-per-query", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=16.0)
@@ -574,6 +575,33 @@ def main():
                                         for i, name in enumerate(pisa.PHASES)}}
             del vwork
         out["score_variants"] = vout
+
+    # ---- backward of the attention with the selection fixed (dQ, dK, dV) ----
+    if not args.no_backward:
+        gen = torch.Generator(device=dev).manual_seed(w.seed + 17)
+        dOd = torch.randn(Qd.shape, generator=gen, device=dev, dtype=torch.float32).to(Qd.dtype)
+        dQ = torch.empty(Qd.shape, dtype=torch.float32, device=dev)
+        dK = torch.empty(Kd.shape, dtype=torch.float32, device=dev)
+        dV = torch.empty(Vd.shape, dtype=torch.float32, device=dev)
+        pisa.pisa_sparse_attn_backward(cfg, Qd, Kd, Vd, idx, dOd, dQ, dK, dV)
+        torch.cuda.synchronize()
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n_bwd = 2
+        g0.record(stream)
+        for _ in range(n_bwd):
+            pisa.pisa_sparse_attn_backward(cfg, Qd, Kd, Vd, idx, dOd, dQ, dK, dV)
+        g1.record(stream)
+        torch.cuda.synchronize()
+        bms = max_over_ranks(g0.elapsed_time(g1) / n_bwd, dist, dev)
+        # per attended (query head, key): 4d FLOP to recompute the softmax and
+        # the output, 10d for the logits again, dP, dQ, dK and dV
+        bflops = alg["attn_flops"] * 14.0 / 4.0
+        out["backward"] = {"ms": bms, "tokens_per_s": job_tokens_per_s(w.B * w.N, world, bms),
+                           "kernel": "attn_bwd_kernel (per-query warps, CUDA cores, fp32 dK/dV reductions)",
+                           "algorithmic_tflop": bflops / 1e12, "achieved_tflops": bflops / (bms / 1e3) / 1e12,
+                           "fp32_fma_peak_tflops": fma_peak,
+                           "frac": bflops / (bms / 1e3) / 1e12 / fma_peak}
+        del dOd, dQ, dK, dV
 
     # ---- decode: 64 sequences, one new token each, against 256K-key caches ----
     if not args.no_decode and w.decode_batch:

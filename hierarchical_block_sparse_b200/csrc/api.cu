@@ -198,6 +198,26 @@ int pisa_sparse_attn(const pisa_cfg* cfg, const void* Q, const void* K, const vo
     return cuda_status(launch_attn(cfg->dtype, cfg->d, Q, K, V, idx, O, p, (cudaStream_t)stream));
 }
 
+int pisa_sparse_attn_backward(const pisa_cfg* cfg, const void* Q, const void* K, const void* V, const int32_t* idx,
+                              const void* dO, float* dQ, float* dK, float* dV, void* stream) {
+    int s = check_gpu(cfg);
+    if (s) return s;
+    if (cfg->N == 0) return PISA_OK;
+    if (!Q || !K || !V || !idx || !dO || !dQ || !dK || !dV) return PISA_E_INVALID;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(idx) || !aligned16(dO) || !aligned16(dQ) ||
+        !aligned16(dK) || !aligned16(dV))
+        return PISA_E_ALIGNMENT;
+    const size_t kv_bytes = (size_t)cfg->B * cfg->Hkv * cfg->N * cfg->d * sizeof(float);
+    cudaStream_t st = (cudaStream_t)stream;
+    if (cudaMemsetAsync(dK, 0, kv_bytes, st) != cudaSuccess || cudaMemsetAsync(dV, 0, kv_bytes, st) != cudaSuccess)
+        return PISA_E_CUDA;
+    AttnParams p;
+    p.B = cfg->B; p.Hq = cfg->Hq; p.Hkv = cfg->Hkv; p.N = cfg->N; p.C = cfg->C; p.K = cfg->K;
+    p.causal = cfg->causal;
+    p.qscale = (float)(1.4426950408889634 / sqrt((double)cfg->d));
+    return cuda_status(launch_attn_bwd(cfg->dtype, cfg->d, Q, K, V, idx, dO, dQ, dK, dV, p, st));
+}
+
 int pisa_forward(const pisa_cfg* cfg, const void* Q, const void* K, const void* V, float* pyr, int32_t* idx, void* O,
                  void* stream) {
     int s = check_gpu(cfg);

@@ -57,6 +57,8 @@ cudaError_t launch_attn_bm(const void* Q, const void* K, const void* V, const in
                            cudaStream_t st);
 
 cudaError_t launch_pool(int dtype, int d, const void* K, float* pyr, const PoolParams& p, cudaStream_t st);
+cudaError_t launch_attn_bwd(int dtype, int d, const void* Q, const void* K, const void* V, const int32_t* idx,
+                            const void* dO, float* dQ, float* dK, float* dV, const AttnParams& p, cudaStream_t st);
 cudaError_t launch_pyramid_grow(const float* old_pyr, float* new_pyr, int64_t units, int d, const Geom& go,
                                 const Geom& gn, cudaStream_t st);
 cudaError_t launch_select(int dtype, int d, const void* Q, const void* K, const float* pyr, int32_t* idx,

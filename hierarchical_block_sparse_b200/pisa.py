@@ -82,6 +82,7 @@ def load(path: str | None = None):
             "pisa_build_pyramid_prefix": (ctypes.c_int, [cfgp, P, P, P, P]),
             "pisa_pyramid_append": (ctypes.c_int, [cfgp, P, P, P, P, P, P, P]),
             "pisa_pyramid_grow": (ctypes.c_int, [cfgp, P, cfgp, P, P]),
+            "pisa_sparse_attn_backward": (ctypes.c_int, [cfgp, P, P, P, P, P, P, P, P, P]),
             "pisa_decode": (ctypes.c_int, [cfgp, P, P, P, P, P, P, P, P]),
             "pisa_decode_step": (ctypes.c_int, [cfgp, P, P, P, P, P, P, P, P, P, P]),
             "pisa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -259,6 +260,12 @@ def pisa_build_pyramid_prefix(cfg, Kc, length, pyr):
 def pisa_pyramid_append(cfg, Kc, Vc, pyr, k_new, v_new, pos):
     _check("pisa_pyramid_append", load().pisa_pyramid_append(ctypes.byref(cfg), _ptr(Kc), _ptr(Vc), _ptr(pyr),
                                                              _ptr(k_new), _ptr(v_new), _ptr(pos), _stream()))
+
+
+def pisa_sparse_attn_backward(cfg, Q, K, V, idx, dO, dQ, dK, dV):
+    """dQ, dK, dV (fp32) of the sparse attention for the fixed selection idx."""
+    _check("pisa_sparse_attn_backward", load().pisa_sparse_attn_backward(
+        ctypes.byref(cfg), _ptr(Q), _ptr(K), _ptr(V), _ptr(idx), _ptr(dO), _ptr(dQ), _ptr(dK), _ptr(dV), _stream()))
 
 
 def pisa_pyramid_grow(cfg_old, pyr_old, cfg_new, pyr_new):

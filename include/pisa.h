@@ -129,6 +129,18 @@ int pisa_select(const pisa_cfg *cfg, const void *Q, const void *K, const float *
 int pisa_sparse_attn(const pisa_cfg *cfg, const void *Q, const void *K, const void *V,
                      const int32_t *idx, void *O, void *stream);
 
+/* Backward of pisa_sparse_attn with the selection idx held fixed (close
+ * reading §5.3: the gradient flows only through the selected attention
+ * entries). Given Q, K, V, idx as in the forward and dO (the gradient of the
+ * loss with respect to O; [B, Hq, N, d], dtype of Q), writes
+ *   dQ: fp32 [B, Hq, N, d];  dK, dV: fp32 [B, Hkv, N, d] (summed over the
+ *   query heads of each KV head; both are zeroed by the call first).
+ * The softmax statistics are recomputed from Q, K, V and idx. Same limits and
+ * errors as pisa_sparse_attn. */
+int pisa_sparse_attn_backward(const pisa_cfg *cfg, const void *Q, const void *K, const void *V,
+                              const int32_t *idx, const void *dO, float *dQ, float *dK, float *dV,
+                              void *stream);
+
 /* The whole prefill path, in order on one stream: pisa_build_pyramid, then
  * pisa_select, then pisa_sparse_attn. pyr and idx are caller-owned outputs. */
 int pisa_forward(const pisa_cfg *cfg, const void *Q, const void *K, const void *V,
