@@ -577,30 +577,49 @@ def main():
         out["score_variants"] = vout
 
     # ---- backward of the attention with the selection fixed (dQ, dK, dV) ----
+    # Block-major on the tensor cores (pisa_sparse_attn_backward_ws, phases
+    # timed with events), and the per-query CUDA-core call for comparison.
     if not args.no_backward:
         gen = torch.Generator(device=dev).manual_seed(w.seed + 17)
         dOd = torch.randn(Qd.shape, generator=gen, device=dev, dtype=torch.float32).to(Qd.dtype)
         dQ = torch.empty(Qd.shape, dtype=torch.float32, device=dev)
         dK = torch.empty(Kd.shape, dtype=torch.float32, device=dev)
         dV = torch.empty(Vd.shape, dtype=torch.float32, device=dev)
-        pisa.pisa_sparse_attn_backward(cfg, Qd, Kd, Vd, idx, dOd, dQ, dK, dV)
-        torch.cuda.synchronize()
-        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        n_bwd = 2
-        g0.record(stream)
-        for _ in range(n_bwd):
-            pisa.pisa_sparse_attn_backward(cfg, Qd, Kd, Vd, idx, dOd, dQ, dK, dV)
-        g1.record(stream)
-        torch.cuda.synchronize()
-        bms = max_over_ranks(g0.elapsed_time(g1) / n_bwd, dist, dev)
         # per attended (query head, key): 4d FLOP to recompute the softmax and
         # the output, 10d for the logits again, dP, dQ, dK and dV
         bflops = alg["attn_flops"] * 14.0 / 4.0
+        bws = pisa.alloc_backward_workspace(cfg, dev)
+        nbp = len(pisa.BWD_PHASES)
+        for _ in range(2):
+            pisa.pisa_sparse_attn_backward_ws(cfg, Qd, Kd, Vd, idx, dOd, dQ, dK, dV, bws)
+        torch.cuda.synchronize()
+        bev = [[torch.cuda.Event(enable_timing=True) for _ in range(nbp + 1)] for _ in range(3)]
+        for e in bev:
+            for x in e:
+                x.record(stream)
+        torch.cuda.synchronize()
+        for e in bev:
+            pisa.pisa_sparse_attn_backward_ws_events(cfg, Qd, Kd, Vd, idx, dOd, dQ, dK, dV, bws, e)
+        torch.cuda.synchronize()
+        bms = max_over_ranks(bev[0][0].elapsed_time(bev[-1][nbp]) / len(bev), dist, dev)
+        del bws
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        g0.record(stream)
+        pisa.pisa_sparse_attn_backward(cfg, Qd, Kd, Vd, idx, dOd, dQ, dK, dV)
+        g1.record(stream)
+        torch.cuda.synchronize()
+        pq_ms = max_over_ranks(g0.elapsed_time(g1), dist, dev)
         out["backward"] = {"ms": bms, "tokens_per_s": job_tokens_per_s(w.B * w.N, world, bms),
-                           "kernel": "attn_bwd_kernel (per-query warps, CUDA cores, fp32 dK/dV reductions)",
+                           "call": "pisa_sparse_attn_backward_ws",
+                           "kernel": "bwd_tile_kernel (key-major tcgen05 tiles; dK, dV in TMEM per leaf) after "
+                                     "the forward recompute",
+                           "phase_ms": {name: float(np.mean([e[i].elapsed_time(e[i + 1]) for e in bev]))
+                                        for i, name in enumerate(pisa.BWD_PHASES)},
                            "algorithmic_tflop": bflops / 1e12, "achieved_tflops": bflops / (bms / 1e3) / 1e12,
-                           "fp32_fma_peak_tflops": fma_peak,
-                           "frac": bflops / (bms / 1e3) / 1e12 / fma_peak}
+                           "bf16_tensor_peak_tflops": tc_peak,
+                           "frac": bflops / (bms / 1e3) / 1e12 / tc_peak,
+                           "per_query_cuda_core_ms": pq_ms,
+                           "per_query_cuda_core_frac_of_fp32_fma": bflops / (pq_ms / 1e3) / 1e12 / fma_peak}
         del dOd, dQ, dK, dV
 
     # ---- decode: 64 sequences, one new token each, against 256K-key caches ----

@@ -295,6 +295,46 @@ int pisa_sparse_attn_ws(const pisa_cfg* cfg, const void* Q, const void* K, const
                                       nullptr, (cudaStream_t)stream));
 }
 
+static int backward_ws(const pisa_cfg* cfg, const void* Q, const void* K, const void* V, const int32_t* idx,
+                       const void* dO, float* dQ, float* dK, float* dV, void* workspace, size_t workspace_bytes,
+                       const PhaseEvents* ev, void* stream) {
+    int s = check_bm(cfg);
+    if (s) return s;
+    if (cfg->N == 0) return PISA_OK;
+    if (!Q || !K || !V || !idx || !dO || !dQ || !dK || !dV) return PISA_E_INVALID;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(idx) || !aligned16(dO) || !aligned16(dQ) ||
+        !aligned16(dK) || !aligned16(dV))
+        return PISA_E_ALIGNMENT;
+    if (!workspace) return PISA_E_INVALID;
+    if (((uintptr_t)workspace & 255u) != 0) return PISA_E_ALIGNMENT;
+    if (workspace_bytes < blockmajor_bwd_bytes(bm_shape(cfg))) return PISA_E_INVALID;
+    Geom g;
+    make_geom(cfg->N, cfg->C, &g);
+    return cuda_status(launch_attn_bwd_bm(Q, K, V, idx, dO, dQ, dK, dV, select_params(cfg, g), bm_shape(cfg),
+                                          workspace, ev, (cudaStream_t)stream));
+}
+
+int64_t pisa_backward_workspace_bytes(const pisa_cfg* cfg) {
+    int s = check_bm(cfg);
+    if (s) return s;
+    if (cfg->N == 0) return 0;
+    return (int64_t)blockmajor_bwd_bytes(bm_shape(cfg));
+}
+
+int pisa_sparse_attn_backward_ws(const pisa_cfg* cfg, const void* Q, const void* K, const void* V,
+                                 const int32_t* idx, const void* dO, float* dQ, float* dK, float* dV, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+    return backward_ws(cfg, Q, K, V, idx, dO, dQ, dK, dV, workspace, workspace_bytes, nullptr, stream);
+}
+
+int pisa_sparse_attn_backward_ws_events(const pisa_cfg* cfg, const void* Q, const void* K, const void* V,
+                                        const int32_t* idx, const void* dO, float* dQ, float* dK, float* dV,
+                                        void* workspace, size_t workspace_bytes, void* const* events, int n_events,
+                                        void* stream) {
+    PhaseEvents ev{events, n_events};
+    return backward_ws(cfg, Q, K, V, idx, dO, dQ, dK, dV, workspace, workspace_bytes, &ev, stream);
+}
+
 int pisa_forward_ws_events(const pisa_cfg* cfg, const void* Q, const void* K, const void* V, float* pyr,
                            int32_t* idx, void* O, void* workspace, size_t workspace_bytes, void* const* events,
                            int n_events, void* stream) {

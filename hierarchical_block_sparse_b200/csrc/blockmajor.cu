@@ -28,6 +28,7 @@
 //   added into the accumulator with vector reductions; P is already
 //   normalised, so no rescaling is needed.
 // finalize_kernel converts the accumulator to the output dtype.
+#include <cmath>
 #include <type_traits>
 
 #include "pisa_internal.h"
@@ -1012,6 +1013,388 @@ __global__ void finalize_kernel(const float* __restrict__ oacc, __nv_bfloat16* _
     }
 }
 
+// ---------------------------------------------------------- backward tiles ----
+
+// Backward of the attention with the selection fixed (close reading §02 Eq.(2)
+// differentiated; §5.3: gradients reach only the selected entries), key-major
+// on the tensor cores. Per (query row i, selected key j) with the normaliser
+// L_i (log2 units) and D_i = dO_i . o_i of the recomputed forward:
+//   p = 2^(s*scale - L),  dp = dO_i . v_j,  ds = p (dp - D),
+//   dV_j += p dO_i,  dK_j += ds q_i / sqrt(d),  dQ_i += ds k_j / sqrt(d).
+// Rows are grouped by leaf: bucket (b, kv-head, leaf) holds first the leaf's
+// forced section -- the contiguous range of positions for which it is a forced
+// leaf (rows whose idx does not list it contribute nothing) -- and then the
+// positions that list it freely (the forward's grouping, reused). One tile is
+// 128/G positions x G heads of one bucket. Per tile: S = Q K^T and
+// dP = dO V^T (M = 128 rows, N = 64 keys), P and dS packed to bf16 in shared
+// memory, then dV^T += dO^T P and dK^T += Q^T dS (M = 128 dims, N = 64 keys,
+// both operands MN-major views of the row-major tiles) accumulate in TMEM
+// across the consecutive tiles of a leaf, and dQ = dS K (K read as an MN-major
+// view of its K-major tile) is added to its rows by bulk reductions. Each CTA
+// takes a contiguous range of the tile list (equal tile counts per CTA) and
+// adds its dK / dV accumulators to global memory whenever the leaf changes.
+
+// positions [lo, hi) for which `leaf` is a forced leaf (first: every position;
+// current: its own block; previous: the next block), clipped to N
+__device__ __forceinline__ void forced_range(int64_t leaf, int N, int causal, int mask, int64_t& lo, int64_t& hi) {
+    lo = hi = 0;
+    if (leaf == 0 && (mask & 1)) {
+        hi = N;
+        return;
+    }
+    const bool cur = (mask & 4) || causal, prev = (mask & 2) != 0;
+    const int64_t a = leaf * kBlk;
+    if (cur) {
+        lo = a;
+        hi = a + kBlk;
+    }
+    if (prev) {
+        if (!cur) lo = a + kBlk;
+        hi = a + 2 * kBlk;
+    }
+    lo = min(lo, (int64_t)N);
+    hi = min(hi, (int64_t)N);
+}
+
+// tiles per bucket = ceil((forced section + free entries) / per_tile): totals per scan block
+__global__ void __launch_bounds__(kScanBlock) bwd_total_kernel(const int32_t* __restrict__ counts, int64_t nbuckets,
+                                                              int64_t M1, int per_tile, int N, int causal, int mask,
+                                                              longlong2* __restrict__ bsum, int* __restrict__ err) {
+    __shared__ long long s_a[32], s_b[32];
+    const int64_t i = (int64_t)blockIdx.x * kScanBlock + threadIdx.x;
+    long long c = bucket_count(counts, i, nbuckets, N, err);
+    if (i < nbuckets) {
+        int64_t lo, hi;
+        forced_range(i % M1, N, causal, mask, lo, hi);
+        c += hi - lo;
+    }
+    long long t = (c + per_tile - 1) / per_tile, z = 0;
+    block_scan2(t, z, s_a, s_b);
+    if (threadIdx.x == kScanBlock - 1) bsum[blockIdx.x] = make_longlong2(t, 0);
+}
+
+// tile list (b*Hkv + kvh, leaf, first row of the bucket, rows)
+__global__ void __launch_bounds__(kScanBlock) bwd_place_kernel(const int32_t* __restrict__ counts, int64_t nbuckets,
+                                                              int64_t M1, int per_tile, int N, int causal, int mask,
+                                                              const longlong2* __restrict__ bsum,
+                                                              int4* __restrict__ tiles, int32_t* __restrict__ ntiles) {
+    __shared__ long long s_a[32], s_b[32];
+    __shared__ long long s_pre;
+    long long pt = 0;
+    for (int j = threadIdx.x; j < (int)blockIdx.x; j += kScanBlock) pt += bsum[j].x;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) pt += __shfl_xor_sync(kFull, pt, o);
+    if (threadIdx.x == 0) s_pre = 0;
+    __syncthreads();
+    if ((threadIdx.x & 31) == 0) atomicAdd(reinterpret_cast<unsigned long long*>(&s_pre), (unsigned long long)pt);
+    __syncthreads();
+    const int64_t i = (int64_t)blockIdx.x * kScanBlock + threadIdx.x;
+    long long c = bucket_count(counts, i, nbuckets, N, nullptr);
+    if (i < nbuckets) {
+        int64_t lo, hi;
+        forced_range(i % M1, N, causal, mask, lo, hi);
+        c += hi - lo;
+    }
+    const long long nt = (c + per_tile - 1) / per_tile;
+    long long t = nt, z = 0;
+    block_scan2(t, z, s_a, s_b);
+    const long long bt = s_pre + t - nt;  // exclusive
+    if (i < nbuckets)
+        for (long long j = 0; j < nt; ++j)
+            tiles[bt + j] = make_int4((int)(i / M1), (int)(i % M1), (int)(j * per_tile),
+                                      (int)min((long long)per_tile, c - j * per_tile));
+    if (blockIdx.x == gridDim.x - 1 && threadIdx.x == kScanBlock - 1) *ntiles = (int32_t)(s_pre + t);
+}
+
+// D = dO . O per (query, head), O from the fp32 accumulator of the recomputed
+// forward; one warp per row of [B, Hq, N], written as [B, Hkv, N, G]
+template <int G>
+__global__ void bwd_delta_kernel(const __nv_bfloat16* __restrict__ dO, const float* __restrict__ oacc,
+                                 float* __restrict__ Dr, int64_t rows, int N, int Hq) {
+    const int lane = threadIdx.x & 31;
+    const int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (r >= rows) return;
+    float a[4], o[4];
+    Ld<__nv_bfloat16, 4>::run(dO + r * kD + lane * 4, a);
+    const float4 v = *reinterpret_cast<const float4*>(oacc + r * kD + lane * 4);
+    o[0] = v.x; o[1] = v.y; o[2] = v.z; o[3] = v.w;
+    float s = 0.f;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) s = fmaf(a[e], o[e], s);
+#pragma unroll
+    for (int w = 16; w > 0; w >>= 1) s += __shfl_xor_sync(kFull, s, w);
+    if (lane == 0) {
+        const int64_t t = r % N, bq = r / N;
+        const int64_t b = bq / Hq, head = bq % Hq;
+        const int64_t Hkv = Hq / G;
+        Dr[((b * Hkv + head / G) * N + t) * G + head % G] = s;
+    }
+}
+
+// instruction descriptor (kind::f16, bf16 operands, fp32 accumulator) with
+// either operand MN-major
+__host__ __device__ constexpr uint32_t idesc_bf16_mn(int M, int N, int a_mn_major, int b_mn_major) {
+    return tc::idesc_bf16(M, N, b_mn_major) | ((uint32_t)a_mn_major << 15);
+}
+
+struct BwdParams {
+    int B, Hq, Hkv, N, causal, forced_mask, K;
+    int64_t M1;
+    float qscale;      // log2(e) / sqrt(d)
+    float inv_sqrt_d;  // 1 / sqrt(d)
+    int max_tiles;
+};
+
+// gather 128 rows (head kvh*G + r%G, position rt[r]) of X into a K-major tile;
+// rows with rt < 0 are zero-filled (they enter the row contractions)
+template <int G>
+__device__ __forceinline__ void gather_rows_zero(uint32_t smem, const int* rt, const __nv_bfloat16* X, int64_t b,
+                                                 int kvh, int Hq, int N, int tid) {
+    const int i = tid & 7, c = tid >> 3;  // tid in [0, 128)
+#pragma unroll 4
+    for (int g = 0; g < 16; ++g) {
+        const int r = g * 8 + i;
+        const int t = rt[r];
+        if (t >= 0)
+            tc::cp_async16(smem + tc::kmajor128_off(r, c),
+                           X + (((b * Hq + (int64_t)kvh * G + (r % G)) * N) + t) * kD + c * 8);
+        else
+            tc::cp_async_zero16(smem + tc::kmajor128_off(r, c), X);
+    }
+}
+
+constexpr size_t kBwdSmem = 128 * 1024;  // K, V 16 KB each; Q, dO 32 KB each; P, dS 16 KB each
+static_assert(32768 + 128 * kORowStride <= kBwdSmem, "staged dQ rows fit behind the K and V tiles");
+
+template <int G>
+__global__ void __launch_bounds__(256, 1) bwd_tile_kernel(
+    const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ Kmat,
+    const __nv_bfloat16* __restrict__ Vmat, const __nv_bfloat16* __restrict__ dO, const int32_t* __restrict__ idx,
+    const int4* __restrict__ tiles, const int32_t* __restrict__ ntiles_ptr, const int32_t* __restrict__ offsets,
+    const uint32_t* __restrict__ entries, const float* __restrict__ z2, const float* __restrict__ Dr,
+    float* __restrict__ dQ, float* __restrict__ dK, float* __restrict__ dV, int* __restrict__ err, BwdParams p) {
+    extern __shared__ __align__(1024) uint8_t dsm[];
+    uint8_t* const stage = dsm + 32768;  // staged fp32 rows: dQ rows, or dV / dK rows at a flush
+    __shared__ int rt[128];              // position of each MMA row (-1: contributes nothing)
+    __shared__ float rz[128], rd[128];   // its normaliser (log2) and D
+    __shared__ __align__(8) uint64_t mbar;
+    __shared__ uint32_t tmem_base;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int row = (warp & 3) * 32 + lane;  // TMEM lane of this thread
+    const int half = warp >> 2;              // which half of the columns it handles
+    // TMEM columns: [0, 64) S and [64, 128) dP, then [0, 128) dQ; [128, 192) dV^T; [192, 256) dK^T
+    if (warp == 0) tc::tmem_alloc(&tmem_base, 256);
+    if (tid == 0) {
+        tc::mbar_init(&mbar, 1);
+        tc::fence_mbar_init();
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    const uint32_t tm = tmem_base, lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t k_smem = tc::smem_u32(dsm), v_smem = k_smem + 16384, q_smem = k_smem + 32768,
+                   o_smem = k_smem + 65536, p_smem = k_smem + 98304, s_smem = k_smem + 114688;
+    uint8_t* const sP = dsm + 98304;
+    uint8_t* const sS = dsm + 114688;
+    const int64_t T = min((int64_t)*ntiles_ptr, (int64_t)p.max_tiles);
+    const int64_t t_lo = T * blockIdx.x / gridDim.x, t_hi = T * (blockIdx.x + 1) / gridDim.x;
+    int64_t cur_bh = -1, cur_leaf = -1;
+    bool have_acc = false, ok = true;
+    uint32_t phase = 0;
+
+    // add the leaf's dV / dK accumulators to global memory (all MMAs into them have completed)
+    auto flush = [&]() {
+        tc::tc_fence_after();
+        uint8_t* base = stage + half * 64 * kORowStride;  // half 0: dV rows, half 1: dK rows
+        const float sc = half ? p.inv_sqrt_d : 1.f;
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {
+            float v[32];
+            tc::tmem_ld32(tm + lane_off + 128 + half * 64 + part * 32, v);
+            tc::tmem_ld_wait();
+#pragma unroll
+            for (int q = 0; q < 32; ++q)
+                *reinterpret_cast<float*>(base + (part * 32 + q) * kORowStride + row * 4) = v[q] * sc;
+        }
+        tc::fence_async_smem();
+        tc::tc_fence_before();
+        __syncthreads();
+        if (tid < 128) {
+            const int key = tid & 63, h = tid >> 6;
+            const int64_t krow = cur_leaf * kBlk + key;
+            if (krow < p.N) {
+                tc::bulk_reduce_add_f32((h ? dK : dV) + (cur_bh * p.N + krow) * kD,
+                                        tc::smem_u32(stage + h * 64 * kORowStride + key * kORowStride), kD * 4);
+                tc::bulk_commit();
+            }
+        }
+        tc::bulk_wait_read_all();
+        __syncthreads();
+    };
+
+    for (int64_t tile = t_lo; tile < t_hi && ok; ++tile) {
+        const int4 td = tiles[tile];
+        if (!tile_sane(td, (int64_t)p.B * p.Hkv, p.M1, 1 << 30) || td.w > 128 / G) {  // self-check: never expected
+            if (tid == 0) atomicCAS(err, 0, 12);
+            continue;
+        }
+        const int64_t bh = td.x, leaf = td.y;
+        const int64_t b = bh / p.Hkv;
+        const int kvh = (int)(bh - b * p.Hkv);
+        const bool new_leaf = bh != cur_bh || leaf != cur_leaf;
+        if (new_leaf && have_acc) flush();
+        if (new_leaf) {
+            cur_bh = bh;
+            cur_leaf = leaf;
+            have_acc = false;
+            if (tid < 128) load_kblock(k_smem, Kmat + bh * p.N * kD, leaf * kBlk, p.N, tid);
+            else load_kblock(v_smem, Vmat + bh * p.N * kD, leaf * kBlk, p.N, tid - 128);
+        }
+        // the tile's rows: forced section first, then the free entries
+        if (tid < 128) {
+            const int e = tid / G;
+            int t = -1;
+            if (e < td.w) {
+                const int64_t q = (int64_t)td.z + e;
+                int64_t flo, fhi;
+                forced_range(leaf, p.N, p.causal, p.forced_mask, flo, fhi);
+                if (q < fhi - flo) {
+                    const int64_t tt = flo + q;
+                    const int32_t* ir = idx + (bh * p.N + tt) * p.K;
+                    bool member = false;
+                    for (int k = 0; k < p.K; ++k) member |= ir[k] == (int32_t)leaf;
+                    if (member) t = (int)tt;
+                } else {
+                    const uint32_t v = entries[offsets[bh * p.M1 + leaf] + (q - (fhi - flo))];
+                    if ((int)(v >> 5) < p.N) t = (int)(v >> 5);
+                    else atomicCAS(err, 0, 13);  // self-check: never expected
+                }
+            }
+            rt[tid] = t;
+            float z = 0.f, dd = 0.f;
+            if (t >= 0) {
+                const int64_t u = (bh * p.N + t) * G + (tid % G);
+                z = z2[u];
+                dd = Dr[u];
+            }
+            rz[tid] = z;
+            rd[tid] = dd;
+        }
+        __syncthreads();
+        if (tid < 128) gather_rows_zero<G>(q_smem, rt, Q, b, kvh, p.Hq, p.N, tid);
+        else gather_rows_zero<G>(o_smem, rt, dO, b, kvh, p.Hq, p.N, tid - 128);
+        tc::cp_async_commit();
+        tc::cp_async_wait_all();
+        tc::fence_async_smem();
+        __syncthreads();
+        if (tid == 0) {
+            tc::tc_fence_after();
+            constexpr uint32_t id_s = tc::idesc_bf16(128, 64, 0);
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+                tc::mma_bf16(tm, tc::smem_desc(q_smem + k * 256, 128, 2048), tc::smem_desc(k_smem + k * 256, 128, 2048),
+                             id_s, k > 0);
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+                tc::mma_bf16(tm + 64, tc::smem_desc(o_smem + k * 256, 128, 2048),
+                             tc::smem_desc(v_smem + k * 256, 128, 2048), id_s, k > 0);
+            tc::mma_commit(&mbar);
+        }
+        ok = __syncthreads_and(tc::mbar_wait(&mbar, phase, err, 7)) != 0;
+        phase ^= 1;
+        if (!ok) break;
+        tc::tc_fence_after();
+        // P = 2^(s*scale - L) over the visible keys, dS = P (dP - D), both to bf16
+        {
+            float sv[32], dp[32];
+            tc::tmem_ld32(tm + lane_off + half * 32, sv);
+            tc::tmem_ld32(tm + lane_off + 64 + half * 32, dp);
+            tc::tmem_ld_wait();
+            const int t = rt[row];
+            const int nvalid = t >= 0 ? visible_keys(leaf, t, p.N, p.causal) : 0;
+            const float z = rz[row], dd = rd[row];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                uint32_t wp[4], ws[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int i = c * 8 + q * 2, j = half * 32 + i;
+                    const float p0 = j < nvalid ? exp2f(sv[i] * p.qscale - z) : 0.f;
+                    const float p1 = j + 1 < nvalid ? exp2f(sv[i + 1] * p.qscale - z) : 0.f;
+                    __nv_bfloat162 hp = __floats2bfloat162_rn(p0, p1);
+                    __nv_bfloat162 hs = __floats2bfloat162_rn(p0 * (dp[i] - dd), p1 * (dp[i + 1] - dd));
+                    wp[q] = *reinterpret_cast<uint32_t*>(&hp);
+                    ws[q] = *reinterpret_cast<uint32_t*>(&hs);
+                }
+                const uint32_t off = tc::kmajor64_off(row, half * 4 + c);
+                *reinterpret_cast<uint4*>(sP + off) = make_uint4(wp[0], wp[1], wp[2], wp[3]);
+                *reinterpret_cast<uint4*>(sS + off) = make_uint4(ws[0], ws[1], ws[2], ws[3]);
+            }
+        }
+        tc::fence_async_smem();
+        tc::tc_fence_before();
+        __syncthreads();
+        if (tid == 0) {
+            tc::tc_fence_after();
+            // dV^T += dO^T P and dK^T += Q^T dS: M = 128 dims, N = 64 keys, K = 128 rows (16 per step)
+            constexpr uint32_t id_kv = idesc_bf16_mn(128, 64, 1, 1);
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+                tc::mma_bf16(tm + 128, tc::smem_desc(o_smem + k * 4096, 2048, 128),
+                             tc::smem_desc(p_smem + k * 2048, 1024, 128), id_kv, (have_acc || k > 0) ? 1u : 0u);
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+                tc::mma_bf16(tm + 192, tc::smem_desc(q_smem + k * 4096, 2048, 128),
+                             tc::smem_desc(s_smem + k * 2048, 1024, 128), id_kv, (have_acc || k > 0) ? 1u : 0u);
+            // dQ = dS K: M = 128 rows, N = 128 dims, K = 64 keys (16 per step)
+            constexpr uint32_t id_q = tc::idesc_bf16(128, 128, 1);
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                tc::mma_bf16(tm, tc::smem_desc(s_smem + k * 256, 128, 1024),
+                             tc::smem_desc(k_smem + k * 4096, 2048, 128), id_q, k > 0);
+            tc::mma_commit(&mbar);
+        }
+        ok = __syncthreads_and(tc::mbar_wait(&mbar, phase, err, 8)) != 0;
+        phase ^= 1;
+        if (!ok) break;
+        have_acc = true;
+        tc::tc_fence_after();
+        // dQ rows: staged (the tile's buffers are free) and added with one 512-byte bulk reduction each
+        {
+            uint8_t* srow = stage + row * kORowStride;
+#pragma unroll
+            for (int part = 0; part < 2; ++part) {
+                float v[32];
+                const int col = half * 64 + part * 32;
+                tc::tmem_ld32(tm + lane_off + col, v);
+                tc::tmem_ld_wait();
+#pragma unroll
+                for (int q = 0; q < 32; q += 4)
+                    *reinterpret_cast<float4*>(srow + (col + q) * 4) =
+                        make_float4(v[q] * p.inv_sqrt_d, v[q + 1] * p.inv_sqrt_d, v[q + 2] * p.inv_sqrt_d,
+                                    v[q + 3] * p.inv_sqrt_d);
+            }
+            tc::fence_async_smem();
+        }
+        tc::tc_fence_before();
+        __syncthreads();
+        if (tid < 128 && rt[tid] >= 0) {
+            tc::bulk_reduce_add_f32(dQ + (((b * p.Hq + (int64_t)kvh * G + (tid % G)) * p.N) + rt[tid]) * kD,
+                                    tc::smem_u32(stage + tid * kORowStride), kD * 4);
+            tc::bulk_commit();
+        }
+        tc::bulk_wait_read_all();  // the staged rows have been read: the buffers may be refilled
+        __syncthreads();
+    }
+    if (ok && have_acc) flush();
+    tc::bulk_wait_all();
+    __syncthreads();
+    if (warp == 0) {
+        tc::tc_fence_after();
+        tc::tmem_dealloc(tmem_base, 256);
+    }
+}
+
 // -------------------------------------------------------------- host side ----
 
 static int max_tiles_of(const BmShape& s) {
@@ -1234,9 +1617,64 @@ static cudaError_t attn_bm_t(const void* Q, const void* K, const void* V, const 
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     mark(ev, 8, st);
-    finalize_kernel<<<sm_count() * 8, 256, 0, st>>>(oacc, (__nv_bfloat16*)O, nO / 4);
-    e = cudaGetLastError();
+    if (O) {  // without O the fp32 accumulator in the workspace is the result (the backward's recompute)
+        finalize_kernel<<<sm_count() * 8, 256, 0, st>>>(oacc, (__nv_bfloat16*)O, nO / 4);
+        e = cudaGetLastError();
+    }
     mark(ev, 9, st);
+    return e;
+}
+
+size_t blockmajor_bwd_bytes(const BmShape& s) {
+    const int64_t units = (int64_t)s.B * s.Hkv * s.N;
+    return blockmajor_layout(s).total + (((size_t)units * s.G * 4 + 255) & ~size_t(255));
+}
+
+// Backward with the selection fixed: recompute the forward attention (its
+// normaliser and fp32 output stay in the workspace, with the grouping of the
+// free (query, leaf) pairs), D = dO . O, zero the gradients, list the tiles
+// (forced sections + free entries per leaf) and run the key-major tiles.
+template <int G>
+static cudaError_t attn_bwd_bm_t(const void* Q, const void* K, const void* V, const int32_t* idx, const void* dO,
+                                 float* dQ, float* dK, float* dV, const SelectParams& sp, const BmShape& s,
+                                 uint8_t* ws, const PhaseEvents* ev, cudaStream_t st) {
+    const BmLayout L = blockmajor_layout(s);
+    float* Dr = (float*)(ws + L.total);
+    mark(ev, 0, st);
+    cudaError_t e = attn_bm_t<G>(Q, K, V, idx, nullptr, sp, s, ws, false, nullptr, st);
+    if (e != cudaSuccess) return e;
+    mark(ev, 1, st);
+    const int64_t rows = (int64_t)s.B * s.Hq * s.N;
+    bwd_delta_kernel<G><<<grid_for(rows, 8), 256, 0, st>>>((const __nv_bfloat16*)dO, (const float*)(ws + L.oacc), Dr,
+                                                          rows, s.N, s.Hq);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const size_t kv_bytes = (size_t)s.B * s.Hkv * s.N * kD * 4;
+    if ((e = cudaMemsetAsync(dQ, 0, (size_t)rows * kD * 4, st)) != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(dK, 0, kv_bytes, st)) != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(dV, 0, kv_bytes, st)) != cudaSuccess) return e;
+    const int64_t nb = (int64_t)s.B * s.Hkv * s.M1;
+    const unsigned nblk = (unsigned)((nb + kScanBlock - 1) / kScanBlock);
+    bwd_total_kernel<<<nblk, kScanBlock, 0, st>>>((const int32_t*)(ws + L.counts), nb, s.M1, 128 / G, s.N, sp.causal,
+                                                  sp.forced_mask, (longlong2*)(ws + L.bsum), (int*)(ws + L.misc) + 1);
+    bwd_place_kernel<<<nblk, kScanBlock, 0, st>>>((const int32_t*)(ws + L.counts), nb, s.M1, 128 / G, s.N, sp.causal,
+                                                  sp.forced_mask, (const longlong2*)(ws + L.bsum),
+                                                  (int4*)(ws + L.tiles), (int32_t*)(ws + L.misc));
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    mark(ev, 2, st);
+    BwdParams bp{s.B, s.Hq, s.Hkv, s.N, sp.causal, sp.forced_mask, sp.K, s.M1, sp.qscale,
+                 (float)(1.0 / sqrt((double)kD)), max_tiles_of(s)};
+    auto kern = bwd_tile_kernel<G>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kBwdSmem);
+    if (e != cudaSuccess) return e;
+    kern<<<sm_count(), 256, kBwdSmem, st>>>((const __nv_bfloat16*)Q, (const __nv_bfloat16*)K,
+                                            (const __nv_bfloat16*)V, (const __nv_bfloat16*)dO, idx,
+                                            (const int4*)(ws + L.tiles), (const int32_t*)(ws + L.misc),
+                                            (const int32_t*)(ws + L.offsets), (const uint32_t*)(ws + L.entries),
+                                            (const float*)(ws + L.z2), Dr, dQ, dK, dV, (int*)(ws + L.misc) + 1, bp);
+    e = cudaGetLastError();
+    mark(ev, 3, st);
     return e;
 }
 
@@ -1248,6 +1686,20 @@ cudaError_t launch_select_bm(const void* Q, const void* K, const float* pyr, int
         case 4: return select_bm_t<4>(Q, K, pyr, idx, sp, s, (uint8_t*)ws, ev, st);
         case 8: return select_bm_t<8>(Q, K, pyr, idx, sp, s, (uint8_t*)ws, ev, st);
         case 16: return select_bm_t<16>(Q, K, pyr, idx, sp, s, (uint8_t*)ws, ev, st);
+    }
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_attn_bwd_bm(const void* Q, const void* K, const void* V, const int32_t* idx, const void* dO,
+                               float* dQ, float* dK, float* dV, const SelectParams& sp, const BmShape& s, void* ws,
+                               const PhaseEvents* ev, cudaStream_t st) {
+    uint8_t* w = (uint8_t*)ws;
+    switch (s.G) {
+        case 1: return attn_bwd_bm_t<1>(Q, K, V, idx, dO, dQ, dK, dV, sp, s, w, ev, st);
+        case 2: return attn_bwd_bm_t<2>(Q, K, V, idx, dO, dQ, dK, dV, sp, s, w, ev, st);
+        case 4: return attn_bwd_bm_t<4>(Q, K, V, idx, dO, dQ, dK, dV, sp, s, w, ev, st);
+        case 8: return attn_bwd_bm_t<8>(Q, K, V, idx, dO, dQ, dK, dV, sp, s, w, ev, st);
+        case 16: return attn_bwd_bm_t<16>(Q, K, V, idx, dO, dQ, dK, dV, sp, s, w, ev, st);
     }
     return cudaErrorInvalidValue;
 }

@@ -55,6 +55,11 @@ cudaError_t launch_select_bm(const void* Q, const void* K, const float* pyr, int
 cudaError_t launch_attn_bm(const void* Q, const void* K, const void* V, const int32_t* idx, void* O,
                            const SelectParams& sp, const BmShape& s, void* ws, bool have_z2, const PhaseEvents* ev,
                            cudaStream_t st);
+// backward with the selection fixed: its workspace is the forward's plus D per (query, head)
+size_t blockmajor_bwd_bytes(const BmShape& s);
+cudaError_t launch_attn_bwd_bm(const void* Q, const void* K, const void* V, const int32_t* idx, const void* dO,
+                               float* dQ, float* dK, float* dV, const SelectParams& sp, const BmShape& s, void* ws,
+                               const PhaseEvents* ev, cudaStream_t st);
 
 cudaError_t launch_pool(int dtype, int d, const void* K, float* pyr, const PoolParams& p, cudaStream_t st);
 cudaError_t launch_attn_bwd(int dtype, int d, const void* Q, const void* K, const void* V, const int32_t* idx,

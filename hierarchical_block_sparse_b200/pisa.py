@@ -83,6 +83,10 @@ def load(path: str | None = None):
             "pisa_pyramid_append": (ctypes.c_int, [cfgp, P, P, P, P, P, P, P]),
             "pisa_pyramid_grow": (ctypes.c_int, [cfgp, P, cfgp, P, P]),
             "pisa_sparse_attn_backward": (ctypes.c_int, [cfgp, P, P, P, P, P, P, P, P, P]),
+            "pisa_backward_workspace_bytes": (ctypes.c_int64, [cfgp]),
+            "pisa_sparse_attn_backward_ws": (ctypes.c_int, [cfgp, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]),
+            "pisa_sparse_attn_backward_ws_events": (ctypes.c_int, [cfgp, P, P, P, P, P, P, P, P, P, ctypes.c_size_t,
+                                                                   ctypes.POINTER(ctypes.c_void_p), ctypes.c_int, P]),
             "pisa_decode": (ctypes.c_int, [cfgp, P, P, P, P, P, P, P, P]),
             "pisa_decode_step": (ctypes.c_int, [cfgp, P, P, P, P, P, P, P, P, P, P]),
             "pisa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -266,6 +270,40 @@ def pisa_sparse_attn_backward(cfg, Q, K, V, idx, dO, dQ, dK, dV):
     """dQ, dK, dV (fp32) of the sparse attention for the fixed selection idx."""
     _check("pisa_sparse_attn_backward", load().pisa_sparse_attn_backward(
         ctypes.byref(cfg), _ptr(Q), _ptr(K), _ptr(V), _ptr(idx), _ptr(dO), _ptr(dQ), _ptr(dK), _ptr(dV), _stream()))
+
+
+def pisa_backward_workspace_bytes(cfg) -> int:
+    r = int(load().pisa_backward_workspace_bytes(ctypes.byref(cfg)))
+    if r < 0:
+        _check("pisa_backward_workspace_bytes", r)
+    return r
+
+
+def alloc_backward_workspace(cfg, device="cuda") -> torch.Tensor:
+    """Caller-owned workspace for pisa_sparse_attn_backward_ws (256-byte aligned)."""
+    return torch.empty(max(pisa_backward_workspace_bytes(cfg), 256), dtype=torch.uint8, device=device)
+
+
+def pisa_sparse_attn_backward_ws(cfg, Q, K, V, idx, dO, dQ, dK, dV, ws):
+    """pisa_sparse_attn_backward, block-major on the tensor cores (bf16, d = 128, C = 64)."""
+    _check("pisa_sparse_attn_backward_ws", load().pisa_sparse_attn_backward_ws(
+        ctypes.byref(cfg), _ptr(Q), _ptr(K), _ptr(V), _ptr(idx), _ptr(dO), _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(ws),
+        ws.numel(), _stream()))
+
+
+BWD_PHASES = ["forward_recompute", "delta_and_tiles", "backward_tiles"]
+
+
+def pisa_sparse_attn_backward_ws_events(cfg, Q, K, V, idx, dO, dQ, dK, dV, ws, events):
+    """pisa_sparse_attn_backward_ws recording torch.cuda.Event objects (len(BWD_PHASES) + 1)."""
+    stream = torch.cuda.current_stream()
+    for e in events:
+        if e.cuda_event == 0:
+            e.record(stream)
+    arr = (ctypes.c_void_p * len(events))(*[ctypes.c_void_p(e.cuda_event) for e in events])
+    _check("pisa_sparse_attn_backward_ws_events", load().pisa_sparse_attn_backward_ws_events(
+        ctypes.byref(cfg), _ptr(Q), _ptr(K), _ptr(V), _ptr(idx), _ptr(dO), _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(ws),
+        ws.numel(), arr, len(events), _stream()))
 
 
 def pisa_pyramid_grow(cfg_old, pyr_old, cfg_new, pyr_new):

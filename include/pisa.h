@@ -221,6 +221,34 @@ int pisa_forward_ws_events(const pisa_cfg *cfg, const void *Q, const void *K, co
                            int32_t *idx, void *O, void *workspace, size_t workspace_bytes, void *const *events,
                            int n_events, void *stream);
 
+/* Backward of the attention with the selection idx held fixed, block-major on
+ * the tensor cores: same contract, inputs and outputs as
+ * pisa_sparse_attn_backward (dQ fp32 [B, Hq, N, d]; dK, dV fp32 [B, Hkv, N, d];
+ * all three are zeroed by the call first). Steps, all on `stream`: the forward
+ * attention of pisa_sparse_attn_ws is recomputed into the workspace (the per
+ * (query, head) normaliser and the fp32 output O), D = dO . O per (query,
+ * head), then per leaf and tile of the queries that selected it (its forced
+ * positions first): S = Q K^T, dP = dO V^T, P = softmax weights, dS = P (dP - D)
+ * in bf16, dV += P^T dO and dK += dS^T Q accumulated on chip across the
+ * leaf's tiles, dQ += dS K added to its rows. P and dS enter the tensor cores
+ * as bf16 (as the forward's P does), so results equal the CUDA-core call to
+ * within bf16 rounding of those operands, not bit for bit.
+ * Limits and alignment as the other *_ws calls (bf16, d = 128, C = 64, ...).
+ * Workspace: pisa_backward_workspace_bytes(cfg) bytes, 256-byte aligned;
+ * pisa_workspace_status reads its error word as for the other *_ws calls. */
+int64_t pisa_backward_workspace_bytes(const pisa_cfg *cfg);
+int pisa_sparse_attn_backward_ws(const pisa_cfg *cfg, const void *Q, const void *K, const void *V,
+                                 const int32_t *idx, const void *dO, float *dQ, float *dK, float *dV,
+                                 void *workspace, size_t workspace_bytes, void *stream);
+/* pisa_sparse_attn_backward_ws recording caller events (as
+ * pisa_forward_ws_events) at its phase boundaries: 0 forward recompute,
+ * 1 D, zeroing and the tile list, 2 backward tiles; index 3 marks the end. */
+#define PISA_NUM_BWD_PHASES 3
+int pisa_sparse_attn_backward_ws_events(const pisa_cfg *cfg, const void *Q, const void *K, const void *V,
+                                        const int32_t *idx, const void *dO, float *dQ, float *dK, float *dV,
+                                        void *workspace, size_t workspace_bytes, void *const *events,
+                                        int n_events, void *stream);
+
 /* Allocation-free selection. The pages have no counterpart to this call: it
  * exists for callers that cannot allocate device memory (a host application
  * that owns the GPU memory pool and gives plugins no allocator, serving loops

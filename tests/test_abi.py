@@ -150,3 +150,25 @@ def test_workspace_calls_validate_before_launch(lib):
     P16 = [ctypes.c_void_p(4096), ctypes.c_void_p(4096), ctypes.c_void_p(4096 + 16), ctypes.c_void_p(4096)]
     assert lib.pisa_select_ws(ctypes.byref(cfg), *P16, ctypes.c_void_p(8192), need, None) == -4
     assert lib.pisa_select_noalloc(ctypes.byref(cfg), *P16, None) == -4
+
+
+def test_backward_workspace_validates_before_launch(lib):
+    cfg = pisa.make_cfg(B=1, Hq=4, Hkv=2, N=1000, d=128, C=64, K=8)
+    need = pisa.pisa_backward_workspace_bytes(cfg)
+    # the forward's workspace plus D per (query, head), 256-byte rounded
+    assert need == pisa.pisa_workspace_bytes(cfg) + ((2 * 1000 * 2 * 4 + 255) // 256) * 256
+    P = [ctypes.c_void_p(4096)] * 8   # Q, K, V, idx, dO, dQ, dK, dV
+    call = lib.pisa_sparse_attn_backward_ws
+    assert call(ctypes.byref(cfg), *P, None, need, None) == -1                      # no workspace
+    assert call(ctypes.byref(cfg), *P, ctypes.c_void_p(8192 + 16), need, None) == -4  # misaligned workspace
+    assert call(ctypes.byref(cfg), *P, ctypes.c_void_p(8192), need - 1, None) == -1   # too small
+    bad = list(P)
+    bad[5] = ctypes.c_void_p(4096 + 4)                                              # misaligned dQ
+    assert call(ctypes.byref(cfg), *bad, ctypes.c_void_p(8192), need, None) == -4
+    bad[5] = None
+    assert call(ctypes.byref(cfg), *bad, ctypes.c_void_p(8192), need, None) == -1
+    for field, value in (("C", 32), ("d", 64), ("dtype", 0)):
+        c2 = pisa.make_cfg(B=1, Hq=4, Hkv=2, N=1000, d=128, C=64, K=8)
+        setattr(c2, field, value)
+        assert lib.pisa_backward_workspace_bytes(ctypes.byref(c2)) == -2
+        assert call(ctypes.byref(c2), *P, ctypes.c_void_p(8192), need, None) == -2
