@@ -165,6 +165,7 @@ KERNEL_SOURCES = {
     "topk": [(_BMF, "final Top-K"), _CS + "pisa_walk.cuh", _CS + "pisa_device.cuh"],
     "attn_tiles": [(_BMF, "attention tiles")] + _TILE,
     "forced_tiles": [(_BMF, "forced leaves, dense")] + _TILE,
+    "backward_tiles": [(_BMF, "backward tiles")] + _TILE,
     "pool": [_CS + "pool.cu", _CS + "pisa_device.cuh"],
     "select": [_CS + "select.cu", _CS + "pisa_walk.cuh", _CS + "pisa_device.cuh"],
     "attn": [_CS + "attn.cu", _CS + "pisa_attn.cuh", _CS + "pisa_walk.cuh", _CS + "pisa_device.cuh"],
@@ -602,6 +603,17 @@ def main():
             pisa.pisa_sparse_attn_backward_ws_events(cfg, Qd, Kd, Vd, idx, dOd, dQ, dK, dV, bws, e)
         torch.cuda.synchronize()
         bms = max_over_ranks(bev[0][0].elapsed_time(bev[-1][nbp]) / len(bev), dist, dev)
+        # from the state the forward left in its workspace (training steps that keep it)
+        pisa.pisa_forward_ws(cfg, Qd, Kd, Vd, pyr, idx, O, bws)
+        pisa.pisa_sparse_attn_backward_saved_ws(cfg, Qd, Kd, Vd, idx, dOd, dQ, dK, dV, bws)
+        torch.cuda.synchronize()
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        g0.record(stream)
+        for _ in range(3):
+            pisa.pisa_sparse_attn_backward_saved_ws(cfg, Qd, Kd, Vd, idx, dOd, dQ, dK, dV, bws)
+        g1.record(stream)
+        torch.cuda.synchronize()
+        saved_ms = max_over_ranks(g0.elapsed_time(g1) / 3, dist, dev)
         del bws
         g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         g0.record(stream)
@@ -618,6 +630,9 @@ def main():
                            "algorithmic_tflop": bflops / 1e12, "achieved_tflops": bflops / (bms / 1e3) / 1e12,
                            "bf16_tensor_peak_tflops": tc_peak,
                            "frac": bflops / (bms / 1e3) / 1e12 / tc_peak,
+                           "tiles_dram_bytes": measured_traffic("backward_tiles", w.name),
+                           "saved_state_ms": saved_ms,
+                           "saved_state_call": "pisa_sparse_attn_backward_saved_ws (after pisa_forward_ws)",
                            "per_query_cuda_core_ms": pq_ms,
                            "per_query_cuda_core_frac_of_fp32_fma": bflops / (pq_ms / 1e3) / 1e12 / fma_peak}
         del dOd, dQ, dK, dV

@@ -297,7 +297,7 @@ int pisa_sparse_attn_ws(const pisa_cfg* cfg, const void* Q, const void* K, const
 
 static int backward_ws(const pisa_cfg* cfg, const void* Q, const void* K, const void* V, const int32_t* idx,
                        const void* dO, float* dQ, float* dK, float* dV, void* workspace, size_t workspace_bytes,
-                       const PhaseEvents* ev, void* stream) {
+                       bool saved, const PhaseEvents* ev, void* stream) {
     int s = check_bm(cfg);
     if (s) return s;
     if (cfg->N == 0) return PISA_OK;
@@ -311,7 +311,7 @@ static int backward_ws(const pisa_cfg* cfg, const void* Q, const void* K, const 
     Geom g;
     make_geom(cfg->N, cfg->C, &g);
     return cuda_status(launch_attn_bwd_bm(Q, K, V, idx, dO, dQ, dK, dV, select_params(cfg, g), bm_shape(cfg),
-                                          workspace, ev, (cudaStream_t)stream));
+                                          workspace, saved, ev, (cudaStream_t)stream));
 }
 
 int64_t pisa_backward_workspace_bytes(const pisa_cfg* cfg) {
@@ -324,7 +324,13 @@ int64_t pisa_backward_workspace_bytes(const pisa_cfg* cfg) {
 int pisa_sparse_attn_backward_ws(const pisa_cfg* cfg, const void* Q, const void* K, const void* V,
                                  const int32_t* idx, const void* dO, float* dQ, float* dK, float* dV, void* workspace,
                                  size_t workspace_bytes, void* stream) {
-    return backward_ws(cfg, Q, K, V, idx, dO, dQ, dK, dV, workspace, workspace_bytes, nullptr, stream);
+    return backward_ws(cfg, Q, K, V, idx, dO, dQ, dK, dV, workspace, workspace_bytes, false, nullptr, stream);
+}
+
+int pisa_sparse_attn_backward_saved_ws(const pisa_cfg* cfg, const void* Q, const void* K, const void* V,
+                                       const int32_t* idx, const void* dO, float* dQ, float* dK, float* dV,
+                                       void* workspace, size_t workspace_bytes, void* stream) {
+    return backward_ws(cfg, Q, K, V, idx, dO, dQ, dK, dV, workspace, workspace_bytes, true, nullptr, stream);
 }
 
 int pisa_sparse_attn_backward_ws_events(const pisa_cfg* cfg, const void* Q, const void* K, const void* V,
@@ -332,7 +338,7 @@ int pisa_sparse_attn_backward_ws_events(const pisa_cfg* cfg, const void* Q, cons
                                         void* workspace, size_t workspace_bytes, void* const* events, int n_events,
                                         void* stream) {
     PhaseEvents ev{events, n_events};
-    return backward_ws(cfg, Q, K, V, idx, dO, dQ, dK, dV, workspace, workspace_bytes, &ev, stream);
+    return backward_ws(cfg, Q, K, V, idx, dO, dQ, dK, dV, workspace, workspace_bytes, false, &ev, stream);
 }
 
 int pisa_forward_ws_events(const pisa_cfg* cfg, const void* Q, const void* K, const void* V, float* pyr,

@@ -1030,9 +1030,9 @@ __global__ void finalize_kernel(const float* __restrict__ oacc, __nv_bfloat16* _
 // memory, then dV^T += dO^T P and dK^T += Q^T dS (M = 128 dims, N = 64 keys,
 // both operands MN-major views of the row-major tiles) accumulate in TMEM
 // across the consecutive tiles of a leaf, and dQ = dS K (K read as an MN-major
-// view of its K-major tile) is added to its rows by bulk reductions. Each CTA
-// takes a contiguous range of the tile list (equal tile counts per CTA) and
-// adds its dK / dV accumulators to global memory whenever the leaf changes.
+// view of its K-major tile) is added to its rows by bulk reductions. The CTAs
+// take chunks of consecutive tiles round-robin and add their dK / dV
+// accumulators to global memory whenever the leaf changes.
 
 // positions [lo, hi) for which `leaf` is a forced leaf (first: every position;
 // current: its own block; previous: the next block), clipped to N
@@ -1163,8 +1163,22 @@ __device__ __forceinline__ void gather_rows_zero(uint32_t smem, const int* rt, c
     }
 }
 
-constexpr size_t kBwdSmem = 128 * 1024;  // K, V 16 KB each; Q, dO 32 KB each; P, dS 16 KB each
-static_assert(32768 + 128 * kORowStride <= kBwdSmem, "staged dQ rows fit behind the K and V tiles");
+// Shared memory: K [0, 16K), V [16K, 32K), buffer set 0 = Q0 [32K, 64K) and
+// dO0 [64K, 96K), P [96K, 112K), dS [112K, 128K), buffer set 1 = Q1 [128K, 160K)
+// and dO1 [160K, 192K). The next tile's rows are gathered into the other set
+// while this tile computes. Staged fp32 rows (this tile's dQ rows, or the dV /
+// dK rows of a flush; 128 x kORowStride bytes) go to set 0's region
+// [32K, 32K + 66K) or set 1's region [96K, 96K + 66K): each covers its own Q,
+// dO and parts of P / dS, never the other set's Q and dO.
+constexpr size_t kBwdSmem = 192 * 1024;
+constexpr int kBwdChunk = 8;  // consecutive tiles per CTA before it moves on by the grid size
+__host__ __device__ constexpr uint32_t bwd_q(int st) { return st ? 131072u : 32768u; }
+__host__ __device__ constexpr uint32_t bwd_o(int st) { return st ? 163840u : 65536u; }
+__host__ __device__ constexpr uint32_t bwd_stage(int st) { return st ? 98304u : 32768u; }
+constexpr uint32_t kBwdP = 98304, kBwdS = 114688;
+static_assert(bwd_stage(0) + 128 * kORowStride <= bwd_q(1), "set 0 staging stays clear of set 1");
+static_assert(bwd_stage(1) >= bwd_o(0) + 32768 && bwd_stage(1) + 128 * kORowStride <= kBwdSmem,
+              "set 1 staging stays clear of set 0");
 
 template <int G>
 __global__ void __launch_bounds__(256, 1) bwd_tile_kernel(
@@ -1174,9 +1188,8 @@ __global__ void __launch_bounds__(256, 1) bwd_tile_kernel(
     const uint32_t* __restrict__ entries, const float* __restrict__ z2, const float* __restrict__ Dr,
     float* __restrict__ dQ, float* __restrict__ dK, float* __restrict__ dV, int* __restrict__ err, BwdParams p) {
     extern __shared__ __align__(1024) uint8_t dsm[];
-    uint8_t* const stage = dsm + 32768;  // staged fp32 rows: dQ rows, or dV / dK rows at a flush
-    __shared__ int rt[128];              // position of each MMA row (-1: contributes nothing)
-    __shared__ float rz[128], rd[128];   // its normaliser (log2) and D
+    __shared__ int rt[2][128];               // per buffer set: position of each MMA row (-1: contributes nothing)
+    __shared__ float rz[2][128], rd[2][128];  // its normaliser (log2) and D
     __shared__ __align__(8) uint64_t mbar;
     __shared__ uint32_t tmem_base;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -1192,20 +1205,75 @@ __global__ void __launch_bounds__(256, 1) bwd_tile_kernel(
     __syncthreads();
     tc::tc_fence_after();
     const uint32_t tm = tmem_base, lane_off = (uint32_t)((warp & 3) * 32) << 16;
-    const uint32_t k_smem = tc::smem_u32(dsm), v_smem = k_smem + 16384, q_smem = k_smem + 32768,
-                   o_smem = k_smem + 65536, p_smem = k_smem + 98304, s_smem = k_smem + 114688;
-    uint8_t* const sP = dsm + 98304;
-    uint8_t* const sS = dsm + 114688;
+    const uint32_t base = tc::smem_u32(dsm), k_smem = base, v_smem = base + 16384, p_smem = base + kBwdP,
+                   s_smem = base + kBwdS;
+    uint8_t* const sP = dsm + kBwdP;
+    uint8_t* const sS = dsm + kBwdS;
     const int64_t T = min((int64_t)*ntiles_ptr, (int64_t)p.max_tiles);
-    const int64_t t_lo = T * blockIdx.x / gridDim.x, t_hi = T * (blockIdx.x + 1) / gridDim.x;
-    int64_t cur_bh = -1, cur_leaf = -1;
-    bool have_acc = false, ok = true;
-    uint32_t phase = 0;
+    // the k-th tile of this CTA: chunks of kBwdChunk consecutive tiles dealt
+    // round-robin, so that the CTAs work through the list together and the
+    // dQ rows they update stay within a window that L2 holds
+    auto tile_at = [&](int64_t k) -> int64_t {
+        return ((int64_t)blockIdx.x + (k / kBwdChunk) * gridDim.x) * kBwdChunk + k % kBwdChunk;
+    };
+    const int64_t bhs = (int64_t)p.B * p.Hkv;
 
-    // add the leaf's dV / dK accumulators to global memory (all MMAs into them have completed)
-    auto flush = [&]() {
+    // the tile descriptor, or (-1, -1, 0, 0) for a malformed one (self-check: never expected)
+    auto read_tile = [&](int64_t tile) {
+        const int4 td = tiles[tile];
+        if (tile_sane(td, bhs, p.M1, 1 << 30) && td.w <= 128 / G) return td;
+        if (tid == 0) atomicCAS(err, 0, 12);
+        return make_int4(-1, -1, 0, 0);
+    };
+    // rows of a tile into set `st`: forced section first, then the free entries
+    auto setup_rows = [&](const int4& td, int st) {
+        if (tid >= 128) return;
+        const int64_t bh = td.x, leaf = td.y;
+        const int e = tid / G;
+        int t = -1;
+        if (e < td.w) {
+            const int64_t q = (int64_t)td.z + e;
+            int64_t flo, fhi;
+            forced_range(leaf, p.N, p.causal, p.forced_mask, flo, fhi);
+            if (q < fhi - flo) {
+                const int64_t tt = flo + q;
+                const int32_t* ir = idx + (bh * p.N + tt) * p.K;
+                bool member = false;
+                for (int k = 0; k < p.K; ++k) member |= ir[k] == (int32_t)leaf;
+                if (member) t = (int)tt;
+            } else {
+                const uint32_t v = entries[offsets[bh * p.M1 + leaf] + (q - (fhi - flo))];
+                if ((int)(v >> 5) < p.N) t = (int)(v >> 5);
+                else atomicCAS(err, 0, 13);  // self-check: never expected
+            }
+        }
+        rt[st][tid] = t;
+        float z = 0.f, dd = 0.f;
+        if (t >= 0) {
+            const int64_t u = (bh * p.N + t) * G + (tid % G);
+            z = z2[u];
+            dd = Dr[u];
+        }
+        rz[st][tid] = z;
+        rd[st][tid] = dd;
+    };
+    // gather the tile's Q and dO rows into set `st` (rt[st] must be visible to all threads)
+    auto gather = [&](const int4& td, int st) {
+        const int64_t b = td.x >= 0 ? td.x / p.Hkv : 0;
+        const int kvh = td.x >= 0 ? (int)(td.x - b * p.Hkv) : 0;
+        if (tid < 128) gather_rows_zero<G>(base + bwd_q(st), rt[st], Q, b, kvh, p.Hq, p.N, tid);
+        else gather_rows_zero<G>(base + bwd_o(st), rt[st], dO, b, kvh, p.Hq, p.N, tid - 128);
+    };
+    auto load_kv = [&](const int4& td) {
+        const int64_t bh = td.x >= 0 ? td.x : 0, leaf = td.y >= 0 ? td.y : 0;
+        if (tid < 128) load_kblock(k_smem, Kmat + bh * p.N * kD, leaf * kBlk, p.N, tid);
+        else load_kblock(v_smem, Vmat + bh * p.N * kD, leaf * kBlk, p.N, tid - 128);
+    };
+    // add the leaf's dV / dK accumulators (all MMAs into them have completed) to
+    // global memory through the staging region of set `st`
+    auto flush = [&](int64_t bh, int64_t leaf, int st) {
         tc::tc_fence_after();
-        uint8_t* base = stage + half * 64 * kORowStride;  // half 0: dV rows, half 1: dK rows
+        uint8_t* sbase = dsm + bwd_stage(st) + half * 64 * kORowStride;  // half 0: dV rows, half 1: dK rows
         const float sc = half ? p.inv_sqrt_d : 1.f;
 #pragma unroll
         for (int part = 0; part < 2; ++part) {
@@ -1214,17 +1282,17 @@ __global__ void __launch_bounds__(256, 1) bwd_tile_kernel(
             tc::tmem_ld_wait();
 #pragma unroll
             for (int q = 0; q < 32; ++q)
-                *reinterpret_cast<float*>(base + (part * 32 + q) * kORowStride + row * 4) = v[q] * sc;
+                *reinterpret_cast<float*>(sbase + (part * 32 + q) * kORowStride + row * 4) = v[q] * sc;
         }
         tc::fence_async_smem();
         tc::tc_fence_before();
         __syncthreads();
-        if (tid < 128) {
+        if (tid < 128 && bh >= 0) {
             const int key = tid & 63, h = tid >> 6;
-            const int64_t krow = cur_leaf * kBlk + key;
+            const int64_t krow = leaf * kBlk + key;
             if (krow < p.N) {
-                tc::bulk_reduce_add_f32((h ? dK : dV) + (cur_bh * p.N + krow) * kD,
-                                        tc::smem_u32(stage + h * 64 * kORowStride + key * kORowStride), kD * 4);
+                tc::bulk_reduce_add_f32((h ? dK : dV) + (bh * p.N + krow) * kD,
+                                        tc::smem_u32(dsm + bwd_stage(st) + (h * 64 + key) * kORowStride), kD * 4);
                 tc::bulk_commit();
             }
         }
@@ -1232,61 +1300,35 @@ __global__ void __launch_bounds__(256, 1) bwd_tile_kernel(
         __syncthreads();
     };
 
-    for (int64_t tile = t_lo; tile < t_hi && ok; ++tile) {
-        const int4 td = tiles[tile];
-        if (!tile_sane(td, (int64_t)p.B * p.Hkv, p.M1, 1 << 30) || td.w > 128 / G) {  // self-check: never expected
-            if (tid == 0) atomicCAS(err, 0, 12);
-            continue;
-        }
-        const int64_t bh = td.x, leaf = td.y;
-        const int64_t b = bh / p.Hkv;
-        const int kvh = (int)(bh - b * p.Hkv);
-        const bool new_leaf = bh != cur_bh || leaf != cur_leaf;
-        if (new_leaf && have_acc) flush();
-        if (new_leaf) {
-            cur_bh = bh;
-            cur_leaf = leaf;
-            have_acc = false;
-            if (tid < 128) load_kblock(k_smem, Kmat + bh * p.N * kD, leaf * kBlk, p.N, tid);
-            else load_kblock(v_smem, Vmat + bh * p.N * kD, leaf * kBlk, p.N, tid - 128);
-        }
-        // the tile's rows: forced section first, then the free entries
-        if (tid < 128) {
-            const int e = tid / G;
-            int t = -1;
-            if (e < td.w) {
-                const int64_t q = (int64_t)td.z + e;
-                int64_t flo, fhi;
-                forced_range(leaf, p.N, p.causal, p.forced_mask, flo, fhi);
-                if (q < fhi - flo) {
-                    const int64_t tt = flo + q;
-                    const int32_t* ir = idx + (bh * p.N + tt) * p.K;
-                    bool member = false;
-                    for (int k = 0; k < p.K; ++k) member |= ir[k] == (int32_t)leaf;
-                    if (member) t = (int)tt;
-                } else {
-                    const uint32_t v = entries[offsets[bh * p.M1 + leaf] + (q - (fhi - flo))];
-                    if ((int)(v >> 5) < p.N) t = (int)(v >> 5);
-                    else atomicCAS(err, 0, 13);  // self-check: never expected
-                }
-            }
-            rt[tid] = t;
-            float z = 0.f, dd = 0.f;
-            if (t >= 0) {
-                const int64_t u = (bh * p.N + t) * G + (tid % G);
-                z = z2[u];
-                dd = Dr[u];
-            }
-            rz[tid] = z;
-            rd[tid] = dd;
-        }
+    bool have_acc = false, ok = true;
+    uint32_t phase = 0;
+    int4 td = make_int4(-1, -1, 0, 0);
+    int64_t cur_bh = -1, cur_leaf = -1;  // the leaf whose dV / dK are in TMEM
+    int cur_st = 0;                      // the buffer set of the last tile processed
+    if (tile_at(0) < T) {
+        td = read_tile(tile_at(0));
+        setup_rows(td, 0);
         __syncthreads();
-        if (tid < 128) gather_rows_zero<G>(q_smem, rt, Q, b, kvh, p.Hq, p.N, tid);
-        else gather_rows_zero<G>(o_smem, rt, dO, b, kvh, p.Hq, p.N, tid - 128);
+        load_kv(td);
+        gather(td, 0);
         tc::cp_async_commit();
+    }
+    for (int64_t k = 0; tile_at(k) < T; ++k) {
+        const int st = (int)(k & 1);
+        const int64_t bh = td.x, leaf = td.y;
+        cur_bh = bh;
+        cur_leaf = leaf;
+        cur_st = st;
+        const int64_t b = bh >= 0 ? bh / p.Hkv : 0;
+        const int kvh = bh >= 0 ? (int)(bh - b * p.Hkv) : 0;
+        const int64_t next = tile_at(k + 1);
+        const bool has_next = next < T;
+        const int4 tdn = has_next ? read_tile(next) : make_int4(-1, -1, 0, 0);
+        // this tile's rows (and, after a leaf change, its K / V) have landed
         tc::cp_async_wait_all();
         tc::fence_async_smem();
         __syncthreads();
+        const uint32_t q_smem = base + bwd_q(st), o_smem = base + bwd_o(st);
         if (tid == 0) {
             tc::tc_fence_after();
             constexpr uint32_t id_s = tc::idesc_bf16(128, 64, 0);
@@ -1300,6 +1342,8 @@ __global__ void __launch_bounds__(256, 1) bwd_tile_kernel(
                              tc::smem_desc(v_smem + k * 256, 128, 2048), id_s, k > 0);
             tc::mma_commit(&mbar);
         }
+        // the next tile's rows, while S and dP are computed
+        if (has_next) setup_rows(tdn, st ^ 1);
         ok = __syncthreads_and(tc::mbar_wait(&mbar, phase, err, 7)) != 0;
         phase ^= 1;
         if (!ok) break;
@@ -1310,9 +1354,9 @@ __global__ void __launch_bounds__(256, 1) bwd_tile_kernel(
             tc::tmem_ld32(tm + lane_off + half * 32, sv);
             tc::tmem_ld32(tm + lane_off + 64 + half * 32, dp);
             tc::tmem_ld_wait();
-            const int t = rt[row];
+            const int t = rt[st][row];
             const int nvalid = t >= 0 ? visible_keys(leaf, t, p.N, p.causal) : 0;
-            const float z = rz[row], dd = rd[row];
+            const float z = rz[st][row], dd = rd[st][row];
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 uint32_t wp[4], ws[4];
@@ -1354,14 +1398,19 @@ __global__ void __launch_bounds__(256, 1) bwd_tile_kernel(
                              tc::smem_desc(k_smem + k * 4096, 2048, 128), id_q, k > 0);
             tc::mma_commit(&mbar);
         }
+        // the next tile's Q and dO rows into the other set, while these MMAs run
+        if (has_next) {
+            gather(tdn, st ^ 1);
+            tc::cp_async_commit();
+        }
         ok = __syncthreads_and(tc::mbar_wait(&mbar, phase, err, 8)) != 0;
         phase ^= 1;
         if (!ok) break;
         have_acc = true;
         tc::tc_fence_after();
-        // dQ rows: staged (the tile's buffers are free) and added with one 512-byte bulk reduction each
+        // dQ rows: staged in this set's region and added with one 512-byte bulk reduction each
         {
-            uint8_t* srow = stage + row * kORowStride;
+            uint8_t* srow = dsm + bwd_stage(st) + row * kORowStride;
 #pragma unroll
             for (int part = 0; part < 2; ++part) {
                 float v[32];
@@ -1378,15 +1427,24 @@ __global__ void __launch_bounds__(256, 1) bwd_tile_kernel(
         }
         tc::tc_fence_before();
         __syncthreads();
-        if (tid < 128 && rt[tid] >= 0) {
-            tc::bulk_reduce_add_f32(dQ + (((b * p.Hq + (int64_t)kvh * G + (tid % G)) * p.N) + rt[tid]) * kD,
-                                    tc::smem_u32(stage + tid * kORowStride), kD * 4);
+        if (tid < 128 && rt[st][tid] >= 0) {
+            tc::bulk_reduce_add_f32(dQ + (((b * p.Hq + (int64_t)kvh * G + (tid % G)) * p.N) + rt[st][tid]) * kD,
+                                    tc::smem_u32(dsm + bwd_stage(st) + tid * kORowStride), kD * 4);
             tc::bulk_commit();
         }
-        tc::bulk_wait_read_all();  // the staged rows have been read: the buffers may be refilled
+        tc::bulk_wait_read_all();  // the staged rows have been read: the region may be reused
         __syncthreads();
+        // a new leaf next: add this leaf's dV / dK, then load the next K / V
+        if (has_next && (tdn.x != bh || tdn.y != leaf)) {
+            flush(bh, leaf, st);
+            have_acc = false;
+            load_kv(tdn);
+            tc::cp_async_commit();
+        }
+        td = tdn;
     }
-    if (ok && have_acc) flush();
+    if (ok && have_acc) flush(cur_bh, cur_leaf, cur_st);
+    tc::cp_async_wait_all();
     tc::bulk_wait_all();
     __syncthreads();
     if (warp == 0) {
@@ -1634,14 +1692,16 @@ size_t blockmajor_bwd_bytes(const BmShape& s) {
 // normaliser and fp32 output stay in the workspace, with the grouping of the
 // free (query, leaf) pairs), D = dO . O, zero the gradients, list the tiles
 // (forced sections + free entries per leaf) and run the key-major tiles.
+// saved: the workspace already holds that state, left by pisa_forward_ws /
+// pisa_sparse_attn_ws for the same inputs (the recompute is skipped).
 template <int G>
 static cudaError_t attn_bwd_bm_t(const void* Q, const void* K, const void* V, const int32_t* idx, const void* dO,
                                  float* dQ, float* dK, float* dV, const SelectParams& sp, const BmShape& s,
-                                 uint8_t* ws, const PhaseEvents* ev, cudaStream_t st) {
+                                 uint8_t* ws, bool saved, const PhaseEvents* ev, cudaStream_t st) {
     const BmLayout L = blockmajor_layout(s);
     float* Dr = (float*)(ws + L.total);
     mark(ev, 0, st);
-    cudaError_t e = attn_bm_t<G>(Q, K, V, idx, nullptr, sp, s, ws, false, nullptr, st);
+    cudaError_t e = saved ? cudaSuccess : attn_bm_t<G>(Q, K, V, idx, nullptr, sp, s, ws, false, nullptr, st);
     if (e != cudaSuccess) return e;
     mark(ev, 1, st);
     const int64_t rows = (int64_t)s.B * s.Hq * s.N;
@@ -1692,14 +1752,14 @@ cudaError_t launch_select_bm(const void* Q, const void* K, const float* pyr, int
 
 cudaError_t launch_attn_bwd_bm(const void* Q, const void* K, const void* V, const int32_t* idx, const void* dO,
                                float* dQ, float* dK, float* dV, const SelectParams& sp, const BmShape& s, void* ws,
-                               const PhaseEvents* ev, cudaStream_t st) {
+                               bool saved, const PhaseEvents* ev, cudaStream_t st) {
     uint8_t* w = (uint8_t*)ws;
     switch (s.G) {
-        case 1: return attn_bwd_bm_t<1>(Q, K, V, idx, dO, dQ, dK, dV, sp, s, w, ev, st);
-        case 2: return attn_bwd_bm_t<2>(Q, K, V, idx, dO, dQ, dK, dV, sp, s, w, ev, st);
-        case 4: return attn_bwd_bm_t<4>(Q, K, V, idx, dO, dQ, dK, dV, sp, s, w, ev, st);
-        case 8: return attn_bwd_bm_t<8>(Q, K, V, idx, dO, dQ, dK, dV, sp, s, w, ev, st);
-        case 16: return attn_bwd_bm_t<16>(Q, K, V, idx, dO, dQ, dK, dV, sp, s, w, ev, st);
+        case 1: return attn_bwd_bm_t<1>(Q, K, V, idx, dO, dQ, dK, dV, sp, s, w, saved, ev, st);
+        case 2: return attn_bwd_bm_t<2>(Q, K, V, idx, dO, dQ, dK, dV, sp, s, w, saved, ev, st);
+        case 4: return attn_bwd_bm_t<4>(Q, K, V, idx, dO, dQ, dK, dV, sp, s, w, saved, ev, st);
+        case 8: return attn_bwd_bm_t<8>(Q, K, V, idx, dO, dQ, dK, dV, sp, s, w, saved, ev, st);
+        case 16: return attn_bwd_bm_t<16>(Q, K, V, idx, dO, dQ, dK, dV, sp, s, w, saved, ev, st);
     }
     return cudaErrorInvalidValue;
 }

@@ -59,7 +59,7 @@ cudaError_t launch_attn_bm(const void* Q, const void* K, const void* V, const in
 size_t blockmajor_bwd_bytes(const BmShape& s);
 cudaError_t launch_attn_bwd_bm(const void* Q, const void* K, const void* V, const int32_t* idx, const void* dO,
                                float* dQ, float* dK, float* dV, const SelectParams& sp, const BmShape& s, void* ws,
-                               const PhaseEvents* ev, cudaStream_t st);
+                               bool saved, const PhaseEvents* ev, cudaStream_t st);
 
 cudaError_t launch_pool(int dtype, int d, const void* K, float* pyr, const PoolParams& p, cudaStream_t st);
 cudaError_t launch_attn_bwd(int dtype, int d, const void* Q, const void* K, const void* V, const int32_t* idx,

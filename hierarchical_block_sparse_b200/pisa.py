@@ -85,6 +85,8 @@ def load(path: str | None = None):
             "pisa_sparse_attn_backward": (ctypes.c_int, [cfgp, P, P, P, P, P, P, P, P, P]),
             "pisa_backward_workspace_bytes": (ctypes.c_int64, [cfgp]),
             "pisa_sparse_attn_backward_ws": (ctypes.c_int, [cfgp, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]),
+            "pisa_sparse_attn_backward_saved_ws": (ctypes.c_int, [cfgp, P, P, P, P, P, P, P, P, P, ctypes.c_size_t,
+                                                                  P]),
             "pisa_sparse_attn_backward_ws_events": (ctypes.c_int, [cfgp, P, P, P, P, P, P, P, P, P, ctypes.c_size_t,
                                                                    ctypes.POINTER(ctypes.c_void_p), ctypes.c_int, P]),
             "pisa_decode": (ctypes.c_int, [cfgp, P, P, P, P, P, P, P, P]),
@@ -287,6 +289,13 @@ def alloc_backward_workspace(cfg, device="cuda") -> torch.Tensor:
 def pisa_sparse_attn_backward_ws(cfg, Q, K, V, idx, dO, dQ, dK, dV, ws):
     """pisa_sparse_attn_backward, block-major on the tensor cores (bf16, d = 128, C = 64)."""
     _check("pisa_sparse_attn_backward_ws", load().pisa_sparse_attn_backward_ws(
+        ctypes.byref(cfg), _ptr(Q), _ptr(K), _ptr(V), _ptr(idx), _ptr(dO), _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(ws),
+        ws.numel(), _stream()))
+
+
+def pisa_sparse_attn_backward_saved_ws(cfg, Q, K, V, idx, dO, dQ, dK, dV, ws):
+    """The backward reusing what pisa_forward_ws / pisa_sparse_attn_ws left in ws (same inputs)."""
+    _check("pisa_sparse_attn_backward_saved_ws", load().pisa_sparse_attn_backward_saved_ws(
         ctypes.byref(cfg), _ptr(Q), _ptr(K), _ptr(V), _ptr(idx), _ptr(dO), _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(ws),
         ws.numel(), _stream()))
 

@@ -240,6 +240,17 @@ int64_t pisa_backward_workspace_bytes(const pisa_cfg *cfg);
 int pisa_sparse_attn_backward_ws(const pisa_cfg *cfg, const void *Q, const void *K, const void *V,
                                  const int32_t *idx, const void *dO, float *dQ, float *dK, float *dV,
                                  void *workspace, size_t workspace_bytes, void *stream);
+/* pisa_sparse_attn_backward_ws without the forward recompute, for training
+ * steps that keep the forward's workspace: the workspace must hold what
+ * pisa_forward_ws or pisa_sparse_attn_ws left in it for the same cfg, Q, K, V
+ * and idx, with nothing else run on it since (it must be at least
+ * pisa_backward_workspace_bytes(cfg) bytes for both calls). Those calls leave
+ * the normaliser, the fp32 output and the grouping of the selected leaves
+ * there, which is the state the recompute would rebuild. Results and limits as
+ * pisa_sparse_attn_backward_ws; the contents are not checked. */
+int pisa_sparse_attn_backward_saved_ws(const pisa_cfg *cfg, const void *Q, const void *K, const void *V,
+                                       const int32_t *idx, const void *dO, float *dQ, float *dK, float *dV,
+                                       void *workspace, size_t workspace_bytes, void *stream);
 /* pisa_sparse_attn_backward_ws recording caller events (as
  * pisa_forward_ws_events) at its phase boundaries: 0 forward recompute,
  * 1 D, zeroing and the tile list, 2 backward tiles; index 3 marks the end. */

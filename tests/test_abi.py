@@ -167,6 +167,9 @@ def test_backward_workspace_validates_before_launch(lib):
     assert call(ctypes.byref(cfg), *bad, ctypes.c_void_p(8192), need, None) == -4
     bad[5] = None
     assert call(ctypes.byref(cfg), *bad, ctypes.c_void_p(8192), need, None) == -1
+    saved = lib.pisa_sparse_attn_backward_saved_ws
+    assert saved(ctypes.byref(cfg), *P, ctypes.c_void_p(8192), need - 1, None) == -1  # same checks
+    assert saved(ctypes.byref(cfg), *bad, ctypes.c_void_p(8192), need, None) == -1
     for field, value in (("C", 32), ("d", 64), ("dtype", 0)):
         c2 = pisa.make_cfg(B=1, Hq=4, Hkv=2, N=1000, d=128, C=64, K=8)
         setattr(c2, field, value)

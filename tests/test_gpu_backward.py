@@ -128,3 +128,25 @@ def test_block_major_backward_with_unlisted_forced_leaves():
     worst = _worst_vs_oracle(w, Q, K, V, dO, idx, grads)
     print(f"block-major backward, unlisted forced leaves: worst error {worst:.2e}")
     assert worst <= BM_TOL, worst
+
+
+@pytest.mark.parametrize("name", ["mha_ragged", "gqa4", "noncausal_first_only"])
+def test_block_major_backward_from_saved_forward_state(name):
+    # pisa_forward_ws leaves the normaliser, the fp32 output and the grouping in
+    # its workspace; the saved-state backward starts from them
+    w = BM_CASES[name]
+    Q, K, V, _ = make_inputs(w)
+    dev = torch.device("cuda", 0)
+    dO = torch.from_numpy(np.random.default_rng(w.seed + 7).standard_normal(Q.shape).astype(np.float32)).to(Q.dtype)
+    Qd, Kd, Vd, dOd = Q.to(dev), K.to(dev), V.to(dev), dO.to(dev)
+    cfg = pisa.cfg_for(Qd, Kd, C=w.C, K_=w.K, causal=w.causal, forced_mask=w.forced_mask)
+    pyr, idx, O = pisa.alloc_outputs(cfg, dev, Q.dtype)
+    ws = pisa.alloc_backward_workspace(cfg, dev)
+    ws.random_(0, 256)
+    pisa.pisa_forward_ws(cfg, Qd, Kd, Vd, pyr, idx, O, ws)
+    grads = [torch.full(x.shape, float("nan"), dtype=torch.float32, device=dev) for x in (Q, K, V)]
+    pisa.pisa_sparse_attn_backward_saved_ws(cfg, Qd, Kd, Vd, idx, dOd, *grads, ws)
+    assert pisa.pisa_workspace_status(cfg, ws) == 0
+    worst = _worst_vs_oracle(w, Q, K, V, dO, idx.cpu().numpy(), [g.cpu().double().numpy() for g in grads])
+    print(f"block-major backward from saved state {name}: worst error {worst:.2e}")
+    assert worst <= BM_TOL, worst
