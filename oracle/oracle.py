@@ -268,3 +268,60 @@ def attn_backward_rows(Qg: np.ndarray, Kh: np.ndarray, Vh: np.ndarray, idx: np.n
             dQ[h, t] = ds @ KJ * inv
             dK[J] += np.outer(ds, Qg[h, t]) * inv
     return dQ, dK, dV
+
+
+def attn_backward_sampled(Qg: np.ndarray, Kh: np.ndarray, Vh: np.ndarray, idx: np.ndarray, dOg: np.ndarray, *,
+                          C: int, causal: bool = True, rows=(), leaves=()):
+    """Selected entries of attn_backward_rows, for checks at sizes where the
+    full backward is out of reach: dQ of the query positions `rows` (each needs
+    its own row only) and dK, dV of the keys of the leaves `leaves` (each needs
+    every position whose idx lists the leaf: its softmax over all of its
+    selected keys, and its D = dO . o).
+
+    Same arithmetic per row as attn_backward_rows. Returns (dQ [G, len(rows), d],
+    dK [len(leaves), C, d], dV [len(leaves), C, d]) in float64; key rows past N
+    stay zero."""
+    G, N, d = Qg.shape
+    inv = 1.0 / np.sqrt(d)
+
+    def row_terms(t: int, h: int):
+        J = []
+        for leaf in idx[t]:
+            if leaf < 0:
+                continue
+            hi = min((int(leaf) + 1) * C, N)
+            if causal:
+                hi = min(hi, t + 1)
+            J.extend(range(int(leaf) * C, hi))
+        J = np.array(sorted(J), np.int64)
+        q = np.asarray(Qg[h, t], np.float64)
+        do = np.asarray(dOg[h, t], np.float64)
+        KJ = np.asarray(Kh[J], np.float64)
+        VJ = np.asarray(Vh[J], np.float64)
+        s = KJ @ q * inv
+        p = np.exp(s - s.max())
+        p /= p.sum()
+        o = p @ VJ
+        ds = p * (VJ @ do - do @ o)
+        return J, p, ds, q, do, KJ
+
+    dQ = np.zeros((G, len(rows), d))
+    for i, t in enumerate(rows):
+        for h in range(G):
+            J, p, ds, q, do, KJ = row_terms(int(t), h)
+            if J.size:
+                dQ[h, i] = ds @ KJ * inv
+    dK = np.zeros((len(leaves), C, d))
+    dV = np.zeros((len(leaves), C, d))
+    for li, leaf in enumerate(leaves):
+        users = np.nonzero((np.asarray(idx) == leaf).any(axis=1))[0]
+        for t in users:
+            for h in range(G):
+                J, p, ds, q, do, KJ = row_terms(int(t), h)
+                m = (J >= leaf * C) & (J < (leaf + 1) * C)
+                if not m.any():
+                    continue
+                kl = J[m] - leaf * C
+                dV[li, kl] += np.outer(p[m], do)
+                dK[li, kl] += np.outer(ds[m], q) * inv
+    return dQ, dK, dV

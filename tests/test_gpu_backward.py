@@ -150,3 +150,40 @@ def test_block_major_backward_from_saved_forward_state(name):
     worst = _worst_vs_oracle(w, Q, K, V, dO, idx.cpu().numpy(), [g.cpu().double().numpy() for g in grads])
     print(f"block-major backward from saved state {name}: worst error {worst:.2e}")
     assert worst <= BM_TOL, worst
+
+
+def test_block_major_backward_full_size_sampled():
+    # the bench's workload and launch configuration (MHA-8, N = 262144): dQ of
+    # sampled rows and dK, dV of sampled leaves (early, middle, last) against
+    # the oracle's per-entry backward, on two KV heads
+    w = WORKLOADS["mha8_n256k"]
+    Q, K, V, _ = make_inputs(w)
+    dev = torch.device("cuda", 0)
+    dO = torch.from_numpy(np.random.default_rng(w.seed + 7).standard_normal(Q.shape).astype(np.float32)).to(Q.dtype)
+    Qd, Kd, Vd, dOd = Q.to(dev), K.to(dev), V.to(dev), dO.to(dev)
+    cfg = pisa.cfg_for(Qd, Kd, C=w.C, K_=w.K, causal=w.causal, forced_mask=w.forced_mask)
+    pyr, idx, O = pisa.alloc_outputs(cfg, dev, Q.dtype)
+    ws = pisa.alloc_backward_workspace(cfg, dev)
+    pisa.pisa_forward_ws(cfg, Qd, Kd, Vd, pyr, idx, O, ws)
+    grads = [torch.empty(x.shape, dtype=torch.float32, device=dev) for x in (Q, K, V)]
+    pisa.pisa_sparse_attn_backward_ws(cfg, Qd, Kd, Vd, idx, dOd, *grads, ws)
+    assert pisa.pisa_workspace_status(cfg, ws) == 0
+    del Qd, Kd, Vd, dOd, ws
+    idx_h = idx.cpu().numpy()
+    M1 = (w.N + w.C - 1) // w.C
+    rng = np.random.default_rng(5)
+    rows = sorted(set(rng.choice(w.N, size=14, replace=False).tolist()) | {0, w.N - 1})
+    leaves = [37, M1 // 2, M1 - 1]
+    worst = 0.0
+    for h in (0, 5):
+        rQ, rK, rV = oracle.attn_backward_sampled(
+            oracle.to_f64(Q[0, h:h + 1]), oracle.to_f64(K[0, h]), oracle.to_f64(V[0, h]), idx_h[0, h],
+            oracle.to_f64(dO[0, h:h + 1]), C=w.C, causal=w.causal, rows=rows, leaves=leaves)
+        gQ = grads[0][0, h, rows].cpu().double().numpy()
+        gK = torch.stack([grads[1][0, h, l * w.C:(l + 1) * w.C] for l in leaves]).cpu().double().numpy()
+        gV = torch.stack([grads[2][0, h, l * w.C:(l + 1) * w.C] for l in leaves]).cpu().double().numpy()
+        for got, ref in ((gQ, rQ[0]), (gK, rK), (gV, rV)):
+            assert np.isfinite(got).all()
+            worst = max(worst, float(np.abs(got - ref).max()) / max(1.0, float(np.abs(ref).max())))
+    print(f"block-major backward, 256K MHA-8 sampled: worst error {worst:.2e} of max |ref|")
+    assert worst <= BM_TOL, worst

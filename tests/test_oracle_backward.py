@@ -91,3 +91,29 @@ def test_central_differences_on_a_sparse_case():
             args_m = {"Q": (Xm, Kk, V), "K": (Q, Xm, V), "V": (Q, Kk, Xm)}[name]
             num = (loss(*args_p) - loss(*args_m)) / (2 * eps)
             assert grad.flat[flat] == pytest.approx(num, rel=1e-6, abs=1e-8), name
+
+
+@pytest.mark.parametrize("G,causal", [(1, True), (2, False)])
+def test_sampled_backward_equals_the_full_backward(G, causal):
+    # the sampled form (used at sizes where the full backward is too slow)
+    # against the entries of the pinned full backward
+    N, C, d, K = 300, 16, 8, 4
+    rng = np.random.default_rng(31 + G)
+    Q, Kh, Vh, dO = _rand((G, N, d), 32), _rand((N, d), 33), _rand((N, d), 34), _rand((G, N, d), 35)
+    M1 = (N + C - 1) // C
+    idx = np.full((N, K), -1, np.int64)
+    for t in range(N):
+        c = t // C
+        pick = {0, c} | set(rng.choice(max(c, 1), size=min(K - 2, max(c, 1)), replace=False).tolist())
+        pick = sorted(x for x in pick if x <= (c if causal else M1 - 1))[:K]
+        idx[t, :len(pick)] = pick
+    fQ, fK, fV = oracle.attn_backward_rows(Q, Kh, Vh, idx, dO, C=C, causal=causal)
+    rows = [0, 17, 150, N - 1]
+    leaves = [0, 5, M1 - 1]  # the last leaf is ragged (300 = 18 x 16 + 12)
+    sQ, sK, sV = oracle.attn_backward_sampled(Q, Kh, Vh, idx, dO, C=C, causal=causal, rows=rows, leaves=leaves)
+    np.testing.assert_allclose(sQ, fQ[:, rows], rtol=1e-12, atol=1e-12)
+    for li, leaf in enumerate(leaves):
+        n = min(C, N - leaf * C)
+        np.testing.assert_allclose(sK[li, :n], fK[leaf * C:leaf * C + n], rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(sV[li, :n], fV[leaf * C:leaf * C + n], rtol=1e-12, atol=1e-12)
+        assert not sK[li, n:].any() and not sV[li, n:].any()
