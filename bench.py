@@ -624,7 +624,7 @@ def main():
         out["backward"] = {"ms": bms, "tokens_per_s": job_tokens_per_s(w.B * w.N, world, bms),
                            "call": "pisa_sparse_attn_backward_ws",
                            "kernel": "bwd_tile_kernel (key-major tcgen05 tiles; dK, dV in TMEM per leaf) after "
-                                     "the forward recompute",
+                                     "the statistics pass (bwd_stats_kernel: per-leaf LSE and P-weighted dP)",
                            "phase_ms": {name: float(np.mean([e[i].elapsed_time(e[i + 1]) for e in bev]))
                                         for i, name in enumerate(pisa.BWD_PHASES)},
                            "algorithmic_tflop": bflops / 1e12, "achieved_tflops": bflops / (bms / 1e3) / 1e12,

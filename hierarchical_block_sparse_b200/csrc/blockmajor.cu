@@ -1163,6 +1163,172 @@ __device__ __forceinline__ void gather_rows_zero(uint32_t smem, const int* rt, c
     }
 }
 
+// Softmax statistics of the backward from Q, K, V, dO and idx alone (no
+// forward output needed). Per (row, listed leaf), over the leaf's visible keys
+// with x = s * scale (log2 units):
+//   lse = log2 sum_j 2^x_j,   dbar = sum_j 2^(x_j - lse) dp_j   (dp = dO . v),
+// written per (unit, idx slot, head). bwd_combine_kernel then forms
+//   L = log2 sum_l 2^lse_l   and   D = sum_l 2^(lse_l - L) dbar_l = sum_j p_j dp_j,
+// which is dO . o. One tile of the backward's tile list per step: S = Q K^T and
+// dP = dO V^T on the tensor cores (M = 128 rows, N = 64 keys each).
+constexpr size_t kStatsSmem = 96 * 1024;  // Q, dO 32 KB each; K, V 16 KB each
+
+template <int G>
+__global__ void __launch_bounds__(128) bwd_stats_kernel(
+    const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ Kmat,
+    const __nv_bfloat16* __restrict__ Vmat, const __nv_bfloat16* __restrict__ dO, const int32_t* __restrict__ idx,
+    const int4* __restrict__ tiles, const int32_t* __restrict__ ntiles_ptr, const int32_t* __restrict__ offsets,
+    const uint32_t* __restrict__ entries, float* __restrict__ lse_s, float* __restrict__ dbar_s,
+    int* __restrict__ err, BwdParams p) {
+    extern __shared__ __align__(1024) uint8_t dsm[];
+    __shared__ int rt[128], rk[128];  // position and idx slot of each MMA row (rt -1: contributes nothing)
+    __shared__ __align__(8) uint64_t mbar;
+    __shared__ uint32_t tmem_base;
+    const int tid = threadIdx.x, warp = tid >> 5;
+    if (warp == 0) tc::tmem_alloc(&tmem_base, 128);  // S [0, 64), dP [64, 128)
+    if (tid == 0) {
+        tc::mbar_init(&mbar, 1);
+        tc::fence_mbar_init();
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    const uint32_t tm = tmem_base, taddr = tm + ((uint32_t)(warp * 32) << 16);
+    const uint32_t q_smem = tc::smem_u32(dsm), o_smem = q_smem + 32768, k_smem = q_smem + 65536,
+                   v_smem = q_smem + 81920;
+    const int T = min(*ntiles_ptr, p.max_tiles);
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < T && ok; tile += gridDim.x) {
+        const int4 td = tiles[tile];
+        if (!tile_sane(td, (int64_t)p.B * p.Hkv, p.M1, 1 << 30) || td.w > 128 / G) {  // self-check: never expected
+            if (tid == 0) atomicCAS(err, 0, 12);
+            continue;
+        }
+        const int64_t bh = td.x, leaf = td.y;
+        const int64_t b = bh / p.Hkv;
+        const int kvh = (int)(bh - b * p.Hkv);
+        {
+            const int e = tid / G;
+            int t = -1, k = -1;
+            if (e < td.w) {
+                const int64_t q = (int64_t)td.z + e;
+                int64_t flo, fhi;
+                forced_range(leaf, p.N, p.causal, p.forced_mask, flo, fhi);
+                if (q < fhi - flo) {
+                    const int64_t tt = flo + q;
+                    const int32_t* ir = idx + (bh * p.N + tt) * p.K;
+                    for (int j = p.K - 1; j >= 0; --j)
+                        if (ir[j] == (int32_t)leaf) k = j;
+                    if (k >= 0) t = (int)tt;
+                } else {
+                    const uint32_t v = entries[offsets[bh * p.M1 + leaf] + (q - (fhi - flo))];
+                    if ((int)(v >> 5) < p.N && (int)(v & 31u) < p.K) {
+                        t = (int)(v >> 5);
+                        k = (int)(v & 31u);
+                    } else {
+                        atomicCAS(err, 0, 13);  // self-check: never expected
+                    }
+                }
+            }
+            rt[tid] = t;
+            rk[tid] = k;
+        }
+        __syncthreads();
+        gather_rows_zero<G>(q_smem, rt, Q, b, kvh, p.Hq, p.N, tid);
+        gather_rows_zero<G>(o_smem, rt, dO, b, kvh, p.Hq, p.N, tid);
+        load_kblock(k_smem, Kmat + bh * p.N * kD, leaf * kBlk, p.N, tid);
+        load_kblock(v_smem, Vmat + bh * p.N * kD, leaf * kBlk, p.N, tid);
+        tc::cp_async_commit();
+        tc::cp_async_wait_all();
+        tc::fence_async_smem();
+        __syncthreads();
+        if (tid == 0) {
+            tc::tc_fence_after();
+            constexpr uint32_t id_s = tc::idesc_bf16(128, 64, 0);
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+                tc::mma_bf16(tm, tc::smem_desc(q_smem + k * 256, 128, 2048), tc::smem_desc(k_smem + k * 256, 128, 2048),
+                             id_s, k > 0);
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+                tc::mma_bf16(tm + 64, tc::smem_desc(o_smem + k * 256, 128, 2048),
+                             tc::smem_desc(v_smem + k * 256, 128, 2048), id_s, k > 0);
+            tc::mma_commit(&mbar);
+        }
+        ok = __syncthreads_and(tc::mbar_wait(&mbar, phase, err, 9)) != 0;
+        phase ^= 1;
+        if (!ok) break;
+        tc::tc_fence_after();
+        {
+            const int t = rt[tid];
+            const int nvalid = t >= 0 ? visible_keys(leaf, t, p.N, p.causal) : 0;
+            float m = -INFINITY, l = 0.f, dd = 0.f;
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                float sv[32], dp[32];
+                tc::tmem_ld32(taddr + c * 32, sv);
+                tc::tmem_ld32(taddr + 64 + c * 32, dp);
+                tc::tmem_ld_wait();
+                float mc = -INFINITY;
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                    if (c * 32 + j < nvalid) mc = fmaxf(mc, sv[j] * p.qscale);
+                const float mn = fmaxf(m, mc);
+                if (mn != -INFINITY) {
+                    const float sc = exp2f(m - mn);
+                    l *= sc;
+                    dd *= sc;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        if (c * 32 + j < nvalid) {
+                            const float w = exp2f(sv[j] * p.qscale - mn);
+                            l += w;
+                            dd = fmaf(w, dp[j], dd);
+                        }
+                    m = mn;
+                }
+            }
+            if (t >= 0) {
+                const int64_t o = ((bh * p.N + t) * p.K + rk[tid]) * G + (tid % G);
+                lse_s[o] = l > 0.f ? m + log2f(l) : -INFINITY;
+                dbar_s[o] = l > 0.f ? dd / l : 0.f;
+            }
+        }
+        tc::tc_fence_before();
+        __syncthreads();
+    }
+    __syncthreads();
+    if (warp == 0) {
+        tc::tc_fence_after();
+        tc::tmem_dealloc(tm, 128);
+    }
+}
+
+// L (log2) and D per (unit, head) from the per-leaf statistics of the listed leaves
+template <int G>
+__global__ void bwd_combine_kernel(const int32_t* __restrict__ idx, const float* __restrict__ lse_s,
+                                   const float* __restrict__ dbar_s, float* __restrict__ z2, float* __restrict__ Dr,
+                                   int64_t units, int K) {
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= units * G) return;
+    const int64_t unit = i / G;
+    const int h = (int)(i - unit * G);
+    float m = -INFINITY;
+    for (int k = 0; k < K; ++k)
+        if (idx[unit * K + k] >= 0) m = fmaxf(m, lse_s[(unit * K + k) * G + h]);
+    float l = 0.f, dd = 0.f;
+    if (m != -INFINITY)
+        for (int k = 0; k < K; ++k)
+            if (idx[unit * K + k] >= 0) {
+                const float w = exp2f(lse_s[(unit * K + k) * G + h] - m);
+                l += w;
+                dd = fmaf(w, dbar_s[(unit * K + k) * G + h], dd);
+            }
+    z2[i] = l > 0.f ? m + log2f(l) : -INFINITY;
+    Dr[i] = l > 0.f ? dd / l : 0.f;
+}
+
 // Shared memory: K [0, 16K), V [16K, 32K), buffer set 0 = Q0 [32K, 64K) and
 // dO0 [64K, 96K), P [96K, 112K), dS [112K, 128K), buffer set 1 = Q1 [128K, 160K)
 // and dO1 [160K, 192K). The next tile's rows are gathered into the other set
@@ -1688,31 +1854,31 @@ size_t blockmajor_bwd_bytes(const BmShape& s) {
     return blockmajor_layout(s).total + (((size_t)units * s.G * 4 + 255) & ~size_t(255));
 }
 
-// Backward with the selection fixed: recompute the forward attention (its
-// normaliser and fp32 output stay in the workspace, with the grouping of the
-// free (query, leaf) pairs), D = dO . O, zero the gradients, list the tiles
-// (forced sections + free entries per leaf) and run the key-major tiles.
-// saved: the workspace already holds that state, left by pisa_forward_ws /
-// pisa_sparse_attn_ws for the same inputs (the recompute is skipped).
+// Backward with the selection fixed. The softmax statistics L and D per
+// (query, head) come either from the stats pass over the same tiles (the free
+// (query, leaf) pairs grouped as the forward groups them, plus each leaf's
+// forced section) or, when `saved`, from what pisa_forward_ws /
+// pisa_sparse_attn_ws left in the workspace (the normaliser, the fp32 output
+// for D = dO . O, and the grouping). Then the gradients are zeroed and the
+// key-major tiles run.
 template <int G>
 static cudaError_t attn_bwd_bm_t(const void* Q, const void* K, const void* V, const int32_t* idx, const void* dO,
                                  float* dQ, float* dK, float* dV, const SelectParams& sp, const BmShape& s,
                                  uint8_t* ws, bool saved, const PhaseEvents* ev, cudaStream_t st) {
     const BmLayout L = blockmajor_layout(s);
     float* Dr = (float*)(ws + L.total);
-    mark(ev, 0, st);
-    cudaError_t e = saved ? cudaSuccess : attn_bm_t<G>(Q, K, V, idx, nullptr, sp, s, ws, false, nullptr, st);
-    if (e != cudaSuccess) return e;
-    mark(ev, 1, st);
+    const int64_t units = (int64_t)s.B * s.Hkv * s.N;
     const int64_t rows = (int64_t)s.B * s.Hq * s.N;
-    bwd_delta_kernel<G><<<grid_for(rows, 8), 256, 0, st>>>((const __nv_bfloat16*)dO, (const float*)(ws + L.oacc), Dr,
-                                                          rows, s.N, s.Hq);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    const size_t kv_bytes = (size_t)s.B * s.Hkv * s.N * kD * 4;
-    if ((e = cudaMemsetAsync(dQ, 0, (size_t)rows * kD * 4, st)) != cudaSuccess) return e;
-    if ((e = cudaMemsetAsync(dK, 0, kv_bytes, st)) != cudaSuccess) return e;
-    if ((e = cudaMemsetAsync(dV, 0, kv_bytes, st)) != cudaSuccess) return e;
+    mark(ev, 0, st);
+    cudaError_t e;
+    if (saved) {
+        bwd_delta_kernel<G><<<grid_for(rows, 8), 256, 0, st>>>((const __nv_bfloat16*)dO, (const float*)(ws + L.oacc),
+                                                              Dr, rows, s.N, s.Hq);
+    } else {
+        if ((e = cudaMemsetAsync(ws + L.misc, 0, 256, st)) != cudaSuccess) return e;
+        if ((e = build_tiles(idx, sp.K, sp, s, ws, L, st)) != cudaSuccess) return e;
+    }
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
     const int64_t nb = (int64_t)s.B * s.Hkv * s.M1;
     const unsigned nblk = (unsigned)((nb + kScanBlock - 1) / kScanBlock);
     bwd_total_kernel<<<nblk, kScanBlock, 0, st>>>((const int32_t*)(ws + L.counts), nb, s.M1, 128 / G, s.N, sp.causal,
@@ -1720,11 +1886,34 @@ static cudaError_t attn_bwd_bm_t(const void* Q, const void* K, const void* V, co
     bwd_place_kernel<<<nblk, kScanBlock, 0, st>>>((const int32_t*)(ws + L.counts), nb, s.M1, 128 / G, s.N, sp.causal,
                                                   sp.forced_mask, (const longlong2*)(ws + L.bsum),
                                                   (int4*)(ws + L.tiles), (int32_t*)(ws + L.misc));
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    mark(ev, 2, st);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
     BwdParams bp{s.B, s.Hq, s.Hkv, s.N, sp.causal, sp.forced_mask, sp.K, s.M1, sp.qscale,
                  (float)(1.0 / sqrt((double)kD)), max_tiles_of(s)};
+    if (!saved) {
+        // per (unit, slot, head) statistics in the leaf-LSE region and the
+        // (unused here) output accumulator region, then L into z2 and D
+        float* lse_s = (float*)(ws + L.lse);
+        float* dbar_s = (float*)(ws + L.oacc);
+        auto sk = bwd_stats_kernel<G>;
+        if ((e = cudaFuncSetAttribute(sk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kStatsSmem)) !=
+            cudaSuccess)
+            return e;
+        sk<<<sm_count() * 2, 128, kStatsSmem, st>>>((const __nv_bfloat16*)Q, (const __nv_bfloat16*)K,
+                                                    (const __nv_bfloat16*)V, (const __nv_bfloat16*)dO, idx,
+                                                    (const int4*)(ws + L.tiles), (const int32_t*)(ws + L.misc),
+                                                    (const int32_t*)(ws + L.offsets),
+                                                    (const uint32_t*)(ws + L.entries), lse_s, dbar_s,
+                                                    (int*)(ws + L.misc) + 1, bp);
+        bwd_combine_kernel<G><<<grid_for(units * G, 256), 256, 0, st>>>(idx, lse_s, dbar_s, (float*)(ws + L.z2), Dr,
+                                                                        units, sp.K);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    mark(ev, 1, st);
+    const size_t kv_bytes = (size_t)s.B * s.Hkv * s.N * kD * 4;
+    if ((e = cudaMemsetAsync(dQ, 0, (size_t)rows * kD * 4, st)) != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(dK, 0, kv_bytes, st)) != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(dV, 0, kv_bytes, st)) != cudaSuccess) return e;
+    mark(ev, 2, st);
     auto kern = bwd_tile_kernel<G>;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kBwdSmem);
     if (e != cudaSuccess) return e;

@@ -300,7 +300,7 @@ def pisa_sparse_attn_backward_saved_ws(cfg, Q, K, V, idx, dO, dQ, dK, dV, ws):
         ws.numel(), _stream()))
 
 
-BWD_PHASES = ["forward_recompute", "delta_and_tiles", "backward_tiles"]
+BWD_PHASES = ["statistics", "zeroing", "backward_tiles"]
 
 
 def pisa_sparse_attn_backward_ws_events(cfg, Q, K, V, idx, dO, dQ, dK, dV, ws, events):

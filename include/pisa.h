@@ -224,13 +224,14 @@ int pisa_forward_ws_events(const pisa_cfg *cfg, const void *Q, const void *K, co
 /* Backward of the attention with the selection idx held fixed, block-major on
  * the tensor cores: same contract, inputs and outputs as
  * pisa_sparse_attn_backward (dQ fp32 [B, Hq, N, d]; dK, dV fp32 [B, Hkv, N, d];
- * all three are zeroed by the call first). Steps, all on `stream`: the forward
- * attention of pisa_sparse_attn_ws is recomputed into the workspace (the per
- * (query, head) normaliser and the fp32 output O), D = dO . O per (query,
- * head), then per leaf and tile of the queries that selected it (its forced
- * positions first): S = Q K^T, dP = dO V^T, P = softmax weights, dS = P (dP - D)
- * in bf16, dV += P^T dO and dK += dS^T Q accumulated on chip across the
- * leaf's tiles, dQ += dS K added to its rows. P and dS enter the tensor cores
+ * all three are zeroed by the call first). Steps, all on `stream`: the
+ * (query, leaf) pairs of idx are grouped by leaf (each leaf's forced positions
+ * first); a statistics pass over those tiles computes S = Q K^T and dP = dO V^T
+ * and, per pair, the leaf's log-sum-exp and P-weighted dP, combined per
+ * (query, head) into the normaliser L and D = sum_j p_j dp_j (= dO . o); then
+ * per tile: P = softmax weights, dS = P (dP - D) in bf16, dV += P^T dO and
+ * dK += dS^T Q accumulated on chip across the leaf's tiles, dQ += dS K added to
+ * its rows. P and dS enter the tensor cores
  * as bf16 (as the forward's P does), so results equal the CUDA-core call to
  * within bf16 rounding of those operands, not bit for bit.
  * Limits and alignment as the other *_ws calls (bf16, d = 128, C = 64, ...).
@@ -245,15 +246,17 @@ int pisa_sparse_attn_backward_ws(const pisa_cfg *cfg, const void *Q, const void 
  * pisa_forward_ws or pisa_sparse_attn_ws left in it for the same cfg, Q, K, V
  * and idx, with nothing else run on it since (it must be at least
  * pisa_backward_workspace_bytes(cfg) bytes for both calls). Those calls leave
- * the normaliser, the fp32 output and the grouping of the selected leaves
- * there, which is the state the recompute would rebuild. Results and limits as
- * pisa_sparse_attn_backward_ws; the contents are not checked. */
+ * the normaliser, the fp32 output (D = dO . O is taken from it) and the
+ * grouping of the selected leaves there, so the statistics pass is skipped.
+ * Results and limits as pisa_sparse_attn_backward_ws; the contents are not
+ * checked. */
 int pisa_sparse_attn_backward_saved_ws(const pisa_cfg *cfg, const void *Q, const void *K, const void *V,
                                        const int32_t *idx, const void *dO, float *dQ, float *dK, float *dV,
                                        void *workspace, size_t workspace_bytes, void *stream);
 /* pisa_sparse_attn_backward_ws recording caller events (as
- * pisa_forward_ws_events) at its phase boundaries: 0 forward recompute,
- * 1 D, zeroing and the tile list, 2 backward tiles; index 3 marks the end. */
+ * pisa_forward_ws_events) at its phase boundaries: 0 statistics (grouping,
+ * tile list, statistics pass, combine), 1 zeroing of the gradients,
+ * 2 backward tiles; index 3 marks the end. */
 #define PISA_NUM_BWD_PHASES 3
 int pisa_sparse_attn_backward_ws_events(const pisa_cfg *cfg, const void *Q, const void *K, const void *V,
                                         const int32_t *idx, const void *dO, float *dQ, float *dK, float *dV,
