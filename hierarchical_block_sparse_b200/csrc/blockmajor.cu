@@ -1018,7 +1018,8 @@ __global__ void finalize_kernel(const float* __restrict__ oacc, __nv_bfloat16* _
 // Backward of the attention with the selection fixed (close reading §02 Eq.(2)
 // differentiated; §5.3: gradients reach only the selected entries), key-major
 // on the tensor cores. Per (query row i, selected key j) with the normaliser
-// L_i (log2 units) and D_i = dO_i . o_i of the recomputed forward:
+// L_i (log2 units) and D_i = dO_i . o_i (from the statistics pass below, or
+// from a saved forward):
 //   p = 2^(s*scale - L),  dp = dO_i . v_j,  ds = p (dp - D),
 //   dV_j += p dO_i,  dK_j += ds q_i / sqrt(d),  dQ_i += ds k_j / sqrt(d).
 // Rows are grouped by leaf: bucket (b, kv-head, leaf) holds first the leaf's
@@ -1106,8 +1107,8 @@ __global__ void __launch_bounds__(kScanBlock) bwd_place_kernel(const int32_t* __
     if (blockIdx.x == gridDim.x - 1 && threadIdx.x == kScanBlock - 1) *ntiles = (int32_t)(s_pre + t);
 }
 
-// D = dO . O per (query, head), O from the fp32 accumulator of the recomputed
-// forward; one warp per row of [B, Hq, N], written as [B, Hkv, N, G]
+// D = dO . O per (query, head), O from the fp32 accumulator a saved forward
+// left in the workspace; one warp per row of [B, Hq, N], written as [B, Hkv, N, G]
 template <int G>
 __global__ void bwd_delta_kernel(const __nv_bfloat16* __restrict__ dO, const float* __restrict__ oacc,
                                  float* __restrict__ Dr, int64_t rows, int N, int Hq) {
@@ -1841,7 +1842,7 @@ static cudaError_t attn_bm_t(const void* Q, const void* K, const void* V, const 
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     mark(ev, 8, st);
-    if (O) {  // without O the fp32 accumulator in the workspace is the result (the backward's recompute)
+    if (O) {  // without O the fp32 accumulator in the workspace is the result
         finalize_kernel<<<sm_count() * 8, 256, 0, st>>>(oacc, (__nv_bfloat16*)O, nO / 4);
         e = cudaGetLastError();
     }

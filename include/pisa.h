@@ -241,7 +241,7 @@ int64_t pisa_backward_workspace_bytes(const pisa_cfg *cfg);
 int pisa_sparse_attn_backward_ws(const pisa_cfg *cfg, const void *Q, const void *K, const void *V,
                                  const int32_t *idx, const void *dO, float *dQ, float *dK, float *dV,
                                  void *workspace, size_t workspace_bytes, void *stream);
-/* pisa_sparse_attn_backward_ws without the forward recompute, for training
+/* pisa_sparse_attn_backward_ws without the statistics pass, for training
  * steps that keep the forward's workspace: the workspace must hold what
  * pisa_forward_ws or pisa_sparse_attn_ws left in it for the same cfg, Q, K, V
  * and idx, with nothing else run on it since (it must be at least
