@@ -429,6 +429,40 @@ int pisa_pyramid_grow(const pisa_cfg* cfg_old, const float* pyr_old, const pisa_
                                            (cudaStream_t)stream));
 }
 
+int64_t pisa_cache_capacity(int64_t n, int C) {
+    if (C <= 0 || n < 0) return PISA_E_INVALID;
+    int64_t cap = C;
+    while (cap < n) {
+        if (cap > ((int64_t)1 << 40)) return PISA_E_UNSUPPORTED;
+        cap *= 2;
+    }
+    return cap;
+}
+
+int pisa_cache_grow(const pisa_cfg* cfg_old, const void* Kc_old, const void* Vc_old, const float* pyr_old,
+                    const pisa_cfg* cfg_new, void* Kc_new, void* Vc_new, float* pyr_new, void* stream) {
+    int s = check_gpu(cfg_old);
+    if (s) return s;
+    s = check_gpu(cfg_new);
+    if (s) return s;
+    if (cfg_old->B != cfg_new->B || cfg_old->Hq != cfg_new->Hq || cfg_old->Hkv != cfg_new->Hkv ||
+        cfg_old->d != cfg_new->d || cfg_old->C != cfg_new->C || cfg_old->g != cfg_new->g ||
+        cfg_old->dtype != cfg_new->dtype || cfg_new->N < cfg_old->N)
+        return PISA_E_INVALID;
+    if (cfg_old->N == 0) return PISA_OK;
+    if (!Kc_old || !Vc_old || !Kc_new || !Vc_new || Kc_new == Kc_old || Vc_new == Vc_old || Kc_new == Vc_new)
+        return PISA_E_INVALID;
+    if (!aligned16(Kc_old) || !aligned16(Vc_old) || !aligned16(Kc_new) || !aligned16(Vc_new))
+        return PISA_E_ALIGNMENT;
+    const int64_t units = (int64_t)cfg_new->B * cfg_new->Hkv;
+    const int row_bytes = cfg_new->d * (cfg_new->dtype == PISA_DTYPE_BF16 ? 2 : 4);
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaError_t e = launch_cache_grow(Kc_old, Kc_new, units, cfg_old->N, cfg_new->N, row_bytes, st);
+    if (e == cudaSuccess) e = launch_cache_grow(Vc_old, Vc_new, units, cfg_old->N, cfg_new->N, row_bytes, st);
+    if (e != cudaSuccess) return PISA_E_CUDA;
+    return pisa_pyramid_grow(cfg_old, pyr_old, cfg_new, pyr_new, stream);
+}
+
 int pisa_pyramid_append(const pisa_cfg* cfg, void* Kc, void* Vc, float* pyr, const void* k_new, const void* v_new,
                         const int32_t* pos, void* stream) {
     int s = check_gpu(cfg);

@@ -66,6 +66,8 @@ cudaError_t launch_attn_bwd(int dtype, int d, const void* Q, const void* K, cons
                             const void* dO, float* dQ, float* dK, float* dV, const AttnParams& p, cudaStream_t st);
 cudaError_t launch_pyramid_grow(const float* old_pyr, float* new_pyr, int64_t units, int d, const Geom& go,
                                 const Geom& gn, cudaStream_t st);
+cudaError_t launch_cache_grow(const void* src, void* dst, int64_t units, int64_t rows_old, int64_t rows_new,
+                              int row_bytes, cudaStream_t st);
 cudaError_t launch_select(int dtype, int d, const void* Q, const void* K, const float* pyr, int32_t* idx,
                           const SelectParams& p, cudaStream_t st);
 cudaError_t launch_attn(int dtype, int d, const void* Q, const void* K, const void* V, const int32_t* idx,

@@ -162,6 +162,31 @@ cudaError_t launch_pyramid_grow(const float* old_pyr, float* new_pyr, int64_t un
     return cudaGetLastError();
 }
 
+// K or V cache rows into a cache of a larger capacity: per (b, kv-head) unit,
+// rows [0, rows_old) are copied and rows [rows_old, rows_new) are zeroed; one
+// 16-byte chunk per thread and step of a grid-stride loop.
+__global__ void __launch_bounds__(256) cache_grow_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst,
+                                                         int64_t units, int64_t rows_old, int64_t rows_new,
+                                                         int chunks) {
+    const int64_t total = units * rows_new * chunks;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t c = i % chunks, r = (i / chunks) % rows_new, u = i / (chunks * rows_new);
+        dst[i] = r < rows_old ? src[(u * rows_old + r) * chunks + c] : make_uint4(0u, 0u, 0u, 0u);
+    }
+}
+
+cudaError_t launch_cache_grow(const void* src, void* dst, int64_t units, int64_t rows_old, int64_t rows_new,
+                              int row_bytes, cudaStream_t st) {
+    const int chunks = row_bytes / 16;
+    const int64_t total = units * rows_new * chunks;
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t want = (total + 255) / 256, cap = (int64_t)sms * 16;
+    cache_grow_kernel<<<(unsigned)(want < cap ? want : cap), 256, 0, st>>>((const uint4*)src, (uint4*)dst, units,
+                                                                          rows_old, rows_new, chunks);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_pool(int dtype, int d, const void* K, float* pyr, const PoolParams& p, cudaStream_t st) {
     if (dtype == 1) {
         if (d == 128) return launch_pool_t<__nv_bfloat16, 128>(K, pyr, p, st);

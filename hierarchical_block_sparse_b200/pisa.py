@@ -82,6 +82,8 @@ def load(path: str | None = None):
             "pisa_build_pyramid_prefix": (ctypes.c_int, [cfgp, P, P, P, P]),
             "pisa_pyramid_append": (ctypes.c_int, [cfgp, P, P, P, P, P, P, P]),
             "pisa_pyramid_grow": (ctypes.c_int, [cfgp, P, cfgp, P, P]),
+            "pisa_cache_capacity": (ctypes.c_int64, [ctypes.c_int64, ctypes.c_int]),
+            "pisa_cache_grow": (ctypes.c_int, [cfgp, P, P, P, cfgp, P, P, P, P]),
             "pisa_sparse_attn_backward": (ctypes.c_int, [cfgp, P, P, P, P, P, P, P, P, P]),
             "pisa_backward_workspace_bytes": (ctypes.c_int64, [cfgp]),
             "pisa_sparse_attn_backward_ws": (ctypes.c_int, [cfgp, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]),
@@ -318,6 +320,55 @@ def pisa_sparse_attn_backward_ws_events(cfg, Q, K, V, idx, dO, dQ, dK, dV, ws, e
 def pisa_pyramid_grow(cfg_old, pyr_old, cfg_new, pyr_new):
     _check("pisa_pyramid_grow", load().pisa_pyramid_grow(ctypes.byref(cfg_old), _ptr(pyr_old), ctypes.byref(cfg_new),
                                                          _ptr(pyr_new), _stream()))
+
+
+def pisa_cache_capacity(n: int, C: int) -> int:
+    """The library's geometric capacity for n cached keys (smallest C * 2^k >= n)."""
+    r = int(load().pisa_cache_capacity(int(n), int(C)))
+    if r < 0:
+        _check("pisa_cache_capacity", r)
+    return r
+
+
+def pisa_cache_grow(cfg_old, Kc_old, Vc_old, pyr_old, cfg_new, Kc_new, Vc_new, pyr_new):
+    _check("pisa_cache_grow", load().pisa_cache_grow(ctypes.byref(cfg_old), _ptr(Kc_old), _ptr(Vc_old), _ptr(pyr_old),
+                                                     ctypes.byref(cfg_new), _ptr(Kc_new), _ptr(Vc_new),
+                                                     _ptr(pyr_new), _stream()))
+
+
+class DecodeCache:
+    """K and V caches [B, Hkv, capacity, d] and their pyramid, grown by the
+    library's geometric policy: before a step would write at or past the
+    capacity, buffers of pisa_cache_capacity(needed) rows are allocated (torch)
+    and pisa_cache_grow moves the contents. cfg.N is the capacity. The
+    per-sequence positions stay in the caller's pos tensor."""
+
+    def __init__(self, cfg, Kc: torch.Tensor, Vc: torch.Tensor, pyr: torch.Tensor):
+        self.cfg, self.Kc, self.Vc, self.pyr = cfg, Kc, Vc, pyr
+
+    @property
+    def capacity(self) -> int:
+        return int(self.cfg.N)
+
+    def reserve(self, n: int) -> None:
+        """Make room for n keys per sequence (grows geometrically when needed)."""
+        if n <= self.cfg.N:
+            return
+        c = self.cfg
+        new = PisaCfg(c.B, c.Hq, c.Hkv, pisa_cache_capacity(n, c.C), c.d, c.C, c.K, c.g, c.causal, c.forced_mask,
+                      c.dtype, c.score_variant)
+        shape = (c.B, c.Hkv, new.N, c.d)
+        Kc = torch.empty(shape, dtype=self.Kc.dtype, device=self.Kc.device)
+        Vc = torch.empty(shape, dtype=self.Vc.dtype, device=self.Vc.device)
+        pyr = torch.empty((c.B, c.Hkv, pisa_pyramid_rows(new), c.d), dtype=torch.float32, device=self.pyr.device)
+        pisa_cache_grow(c, self.Kc, self.Vc, self.pyr, new, Kc, Vc, pyr)
+        self.cfg, self.Kc, self.Vc, self.pyr = new, Kc, Vc, pyr
+
+    def step(self, q_new, k_new, v_new, pos, idx, o, max_pos: int) -> None:
+        """pisa_decode_step for every sequence, growing first if the largest
+        position (max_pos, a host value: no device read) reaches the capacity."""
+        self.reserve(max_pos + 1)
+        pisa_decode_step(self.cfg, q_new, k_new, v_new, self.Kc, self.Vc, self.pyr, pos, idx, o)
 
 
 def pisa_decode(cfg, q_new, Kc, Vc, pyr, pos, idx, o):

@@ -307,6 +307,23 @@ int pisa_build_pyramid_prefix(const pisa_cfg *cfg, const void *Kc, const int32_t
 int pisa_pyramid_grow(const pisa_cfg *cfg_old, const float *pyr_old, const pisa_cfg *cfg_new, float *pyr_new,
                       void *stream);
 
+/* Geometric capacity policy of a growing decode cache (close reading §5.3:
+ * capacity grows by a fixed ratio, so the upkeep stays amortised O(1) copies
+ * per token): the smallest C * 2^k (k >= 0) that holds n keys. Host only, no
+ * GPU; PISA_E_INVALID for n < 0 or C <= 0, PISA_E_UNSUPPORTED past 2^41. */
+int64_t pisa_cache_capacity(int64_t n, int C);
+
+/* Grow a whole decode cache: K and V caches ([B, Hkv, cfg_old->N, d] of the
+ * cfg dtype) are copied into caches of capacity cfg_new->N (rows from the old
+ * capacity on are zeroed) and the pyramid is re-laid out as pisa_pyramid_grow
+ * does; all on `stream`, in the library's kernels. The caller allocates the
+ * new buffers (pisa_cache_capacity gives the size to grow to) and keeps its
+ * per-sequence positions. Config rules as pisa_pyramid_grow; null, aliased
+ * (new == old, or K and V sharing a buffer) pointers give PISA_E_INVALID,
+ * pointers not 16-byte aligned PISA_E_ALIGNMENT. */
+int pisa_cache_grow(const pisa_cfg *cfg_old, const void *Kc_old, const void *Vc_old, const float *pyr_old,
+                    const pisa_cfg *cfg_new, void *Kc_new, void *Vc_new, float *pyr_new, void *stream);
+
 /* Append one token per sequence: k_new, v_new [B, Hkv, d] are written to cache
  * row pos[b]; the leaf holding pos[b] and each of its ancestors is recomputed
  * as the mean of what exists at length pos[b] + 1 (O(C + L) work per head). */

@@ -175,3 +175,32 @@ def test_backward_workspace_validates_before_launch(lib):
         setattr(c2, field, value)
         assert lib.pisa_backward_workspace_bytes(ctypes.byref(c2)) == -2
         assert call(ctypes.byref(c2), *P, ctypes.c_void_p(8192), need, None) == -2
+
+
+def test_cache_capacity_policy(lib):
+    # the smallest C * 2^k holding n keys (geometric growth)
+    assert [pisa.pisa_cache_capacity(n, 64) for n in (0, 1, 64, 65, 128, 129, 262144, 262145)] == \
+        [64, 64, 64, 128, 128, 256, 262144, 524288]
+    assert pisa.pisa_cache_capacity(1000, 48) == 48 * 32
+    assert lib.pisa_cache_capacity(-1, 64) == -1
+    assert lib.pisa_cache_capacity(10, 0) == -1
+
+
+def test_cache_grow_validates_before_launch(lib):
+    old = pisa.make_cfg(B=2, Hq=2, Hkv=2, N=2048, d=128, C=64, K=8)
+    new = pisa.make_cfg(B=2, Hq=2, Hkv=2, N=4096, d=128, C=64, K=8)
+    P = [ctypes.c_void_p(4096 * (i + 1)) for i in range(6)]  # Kc_old, Vc_old, pyr_old, Kc_new, Vc_new, pyr_new
+    grow = lib.pisa_cache_grow
+
+    def call(o, n, p):
+        return grow(ctypes.byref(o), p[0], p[1], p[2], ctypes.byref(n), p[3], p[4], p[5], None)
+
+    assert call(new, old, P) == -1                                  # smaller new capacity
+    bad = pisa.make_cfg(B=2, Hq=2, Hkv=1, N=4096, d=128, C=64, K=8)
+    assert call(old, bad, P) == -1                                  # other fields differ
+    assert call(old, new, [P[0], P[1], P[2], P[0], P[4], P[5]]) == -1  # K in place
+    assert call(old, new, [P[0], P[1], P[2], P[3], P[3], P[5]]) == -1  # K and V share a buffer
+    assert call(old, new, [P[0], None, P[2], P[3], P[4], P[5]]) == -1
+    assert call(old, new, [P[0], P[1], P[2], ctypes.c_void_p(8 + 4096 * 9), P[4], P[5]]) == -4
+    empty = pisa.make_cfg(B=2, Hq=2, Hkv=2, N=0, d=128, C=64, K=8)
+    assert call(empty, new, P) == 0

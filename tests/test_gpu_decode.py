@@ -209,3 +209,44 @@ def test_pyramid_grow_then_decode_past_the_old_capacity():
             _check_seq(w, cap_new, Kh, Vh, pyr[s], n, q[s], idx[s], o[s])
         pos += 1
     assert int(pos[1]) > cap_old
+
+
+def test_decode_cache_grows_geometrically_inside_the_library():
+    # DecodeCache grows by the library's policy (pisa_cache_capacity) before a
+    # step would write past the capacity; pisa_cache_grow moves K, V and the
+    # pyramid in the library's kernels, and decoding continues past the old capacity
+    w = Workload("dec_grow2", 123, B=1, Hq=4, Hkv=2, N=0, d=128, C=64, K=8, decode_batch=2)
+    cap_old = 2048
+    lens = [1800, 2046]
+    dev = torch.device("cuda", 0)
+    Kc, Vc, Kp, Vp = decode_cache(w, cap_old, 2047, dev)
+    Khost = [decode_rows(Kp, s, 2047) for s in range(2)]
+    Vhost = [decode_rows(Vp, s, 2047) for s in range(2)]
+    for s in range(2):
+        Kc[s, :, lens[s]:] = 0
+        Vc[s, :, lens[s]:] = 0
+    cfg = _cfg(w, 2, cap_old)
+    pyr = torch.zeros((2, w.Hkv, pisa.pisa_pyramid_rows(cfg), w.d), dtype=torch.float32, device=dev)
+    pos = torch.tensor(lens, dtype=torch.int32, device=dev)
+    pisa.pisa_build_pyramid_prefix(cfg, Kc, pos, pyr)
+    cache = pisa.DecodeCache(cfg, Kc, Vc, pyr)
+    caps = []
+    for step in range(5):  # sequence 1 writes positions 2046..2050: the cache grows before position 2048
+        q, k, v = decode_step_inputs(w, step, B=2)
+        idx = torch.full((2, w.Hkv, w.K), -7, dtype=torch.int32, device=dev)
+        o = torch.empty((2, w.Hq, w.d), dtype=q.dtype, device=dev)
+        cache.step(q.to(dev), k.to(dev), v.to(dev), pos, idx, o, max_pos=max(lens) + step)
+        torch.cuda.synchronize()
+        caps.append(cache.capacity)
+        for s in range(2):
+            n = int(pos[s])
+            Kh = torch.cat([Khost[s][:, :n], k[s][:, None]], 1)
+            Vh = torch.cat([Vhost[s][:, :n], v[s][:, None]], 1)
+            Khost[s], Vhost[s] = Kh, Vh
+            _check_seq(w, cache.capacity, Kh, Vh, cache.pyr[s], n, q[s], idx[s], o[s])
+            # the grown caches hold every row written so far, zeros past it
+            assert torch.equal(cache.Kc[s, :, :n + 1].cpu(), Kh)
+            assert torch.equal(cache.Vc[s, :, :n + 1].cpu(), Vh)
+            assert not cache.Kc[s, :, n + 1:].any()
+        pos += 1
+    assert caps == [2048, 2048, 4096, 4096, 4096]
