@@ -358,9 +358,11 @@ class DecodeCache:
         new = PisaCfg(c.B, c.Hq, c.Hkv, pisa_cache_capacity(n, c.C), c.d, c.C, c.K, c.g, c.causal, c.forced_mask,
                       c.dtype, c.score_variant)
         shape = (c.B, c.Hkv, new.N, c.d)
-        Kc = torch.empty(shape, dtype=self.Kc.dtype, device=self.Kc.device)
-        Vc = torch.empty(shape, dtype=self.Vc.dtype, device=self.Vc.device)
-        pyr = torch.empty((c.B, c.Hkv, pisa_pyramid_rows(new), c.d), dtype=torch.float32, device=self.pyr.device)
+        # growing writes every row of the new buffers, except from an empty cache (nothing to move)
+        alloc = torch.zeros if c.N == 0 else torch.empty
+        Kc = alloc(shape, dtype=self.Kc.dtype, device=self.Kc.device)
+        Vc = alloc(shape, dtype=self.Vc.dtype, device=self.Vc.device)
+        pyr = alloc((c.B, c.Hkv, pisa_pyramid_rows(new), c.d), dtype=torch.float32, device=self.pyr.device)
         pisa_cache_grow(c, self.Kc, self.Vc, self.pyr, new, Kc, Vc, pyr)
         self.cfg, self.Kc, self.Vc, self.pyr = new, Kc, Vc, pyr
 

@@ -320,7 +320,9 @@ int64_t pisa_cache_capacity(int64_t n, int C);
  * new buffers (pisa_cache_capacity gives the size to grow to) and keeps its
  * per-sequence positions. Config rules as pisa_pyramid_grow; null, aliased
  * (new == old, or K and V sharing a buffer) pointers give PISA_E_INVALID,
- * pointers not 16-byte aligned PISA_E_ALIGNMENT. */
+ * pointers not 16-byte aligned PISA_E_ALIGNMENT. From an empty cache
+ * (cfg_old->N == 0) there is nothing to move: the call returns PISA_OK and
+ * leaves the new buffers as they are (the caller zeroes them). */
 int pisa_cache_grow(const pisa_cfg *cfg_old, const void *Kc_old, const void *Vc_old, const float *pyr_old,
                     const pisa_cfg *cfg_new, void *Kc_new, void *Vc_new, float *pyr_new, void *stream);
 
