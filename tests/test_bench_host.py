@@ -37,3 +37,16 @@ def test_walk_counts_match_oracle(N, C, K, mask):
 
 def test_fp32_peak_formula():
     assert abs(bench.fp32_fma_peak_tflops(1965.0) - 74.45) < 0.01
+
+
+def test_kernel_source_sections_resolve():
+    # every kernel's measured-traffic key hashes existing files and section
+    # markers (a renamed section would otherwise silently drop the record)
+    for name, parts in bench.KERNEL_SOURCES.items():
+        assert len(bench.source_sha(parts)) == 16, name
+
+
+def test_measured_traffic_is_keyed_by_workload_and_source():
+    assert bench.measured_traffic("stage1", "no_such_workload") is None
+    rec = bench.measured_traffic("stage1", "mha8_n256k")
+    assert rec is None or rec > 0
