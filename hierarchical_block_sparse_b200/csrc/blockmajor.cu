@@ -24,10 +24,14 @@
 //   through the grouping, whose atomics would otherwise pile onto a few leaves.
 // Attention (attn_tile_kernel): the kept non-forced (query, leaf) pairs are
 //   grouped the same way; per tile S = Q K^T (tcgen05, TMEM), P = 2^(S*scale - Z)
-//   in bf16, O_part = P V (tcgen05, V as an MN-major operand), and O_part is
-//   added into the accumulator with vector reductions; P is already
-//   normalised, so no rescaling is needed.
+//   in bf16, O_part = P V (tcgen05, V as an MN-major operand), and each row of
+//   O_part is added into the accumulator with one 512-byte bulk reduction; P
+//   is already normalised, so no rescaling is needed.
 // finalize_kernel converts the accumulator to the output dtype.
+// Backward with the selection fixed (bwd_*): the same leaf grouping plus each
+//   leaf's forced section; a statistics pass (S and dP per tile) gives every
+//   (query, head) its normaliser and D, then key-major tiles accumulate dK and
+//   dV per leaf in TMEM and add dQ rows with bulk reductions.
 #include <cmath>
 #include <type_traits>
 
