@@ -1,5 +1,8 @@
-"""GPU parity of pisa_sparse_attn_backward (fixed selection) against the
-oracle's fp64 backward, on the selection the GPU itself made."""
+"""GPU parity of the backward with the selection fixed -- the CUDA-core call
+(pisa_sparse_attn_backward) and the tensor-core calls
+(pisa_sparse_attn_backward_ws, pisa_sparse_attn_backward_saved_ws) -- against
+the oracle's fp64 backward, on the selection the GPU itself made; at the
+bench's size on sampled rows and leaves."""
 import numpy as np
 import pytest
 import torch
