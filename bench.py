@@ -312,6 +312,142 @@ def size_oracle_sample(w, Q, K, V, target_s: float):
     return int(min(max(8, budget / max(per_row, 1e-6)), Q.shape[2]))
 
 
+# ------------------------------------------------------- measured FMA peak ----
+
+def measure_fma_peak(dev, stream, blocks_per_sm: int = 8, iters: int = 20000, reps: int = 5):
+    """fp32 FMA throughput of this GPU, measured with pisa_fma_probe (scalar and
+    packed fp32x2 chains, full occupancy), CUDA events on the launch stream,
+    with the SM clock sampled during the timed launches."""
+    import torch
+    from hierarchical_block_sparse_b200 import pisa
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    blocks = sms * blocks_per_sm
+    out = torch.empty(blocks * 256, dtype=torch.float32, device=dev)
+    res = {}
+    with ClockSampler(dev.index) as clk:
+        for packed in (False, True):
+            for _ in range(2):
+                pisa.pisa_fma_probe(out, blocks, iters, packed)
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(reps):
+                pisa.pisa_fma_probe(out, blocks, iters, packed)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            flop = blocks * 256.0 * iters * 64 * (2 if packed else 1) * reps
+            res["packed_tflops" if packed else "scalar_tflops"] = flop / (e0.elapsed_time(e1) / 1e3) / 1e12
+    res["tflops"] = max(res["scalar_tflops"], res["packed_tflops"])
+    res["clocks"] = clk.summary()
+    res["how"] = (f"pisa_fma_probe: {blocks} blocks x 256 threads, 8 independent chains of {4 * iters} FMAs each, "
+                  f"scalar and packed fp32x2, {reps} launches after 2 warm-up, CUDA events")
+    return res
+
+
+def dominant_roofline(w, phase_ms, alg, pk, fma_peak, fma_note, tc_peak):
+    """Roofline entry for the phase that takes the most time."""
+    dom = max(phase_ms, key=phase_ms.get)
+    t_dom = phase_ms[dom] / 1e3
+    tc_note = "bf16 dense, sustained (MEASURED_PEAKS.json)"
+    if dom == "attn_tiles":
+        roof = {"kernel": "attn_tile_kernel", "bound": "tensor", "achieved": alg["attn_free_flops"] / t_dom / 1e12,
+                "peak": tc_peak, "unit": "TFLOP/s", "algorithmic_per_launch": alg["attn_free_flops"],
+                "peak_note": tc_note}
+    elif dom == "forced_tiles":
+        roof = {"kernel": "forced_tile_kernel", "bound": "tensor",
+                "achieved": alg["attn_forced_flops"] / t_dom / 1e12, "peak": tc_peak, "unit": "TFLOP/s",
+                "algorithmic_per_launch": alg["attn_forced_flops"], "peak_note": tc_note}
+    elif dom == "leaf_scores":
+        roof = {"kernel": "leaf_score_kernel", "bound": "tensor", "achieved": alg["leaf_flops"] / t_dom / 1e12,
+                "peak": tc_peak, "unit": "TFLOP/s", "algorithmic_per_launch": alg["leaf_flops"],
+                "peak_note": tc_note}
+    elif dom == "stage1":
+        roof = {"kernel": "stage1_kernel", "bound": "alu", "achieved": alg["internal_flops"] / t_dom / 1e12,
+                "peak": fma_peak, "unit": "TFLOP/s", "algorithmic_per_launch": alg["internal_flops"],
+                "peak_note": fma_note}
+    else:
+        b = alg["pool_bytes"] if dom == "pyramid" else alg["selection_bytes"]
+        roof = {"kernel": dom, "bound": "hbm", "achieved": b / t_dom / 1e9, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "algorithmic_per_launch": b}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = measured_traffic(dom, w.name)
+    roof["launch_ms"] = phase_ms[dom]
+    return roof
+
+
+SELECTION_PHASES = ("pyramid", "stage1", "group_candidates", "leaf_scores", "topk")
+
+
+def time_bsa(cfg, Qd, Kd, pyr, idx, stream):
+    """Flat BSA selection (pyramid + Eq.1 scan over every eligible leaf), ms."""
+    import torch
+    from hierarchical_block_sparse_b200 import pisa
+    bidx = torch.empty_like(idx)
+    pisa.pisa_build_pyramid(cfg, Kd, pyr)
+    pisa.pisa_bsa_select(cfg, Qd, pyr, bidx)
+    torch.cuda.synchronize()
+    b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    b0.record(stream)
+    pisa.pisa_build_pyramid(cfg, Kd, pyr)
+    pisa.pisa_bsa_select(cfg, Qd, pyr, bidx)
+    b1.record(stream)
+    torch.cuda.synchronize()
+    return b0.elapsed_time(b1)
+
+
+def prefill_config_line(w, dev, stream, steps, warmup, pk, fma_peak, fma_note, tc_peak, bsa=True):
+    """One workload's prefill measured like the headline step (pisa_forward_ws,
+    phase events on the launch stream, inputs larger than L2): ms per step,
+    tokens/s, selection ms, the dominant kernel's roofline, HBM fractions and
+    the flat BSA selection beside it."""
+    import torch
+    from hierarchical_block_sparse_b200 import pisa
+    from hierarchical_block_sparse_b200.workloads import make_inputs
+    Q, K, V, _ = make_inputs(w)
+    Qd, Kd, Vd = Q.to(dev), K.to(dev), V.to(dev)
+    del Q, K, V
+    cfg = pisa.cfg_for(Qd, Kd, C=w.C, K_=w.K, causal=w.causal, forced_mask=w.forced_mask)
+    pyr, idx, O = pisa.alloc_outputs(cfg, dev, Qd.dtype)
+    work = pisa.alloc_workspace(cfg, dev)
+    nph = len(pisa.PHASES)
+    for _ in range(warmup):
+        pisa.pisa_forward_ws(cfg, Qd, Kd, Vd, pyr, idx, O, work)
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nph + 1)] for _ in range(steps)]
+    for e in evs:
+        for x in e:
+            x.record(stream)
+    torch.cuda.synchronize()
+    for e in evs:
+        pisa.pisa_forward_ws_events(cfg, Qd, Kd, Vd, pyr, idx, O, work, e)
+    torch.cuda.synchronize()
+    if pisa.pisa_workspace_status(cfg, work) != 0:
+        raise RuntimeError(f"a tensor-core tile timed out ({w.name})")
+    ms = evs[0][0].elapsed_time(evs[-1][nph]) / steps
+    phase_ms = {name: float(np.mean([e[i].elapsed_time(e[i + 1]) for e in evs])) for i, name in enumerate(pisa.PHASES)}
+    sel = sum(phase_ms[k] for k in SELECTION_PHASES)
+    alg = algorithmic(w, w.N)
+    hbm = pk["hbm_gbs"] * 1e9
+    out = {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d, "C": w.C, "K": w.K,
+           "steps": steps, "ms_per_step": ms, "tokens_per_s": w.B * w.N / (ms / 1e3),
+           "selection_ms": sel, "attention_ms": ms - sel, "phase_ms": phase_ms,
+           "hbm_roofline_frac": {"prefill": alg["prefill_bytes"] / (ms / 1e3) / hbm,
+                                 "selection": alg["selection_bytes"] / (sel / 1e3) / hbm,
+                                 "pyramid": alg["pool_bytes"] / (phase_ms["pyramid"] / 1e3) / hbm},
+           "roofline": dominant_roofline(w, phase_ms, alg, pk, fma_peak, fma_note, tc_peak),
+           "work": {"internal_tflop": alg["internal_flops"] / 1e12, "leaf_tflop": alg["leaf_flops"] / 1e12,
+                    "attn_tflop": alg["attn_flops"] / 1e12}}
+    if bsa:
+        out["bsa_selection_ms"] = time_bsa(cfg, Qd, Kd, pyr, idx, stream)
+        out["pisa_vs_bsa_selection_speedup"] = out["bsa_selection_ms"] / sel
+    del Qd, Kd, Vd, pyr, idx, O, work
+    torch.cuda.empty_cache()
+    return out
+
+
+PER_CONFIG = ("mha16_n16k", "needle_mha16_n64k", "gqa32x8_n128k")
+
+
 # -------------------------------------------------------------------- main ----
 
 def main():
@@ -326,6 +462,7 @@ def main():
     ap.add_argument("--no-variants", action="store_true", help="skip timing the PISA-1 / PISA-2 scores")
     ap.add_argument("--no-backward", action="store_true", help="skip timing the attention backward")
     ap.add_argument("--no-per-query", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true", help="skip the 16K / 64K / 128K workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=16.0)
     ap.add_argument("--decode-batch", type=int, default=0, help="override the decode batch (profiling)")
@@ -423,36 +560,17 @@ def main():
     alg = algorithmic(w, w.N)
     pk = peaks()
     clocks = clk.summary()
-    fma_peak = fp32_fma_peak_tflops(pk["sm_max_mhz"])
     tc_peak = pk["bf16_tflops_sustained"] or pk["bf16_tflops"]
-    dom = max(phase_ms, key=phase_ms.get)
-    t_dom = phase_ms[dom] / 1e3
-    if dom == "attn_tiles":
-        roof = {"kernel": "attn_tile_kernel", "bound": "tensor", "achieved": alg["attn_free_flops"] / t_dom / 1e12,
-                "peak": tc_peak, "unit": "TFLOP/s", "algorithmic_per_launch": alg["attn_free_flops"],
-                "peak_note": "bf16 dense, sustained (MEASURED_PEAKS.json)"}
-    elif dom == "forced_tiles":
-        roof = {"kernel": "forced_tile_kernel", "bound": "tensor",
-                "achieved": alg["attn_forced_flops"] / t_dom / 1e12, "peak": tc_peak, "unit": "TFLOP/s",
-                "algorithmic_per_launch": alg["attn_forced_flops"],
-                "peak_note": "bf16 dense, sustained (MEASURED_PEAKS.json)"}
-    elif dom == "leaf_scores":
-        roof = {"kernel": "leaf_score_kernel", "bound": "tensor", "achieved": alg["leaf_flops"] / t_dom / 1e12,
-                "peak": tc_peak, "unit": "TFLOP/s", "algorithmic_per_launch": alg["leaf_flops"],
-                "peak_note": "bf16 dense, sustained (MEASURED_PEAKS.json)"}
-    elif dom == "stage1":
-        roof = {"kernel": "stage1_kernel", "bound": "alu", "achieved": alg["internal_flops"] / t_dom / 1e12,
-                "peak": fma_peak, "unit": "TFLOP/s", "algorithmic_per_launch": alg["internal_flops"],
-                "peak_note": "fp32 FMA: 148 SMs x 128 lanes x 2 FLOP x max SM clock"}
-    else:
-        b = alg["pool_bytes"] if dom == "pyramid" else alg["selection_bytes"]
-        roof = {"kernel": dom, "bound": "hbm", "achieved": b / t_dom / 1e9, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                "algorithmic_per_launch": b}
-    roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["traffic"] = measured_traffic(dom, w.name)
-    roof["launch_ms"] = phase_ms[dom]
+    fma = measure_fma_peak(dev, stream)
+    fma_derived = fp32_fma_peak_tflops(pk["sm_max_mhz"])
+    fma_peak = fma["tflops"]
+    fma_note = ("fp32 FMA measured on this GPU with pisa_fma_probe (max of scalar and packed chains); "
+                f"derived 148 SMs x 128 lanes x 2 FLOP x max clock = {fma_derived:.1f} TFLOP/s")
+    roof = dominant_roofline(w, phase_ms, alg, pk, fma_peak, fma_note, tc_peak)
+    if roof["bound"] == "alu":
+        roof["peak_source"] = "measured"
 
-    sel_total = sum(phase_ms[k] for k in ("pyramid", "stage1", "group_candidates", "leaf_scores", "topk"))
+    sel_total = sum(phase_ms[k] for k in SELECTION_PHASES)
     hbm = pk["hbm_gbs"] * 1e9
     out = {
         "metric": metric, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
@@ -470,6 +588,9 @@ def main():
                  "attn_tflop": alg["attn_flops"] / 1e12},
         "roofline": roof,
         "peaks_source": pk["source"],
+        "fp32_fma_peak": {"measured_tflops": fma_peak, "scalar_tflops": fma["scalar_tflops"],
+                          "packed_tflops": fma["packed_tflops"], "derived_tflops": fma_derived,
+                          "clocks": fma["clocks"], "how": fma["how"]},
         "clocks": clocks,
         "gpu_launches": launches_per_step * args.steps,
     }
@@ -538,20 +659,9 @@ def main():
 
     # ---- flat BSA selection, the quadratic comparison ----
     if not args.no_bsa:
-        bidx = torch.empty_like(idx)
-        pisa.pisa_build_pyramid(cfg, Kd, pyr)
-        pisa.pisa_bsa_select(cfg, Qd, pyr, bidx)
-        torch.cuda.synchronize()
-        b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        b0.record(stream)
-        pisa.pisa_build_pyramid(cfg, Kd, pyr)
-        pisa.pisa_bsa_select(cfg, Qd, pyr, bidx)
-        b1.record(stream)
-        torch.cuda.synchronize()
-        out["bsa_selection_ms"] = b0.elapsed_time(b1)
+        out["bsa_selection_ms"] = time_bsa(cfg, Qd, Kd, pyr, idx, stream)
         out["bsa_kernel"] = "per-query CUDA-core flat scan (bsa_kernel)"
         out["pisa_vs_bsa_selection_speedup"] = out["bsa_selection_ms"] / sel_total
-        del bidx
 
     # ---- the same step ranking by the PISA-1 / PISA-2 scores (Eq.8-9 ablations) ----
     if not args.no_variants:
@@ -643,6 +753,20 @@ def main():
 
     del Qd, Kd, Vd, pyr, idx, O, work
     torch.cuda.empty_cache()
+
+    # ---- the other prefill workloads (16K, 64K planted retrieval, 128K GQA 32/8) ----
+    if not args.no_per_config:
+        per = {}
+        for name in PER_CONFIG:
+            wc = WORKLOADS[name]
+            line = prefill_config_line(wc, dev, stream, min(args.steps, 5), 3, pk, fma_peak, fma_note, tc_peak,
+                                       bsa=not args.no_bsa)
+            line["ms_per_step"] = max_over_ranks(line["ms_per_step"], dist, dev)
+            line["tokens_per_s"] = job_tokens_per_s(wc.B * wc.N, world, line["ms_per_step"])
+            per[name] = line
+        out["per_config"] = per
+        out["selection_ms_by_n"] = {str(v["N"]): v["selection_ms"] for v in per.values()}
+        out["selection_ms_by_n"][str(w.N)] = sel_total
 
     if dist:
         dist.barrier()

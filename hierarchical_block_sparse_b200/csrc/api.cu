@@ -64,12 +64,8 @@ int geom_any(const pisa_cfg* c, int64_t* M, int64_t* off, int maxl) {
 }
 
 SelectParams select_params(const pisa_cfg* c, const Geom& g) {
-    SelectParams p;
-    p.B = c->B; p.Hq = c->Hq; p.Hkv = c->Hkv; p.N = c->N; p.C = c->C; p.K = c->K;
-    p.causal = c->causal; p.forced_mask = c->forced_mask;
-    p.qscale = (float)(1.4426950408889634 / sqrt((double)c->d));
+    SelectParams p = select_params_of(c);
     p.geom = g;
-    p.variant = c->score_variant;
     return p;
 }
 
@@ -93,21 +89,41 @@ int check_bm(const pisa_cfg* c) {
     return PISA_OK;
 }
 
-BmShape bm_shape(const pisa_cfg* c) {
-    BmShape s;
-    s.B = c->B; s.Hq = c->Hq; s.Hkv = c->Hkv; s.N = c->N; s.G = c->Hq / c->Hkv;
-    s.M1 = ((int64_t)c->N + c->C - 1) / c->C;
-    Geom g;
-    make_geom(c->N, c->C, &g);
-    s.rows = g.rows;
-    s.variant = c->score_variant;
-    return s;
-}
+BmShape bm_shape(const pisa_cfg* c) { return bm_shape_of(c); }
 
 int check_ws(const pisa_cfg* c, const void* ws, size_t bytes) {
     if (!ws) return PISA_E_INVALID;
     if (((uintptr_t)ws & 255u) != 0) return PISA_E_ALIGNMENT;
     if (bytes < blockmajor_layout(bm_shape(c)).total) return PISA_E_INVALID;
+    return PISA_OK;
+}
+
+// every check pisa_forward_ws makes, before anything is enqueued
+int check_forward_ws(const pisa_cfg* c, const void* Q, const void* K, const void* V, const float* pyr,
+                     const int32_t* idx, const void* O, const void* ws, size_t bytes) {
+    int s = check_bm(c);
+    if (s) return s;
+    if (c->N == 0) return PISA_OK;
+    if (!Q || !K || !V || !pyr || !idx || !O) return PISA_E_INVALID;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned32(pyr) || !aligned16(idx) || !aligned16(O))
+        return PISA_E_ALIGNMENT;
+    return check_ws(c, ws, bytes);
+}
+
+// checks of a pyramid re-layout from cfg_old's capacity to cfg_new's
+int check_grow(const pisa_cfg* o, const pisa_cfg* n) {
+    int s = check_gpu(o);
+    if (s) return s;
+    s = check_gpu(n);
+    if (s) return s;
+    if (o->B != n->B || o->Hq != n->Hq || o->Hkv != n->Hkv || o->d != n->d || o->C != n->C || o->g != n->g ||
+        o->dtype != n->dtype || n->N < o->N)
+        return PISA_E_INVALID;
+    return PISA_OK;
+}
+int check_grow_pyramids(const float* pyr_old, const float* pyr_new) {
+    if (!pyr_old || !pyr_new || pyr_old == pyr_new) return PISA_E_INVALID;
+    if (!aligned16(pyr_old) || !aligned16(pyr_new)) return PISA_E_ALIGNMENT;
     return PISA_OK;
 }
 
@@ -344,15 +360,10 @@ int pisa_sparse_attn_backward_ws_events(const pisa_cfg* cfg, const void* Q, cons
 int pisa_forward_ws_events(const pisa_cfg* cfg, const void* Q, const void* K, const void* V, float* pyr,
                            int32_t* idx, void* O, void* workspace, size_t workspace_bytes, void* const* events,
                            int n_events, void* stream) {
-    int s = check_bm(cfg);
+    int s = check_forward_ws(cfg, Q, K, V, pyr, idx, O, workspace, workspace_bytes);
     if (s) return s;
     if (cfg->N == 0) return PISA_OK;
-    if (!Q || !K || !V || !pyr || !idx || !O) return PISA_E_INVALID;
-    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned32(pyr) || !aligned16(idx) || !aligned16(O))
-        return PISA_E_ALIGNMENT;
     if (n_events < 0 || (n_events > 0 && !events)) return PISA_E_INVALID;
-    s = check_ws(cfg, workspace, workspace_bytes);
-    if (s) return s;
     const PhaseEvents ev{events, n_events};
     cudaStream_t st = (cudaStream_t)stream;
     if (n_events > 0 && events[0]) cudaEventRecord((cudaEvent_t)events[0], st);
@@ -371,7 +382,8 @@ int pisa_forward_ws_events(const pisa_cfg* cfg, const void* Q, const void* K, co
 int pisa_forward_host(const pisa_cfg* cfg, const void* Q_host, const void* K_host, const void* V_host,
                       int32_t* idx_host, void* O_host, void* Q, void* K, void* V, float* pyr, int32_t* idx,
                       void* O, void* workspace, size_t workspace_bytes, void* stream) {
-    int s = check_bm(cfg);
+    // every check of the device step comes first: a failed call enqueues no copy
+    int s = check_forward_ws(cfg, Q, K, V, pyr, idx, O, workspace, workspace_bytes);
     if (s) return s;
     if (cfg->N == 0) return PISA_OK;
     if (!Q_host || !K_host || !V_host || !idx_host || !O_host) return PISA_E_INVALID;
@@ -380,7 +392,6 @@ int pisa_forward_host(const pisa_cfg* cfg, const void* Q_host, const void* K_hos
     const size_t kv_bytes = (size_t)cfg->B * cfg->Hkv * cfg->N * cfg->d * es;
     const size_t idx_bytes = (size_t)cfg->B * cfg->Hkv * cfg->N * cfg->K * sizeof(int32_t);
     cudaStream_t st = (cudaStream_t)stream;
-    if (!Q || !K || !V) return PISA_E_INVALID;
     if (cudaMemcpyAsync(Q, Q_host, q_bytes, cudaMemcpyHostToDevice, st) != cudaSuccess ||
         cudaMemcpyAsync(K, K_host, kv_bytes, cudaMemcpyHostToDevice, st) != cudaSuccess ||
         cudaMemcpyAsync(V, V_host, kv_bytes, cudaMemcpyHostToDevice, st) != cudaSuccess)
@@ -411,17 +422,11 @@ int pisa_build_pyramid_prefix(const pisa_cfg* cfg, const void* Kc, const int32_t
 
 int pisa_pyramid_grow(const pisa_cfg* cfg_old, const float* pyr_old, const pisa_cfg* cfg_new, float* pyr_new,
                       void* stream) {
-    int s = check_gpu(cfg_old);
+    int s = check_grow(cfg_old, cfg_new);
     if (s) return s;
-    s = check_gpu(cfg_new);
-    if (s) return s;
-    if (cfg_old->B != cfg_new->B || cfg_old->Hq != cfg_new->Hq || cfg_old->Hkv != cfg_new->Hkv ||
-        cfg_old->d != cfg_new->d || cfg_old->C != cfg_new->C || cfg_old->g != cfg_new->g ||
-        cfg_old->dtype != cfg_new->dtype || cfg_new->N < cfg_old->N)
-        return PISA_E_INVALID;
     if (cfg_old->N == 0) return PISA_OK;
-    if (!pyr_old || !pyr_new || pyr_old == pyr_new) return PISA_E_INVALID;
-    if (!aligned16(pyr_old) || !aligned16(pyr_new)) return PISA_E_ALIGNMENT;
+    s = check_grow_pyramids(pyr_old, pyr_new);
+    if (s) return s;
     Geom go, gn;
     make_geom(cfg_old->N, cfg_old->C, &go);
     make_geom(cfg_new->N, cfg_new->C, &gn);
@@ -441,19 +446,16 @@ int64_t pisa_cache_capacity(int64_t n, int C) {
 
 int pisa_cache_grow(const pisa_cfg* cfg_old, const void* Kc_old, const void* Vc_old, const float* pyr_old,
                     const pisa_cfg* cfg_new, void* Kc_new, void* Vc_new, float* pyr_new, void* stream) {
-    int s = check_gpu(cfg_old);
+    // every check, the pyramids' included, comes before the first launch
+    int s = check_grow(cfg_old, cfg_new);
     if (s) return s;
-    s = check_gpu(cfg_new);
-    if (s) return s;
-    if (cfg_old->B != cfg_new->B || cfg_old->Hq != cfg_new->Hq || cfg_old->Hkv != cfg_new->Hkv ||
-        cfg_old->d != cfg_new->d || cfg_old->C != cfg_new->C || cfg_old->g != cfg_new->g ||
-        cfg_old->dtype != cfg_new->dtype || cfg_new->N < cfg_old->N)
-        return PISA_E_INVALID;
     if (cfg_old->N == 0) return PISA_OK;
     if (!Kc_old || !Vc_old || !Kc_new || !Vc_new || Kc_new == Kc_old || Vc_new == Vc_old || Kc_new == Vc_new)
         return PISA_E_INVALID;
     if (!aligned16(Kc_old) || !aligned16(Vc_old) || !aligned16(Kc_new) || !aligned16(Vc_new))
         return PISA_E_ALIGNMENT;
+    s = check_grow_pyramids(pyr_old, pyr_new);
+    if (s) return s;
     const int64_t units = (int64_t)cfg_new->B * cfg_new->Hkv;
     const int row_bytes = cfg_new->d * (cfg_new->dtype == PISA_DTYPE_BF16 ? 2 : 4);
     cudaStream_t st = (cudaStream_t)stream;

@@ -3,8 +3,10 @@
 #pragma once
 
 #include <cuda_runtime.h>
+#include <math.h>
 #include <stdint.h>
 
+#include "pisa.h"
 #include "pisa_device.cuh"
 
 namespace pisa {
@@ -60,6 +62,28 @@ size_t blockmajor_bwd_bytes(const BmShape& s);
 cudaError_t launch_attn_bwd_bm(const void* Q, const void* K, const void* V, const int32_t* idx, const void* dO,
                                float* dQ, float* dK, float* dV, const SelectParams& sp, const BmShape& s, void* ws,
                                bool saved, const PhaseEvents* ev, cudaStream_t st);
+
+// The parameter blocks of a problem statement (the public pisa_cfg), built
+// in one place for every entry point that launches the block-major path.
+inline SelectParams select_params_of(const pisa_cfg* c) {
+    SelectParams p;
+    p.B = c->B; p.Hq = c->Hq; p.Hkv = c->Hkv; p.N = c->N; p.C = c->C; p.K = c->K;
+    p.causal = c->causal; p.forced_mask = c->forced_mask;
+    p.qscale = (float)(1.4426950408889634 / sqrt((double)c->d));
+    make_geom(c->N, c->C, &p.geom);
+    p.variant = c->score_variant;
+    return p;
+}
+inline BmShape bm_shape_of(const pisa_cfg* c) {
+    BmShape s;
+    s.B = c->B; s.Hq = c->Hq; s.Hkv = c->Hkv; s.N = c->N; s.G = c->Hq / c->Hkv;
+    s.M1 = ((int64_t)c->N + c->C - 1) / c->C;
+    Geom g;
+    make_geom(c->N, c->C, &g);
+    s.rows = g.rows;
+    s.variant = c->score_variant;
+    return s;
+}
 
 cudaError_t launch_pool(int dtype, int d, const void* K, float* pyr, const PoolParams& p, cudaStream_t st);
 cudaError_t launch_attn_bwd(int dtype, int d, const void* Q, const void* K, const void* V, const int32_t* idx,

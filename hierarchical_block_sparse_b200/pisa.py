@@ -79,6 +79,7 @@ def load(path: str | None = None):
             "pisa_forward_ws_events": (ctypes.c_int, [cfgp, P, P, P, P, P, P, P, ctypes.c_size_t,
                                                       ctypes.POINTER(ctypes.c_void_p), ctypes.c_int, P]),
             "pisa_select_noalloc": (ctypes.c_int, [cfgp, P, P, P, P, P]),
+            "pisa_select_noalloc_status": (ctypes.c_int, [cfgp, P]),
             "pisa_build_pyramid_prefix": (ctypes.c_int, [cfgp, P, P, P, P]),
             "pisa_pyramid_append": (ctypes.c_int, [cfgp, P, P, P, P, P, P, P]),
             "pisa_pyramid_grow": (ctypes.c_int, [cfgp, P, cfgp, P, P]),
@@ -93,6 +94,7 @@ def load(path: str | None = None):
                                                                    ctypes.POINTER(ctypes.c_void_p), ctypes.c_int, P]),
             "pisa_decode": (ctypes.c_int, [cfgp, P, P, P, P, P, P, P, P]),
             "pisa_decode_step": (ctypes.c_int, [cfgp, P, P, P, P, P, P, P, P, P, P]),
+            "pisa_fma_probe": (ctypes.c_int, [P, ctypes.c_int, ctypes.c_int, ctypes.c_int, P]),
             "pisa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
             "pisa_version": (ctypes.c_char_p, []),
         }
@@ -240,6 +242,20 @@ def pisa_select_noalloc(cfg, Q, K, pyr, idx):
     device share it, so they must not overlap on the GPU)."""
     _check("pisa_select_noalloc", load().pisa_select_noalloc(ctypes.byref(cfg), _ptr(Q), _ptr(K), _ptr(pyr),
                                                              _ptr(idx), _stream()))
+
+
+def pisa_select_noalloc_status(cfg) -> int:
+    """Error word of the last pisa_select_noalloc on this device: 0, or -5
+    (PISA_E_TIMEOUT) when a tile gave up a bounded wait or a self-check failed
+    (synchronises the current stream)."""
+    return int(load().pisa_select_noalloc_status(ctypes.byref(cfg), _stream()))
+
+
+def pisa_fma_probe(out, blocks: int, iters: int, packed: bool):
+    """Launch the fp32 FMA throughput probe on the current stream (out: fp32, blocks * 256 elements)."""
+    assert out.numel() >= blocks * 256 and out.dtype == torch.float32
+    _check("pisa_fma_probe", load().pisa_fma_probe(_ptr(out), int(blocks), int(iters), int(bool(packed)),
+                                                   _stream()))
 
 
 PHASES = ["pyramid", "stage1", "group_candidates", "leaf_scores", "topk", "group_kept", "forced_tiles",

@@ -273,14 +273,22 @@ int pisa_sparse_attn_backward_ws_events(const pisa_cfg *cfg, const void *Q, cons
  * caller workspace; it calls no allocating routine.
  * - Problems whose selection scratch exceeds that size return
  *   PISA_E_SCRATCH_LIMIT (about 73 K query units B*Hkv*N for G = 1).
- * - The first call on a device looks up the array's device address (once per
- *   device, that device current); make it before any stream capture.
- * - All calls on a device share the array and it keeps the previous call's
+ * - The first call in a CUDA context (a device's primary context, or one the
+ *   caller made current through the driver API) looks up the array's device
+ *   address there, with that context current; make it before any stream
+ *   capture. A failed lookup is retried on the next call.
+ * - All calls in a context share the array and it keeps the previous call's
  *   contents; each call clears what must start at zero. Calls that overlap on
  *   the GPU (other streams, other threads) race on the array: serialise them. */
 #define PISA_NOALLOC_SCRATCH_BYTES (32u << 20)
 int pisa_select_noalloc(const pisa_cfg *cfg, const void *Q, const void *K, const float *pyr, int32_t *idx,
                         void *stream);
+/* Error word of the last pisa_select_noalloc on this device (no counterpart on
+ * the pages, like the call itself): synchronises `stream` and returns PISA_OK,
+ * or PISA_E_TIMEOUT when a tensor-core tile gave up a bounded wait or a
+ * self-check of the selection failed (its idx is then not to be used).
+ * `cfg` must be the configuration of that call; the same size limits apply. */
+int pisa_select_noalloc_status(const pisa_cfg *cfg, void *stream);
 
 /* ---- decode path (close reading §5.1 last paragraph; §5.3 "decode cache") ----
  * For decode calls cfg->N is the cache CAPACITY: Kc, Vc: [B, Hkv, N, d] and the
@@ -355,6 +363,16 @@ int pisa_decode_step(const pisa_cfg *cfg, const void *q_new, const void *k_new, 
 /* ---- misc --------------------------------------------------------------------- */
 
 /* Static English text for a status code (never NULL). */
+/* ---- measurement ----
+ * CUDA-core fp32 FMA throughput probe (no counterpart on the pages): `blocks`
+ * blocks of 256 threads, each thread running 8 independent chains of
+ * 4 * `iters` FMAs, scalar (`packed` = 0) or packed fp32x2 (`packed` = 1);
+ * FLOP per launch = blocks * 256 * iters * 64 (x2 when packed). `out` receives
+ * blocks * 256 floats (device memory, caller-owned). Returns PISA_E_INVALID on
+ * a null `out` or non-positive sizes. Used to measure the peak that the walk
+ * kernels' arithmetic is compared against. */
+int pisa_fma_probe(float *out, int blocks, int iters, int packed, void *stream);
+
 const char *pisa_status_string(int status);
 /* Library version string, e.g. "pisa-b200 0.1.0 sm_100a". */
 const char *pisa_version(void);

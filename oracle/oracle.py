@@ -315,6 +315,9 @@ def attn_backward_sampled(Qg: np.ndarray, Kh: np.ndarray, Vh: np.ndarray, idx: n
     dV = np.zeros((len(leaves), C, d))
     for li, leaf in enumerate(leaves):
         users = np.nonzero((np.asarray(idx) == leaf).any(axis=1))[0]
+        if len(users) > 2048:  # many users (a forced first leaf): the same sums, batched over the users
+            dK[li], dV[li] = attn_backward_leaf(Qg, Kh, Vh, idx, dOg, int(leaf), C=C, causal=causal)
+            continue
         for t in users:
             for h in range(G):
                 J, p, ds, q, do, KJ = row_terms(int(t), h)
@@ -325,3 +328,43 @@ def attn_backward_sampled(Qg: np.ndarray, Kh: np.ndarray, Vh: np.ndarray, idx: n
                 dV[li, kl] += np.outer(p[m], do)
                 dK[li, kl] += np.outer(ds[m], q) * inv
     return dQ, dK, dV
+
+
+def attn_backward_leaf(Qg: np.ndarray, Kh: np.ndarray, Vh: np.ndarray, idx: np.ndarray, dOg: np.ndarray,
+                       leaf: int, *, C: int, causal: bool = True):
+    """dK and dV of the keys of one leaf (the backward of Eq.(2) over fixed
+    selected leaves, close reading §5.3), summed over every position whose idx
+    lists the leaf, for leaves with many such positions (a forced first leaf
+    has all N of them).
+
+    Per user row t and head h: its softmax normaliser (the log-sum-exp over all
+    of its selected keys, j <= t when causal) and its output o come from
+    attn_rows; then for the leaf's keys j: p_j = exp(q.k_j / sqrt(d) - lse),
+    dp_j = dO . v_j, ds_j = p_j (dp_j - dO . o); dV_j += p_j dO and
+    dK_j += ds_j q / sqrt(d). The same terms as attn_backward_rows, taken for
+    all users at once. Returns (dK [C, d], dV [C, d]) in float64; key rows
+    past N stay zero."""
+    G, N, d = Qg.shape
+    inv = 1.0 / np.sqrt(d)
+    idx = np.asarray(idx)
+    users = np.nonzero((idx == leaf).any(axis=1))[0].astype(np.int64)
+    dK = np.zeros((C, d))
+    dV = np.zeros((C, d))
+    lo, hi = leaf * C, min((leaf + 1) * C, N)
+    if users.size == 0 or lo >= N:
+        return dK, dV
+    Kl = np.asarray(Kh[lo:hi], np.float64)
+    Vl = np.asarray(Vh[lo:hi], np.float64)
+    keys = np.arange(lo, hi)
+    for h in range(G):
+        q = np.asarray(Qg[h][users], np.float64)
+        do = np.asarray(dOg[h][users], np.float64)
+        o, lse = attn_rows(q, users, Kh, Vh, idx[users], C=C, causal=causal, N=N, want_lse=True)
+        s = q @ Kl.T * inv
+        p = np.exp(s - lse[:, None])
+        if causal:
+            p = np.where(keys[None, :] <= users[:, None], p, 0.0)
+        ds = p * (do @ Vl.T - np.sum(do * o, axis=1)[:, None])
+        dV[:hi - lo] += p.T @ do
+        dK[:hi - lo] += ds.T @ q * inv
+    return dK, dV

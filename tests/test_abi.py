@@ -204,3 +204,46 @@ def test_cache_grow_validates_before_launch(lib):
     assert call(old, new, [P[0], P[1], P[2], ctypes.c_void_p(8 + 4096 * 9), P[4], P[5]]) == -4
     empty = pisa.make_cfg(B=2, Hq=2, Hkv=2, N=0, d=128, C=64, K=8)
     assert call(empty, new, P) == 0
+
+
+def test_forward_host_validates_before_any_copy(lib):
+    # every check of the device step runs before the first host-to-device copy:
+    # a bad argument comes back as its own status (not as a failed copy)
+    cfg = pisa.make_cfg(B=1, Hq=2, Hkv=2, N=1000, d=128, C=64, K=8)
+    need = pisa.pisa_workspace_bytes(cfg)
+    H = [ctypes.c_void_p(1 << 20)] * 5                       # Q, K, V, idx, O on the host
+    D = [ctypes.c_void_p(4096 * (i + 1)) for i in range(6)]  # Q, K, V, pyr, idx, O on the device
+    ws = ctypes.c_void_p(1 << 24)
+
+    def call(dev, w=ws, n=need, host=H):
+        return lib.pisa_forward_host(ctypes.byref(cfg), *host, *dev, w, n, None)
+
+    assert call([D[0], D[1], D[2], None, D[4], D[5]]) == -1                     # no pyramid
+    assert call([D[0], D[1], D[2], ctypes.c_void_p(4096 * 4 + 16), D[4], D[5]]) == -4  # pyramid 16- not 32-aligned
+    assert call([D[0], D[1], D[2], D[3], None, D[5]]) == -1                     # no idx
+    assert call(D, w=None) == -1                                                 # no workspace
+    assert call(D, n=need - 1) == -1                                             # workspace too small
+    assert call(D, w=ctypes.c_void_p((1 << 24) + 128)) == -4                     # workspace misaligned
+    assert call(D, host=[H[0], None, H[2], H[3], H[4]]) == -1                   # no host K
+
+
+def test_cache_grow_checks_the_pyramids_before_the_cache_copies(lib):
+    old = pisa.make_cfg(B=2, Hq=2, Hkv=2, N=2048, d=128, C=64, K=8)
+    new = pisa.make_cfg(B=2, Hq=2, Hkv=2, N=4096, d=128, C=64, K=8)
+    P = [ctypes.c_void_p(4096 * (i + 1)) for i in range(6)]  # Kc_old, Vc_old, pyr_old, Kc_new, Vc_new, pyr_new
+
+    def call(p):
+        return lib.pisa_cache_grow(ctypes.byref(old), p[0], p[1], p[2], ctypes.byref(new), p[3], p[4], p[5], None)
+
+    assert call([P[0], P[1], None, P[3], P[4], P[5]]) == -1                     # no old pyramid
+    assert call([P[0], P[1], P[2], P[3], P[4], P[2]]) == -1                     # pyramid grown in place
+    assert call([P[0], P[1], P[2], P[3], P[4], ctypes.c_void_p(8 + 4096 * 6)]) == -4
+
+
+def test_select_noalloc_status_validates(lib):
+    big = pisa.make_cfg(B=1, Hq=8, Hkv=8, N=262144, d=128, C=64, K=16)
+    assert lib.pisa_select_noalloc_status(ctypes.byref(big), None) == -6
+    bad = pisa.make_cfg(B=1, Hq=2, Hkv=2, N=1000, d=128, C=32, K=8)
+    assert lib.pisa_select_noalloc_status(ctypes.byref(bad), None) == -2
+    empty = pisa.make_cfg(B=1, Hq=2, Hkv=2, N=0, d=128, C=64, K=8)
+    assert lib.pisa_select_noalloc_status(ctypes.byref(empty), None) == 0

@@ -175,8 +175,12 @@ def test_block_major_backward_full_size_sampled():
     idx_h = idx.cpu().numpy()
     M1 = (w.N + w.C - 1) // w.C
     rng = np.random.default_rng(5)
-    rows = sorted(set(rng.choice(w.N, size=14, replace=False).tolist()) | {0, w.N - 1})
-    leaves = [37, M1 // 2, M1 - 1]
+    # rows: the first leaf's edges (C - 1, C, 2C) beside random ones; leaves:
+    # the first (forced for every position: its bucket spans thousands of
+    # tiles and many CTAs), the second, both sides of a scan-block boundary of
+    # the bucket counts (1024 buckets), the middle and the last
+    rows = sorted(set(rng.choice(w.N, size=14, replace=False).tolist()) | {0, w.C - 1, w.C, 2 * w.C, w.N - 1})
+    leaves = [0, 1, 37, 1023, 1024, M1 // 2, M1 - 1]
     worst = 0.0
     for h in (0, 5):
         rQ, rK, rV = oracle.attn_backward_sampled(

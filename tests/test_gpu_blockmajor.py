@@ -1,6 +1,8 @@
 """GPU parity of the block-major tensor-core path (pisa_forward_ws,
 pisa_select_ws, pisa_sparse_attn_ws) against the oracle, and its agreement
 with the per-query path."""
+import ctypes
+
 import numpy as np
 import pytest
 import torch
@@ -58,13 +60,32 @@ def test_blockmajor_named_workload_full_size(name):
     _report("ws:" + name, stats)
     t = torch.arange(w.N, device=idx.device)
     assert bool((idx.max(-1).values == t // w.C).all())
-    # agreement with the per-query path on every row (near-ties aside)
+    # every row: the per-query path is an independent GPU implementation of
+    # the same walk; each row where the two disagree goes to the oracle, and
+    # the tensor-core row must equal the oracle's unless the oracle's margin
+    # is inside the tie band (the per-query row is held to the same rule)
     ref = parity.gpu_prefill(w, Q, K, V, ws=False)
-    same = (ref["idx"] == idx).all(-1).float().mean().item()
-    print(f"[blockmajor] {name}: rows equal to the per-query path {same:.5f}")
-    assert same > 0.98
-    dO = (ref["O"].float() - res["O"].float()).abs().max().item()
-    assert dO <= 2 * parity.O_TOL["bf16"] or same < 1.0
+    differ = (ref["idx"] != idx).any(-1)  # [B, Hkv, N]
+    n_diff = int(differ.sum())
+    print(f"[blockmajor] {name}: rows differing from the per-query path: {n_diff} of {differ.numel()}")
+    dstats = []
+    for b in range(w.B):
+        for h in range(w.Hkv):
+            rows = torch.nonzero(differ[b, h]).flatten().cpu().tolist()
+            if rows:
+                dstats.append(parity.check_head(w, Q, K, V, res, b, h, rows))
+                parity.check_head(w, Q, K, V, ref, b, h, rows)
+    if dstats:
+        ex = sum(s["exempt"] for s in dstats)
+        print(f"[blockmajor] {name}: differing rows checked against the oracle: {n_diff}, "
+              f"inside the tie band {ex}, tensor-core row equal to the oracle's there "
+              f"{sum(s['exempt_equal'] for s in dstats)}, max|dO| {max(s['o_err'] for s in dstats):.3g}")
+    agree = ~differ
+    if bool(agree.any()):
+        G = w.Hq // w.Hkv
+        rows_ok = agree.repeat_interleave(G, dim=1)
+        dO = (ref["O"].float() - res["O"].float()).abs().amax(-1)[rows_ok].max().item()
+        assert dO <= 2 * parity.O_TOL["bf16"], dO
 
 
 @pytest.mark.parametrize("name", ["bm_ragged", "bm_gqa4", "bm_noncausal"])
@@ -127,3 +148,27 @@ def test_forward_host_equals_forward_ws():
     # the attention tiles add fp32 partial outputs in an order that varies from
     # run to run, so O agrees to rounding, not bit for bit
     assert float((Oh.float() - res["O"].float().cpu()).abs().max()) <= parity.O_TOL[w.dtype]
+
+
+def test_failed_forward_host_writes_nothing():
+    # a call that fails validation enqueues no copy: the device buffers keep a sentinel
+    w = SMALL["bm_ragged"]
+    Q, K, V, _ = make_inputs(w)
+    dev = torch.device("cuda", 0)
+    cfg = pisa.make_cfg(B=w.B, Hq=w.Hq, Hkv=w.Hkv, N=w.N, d=w.d, C=w.C, K=w.K)
+    Qd, Kd, Vd = (torch.full(x.shape, 3.0, dtype=x.dtype, device=dev) for x in (Q, K, V))
+    pyr, idx, O = pisa.alloc_outputs(cfg, dev, Q.dtype)
+    work = pisa.alloc_workspace(cfg, dev)
+    Ih = torch.zeros(idx.shape, dtype=idx.dtype).pin_memory()
+    Oh = torch.zeros(O.shape, dtype=O.dtype).pin_memory()
+    lib = pisa.load()
+    p = lambda t: ctypes.c_void_p(t.data_ptr())  # noqa: E731
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    for bad_pyr, bad_bytes in ((None, work.numel()), (p(pyr), work.numel() - 256)):
+        st = lib.pisa_forward_host(ctypes.byref(cfg), p(Q.pin_memory()), p(K.pin_memory()), p(V.pin_memory()),
+                                   p(Ih), p(Oh), p(Qd), p(Kd), p(Vd), bad_pyr, p(idx), p(O), p(work), bad_bytes,
+                                   stream)
+        torch.cuda.synchronize()
+        assert st == -1
+        for x in (Qd, Kd, Vd):
+            assert bool((x == 3.0).all()), "a failed call copied into the device buffers"

@@ -250,3 +250,23 @@ def test_decode_cache_grows_geometrically_inside_the_library():
             assert not cache.Kc[s, :, n + 1:].any()
         pos += 1
     assert caps == [2048, 2048, 4096, 4096, 4096]
+
+
+def test_failed_cache_grow_writes_nothing():
+    # a null or aliased pyramid is rejected before the K and V copies are launched
+    import ctypes
+    dev = torch.device("cuda", 0)
+    old = pisa.make_cfg(B=2, Hq=2, Hkv=2, N=1024, d=128, C=64, K=8)
+    new = pisa.make_cfg(B=2, Hq=2, Hkv=2, N=2048, d=128, C=64, K=8)
+    Kc, Vc = (torch.randn(2, 2, 1024, 128, device=dev).to(torch.bfloat16) for _ in range(2))
+    Kn, Vn = (torch.full((2, 2, 2048, 128), 3.0, dtype=torch.bfloat16, device=dev) for _ in range(2))
+    po = torch.zeros((2, 2, pisa.pisa_pyramid_rows(old), 128), dtype=torch.float32, device=dev)
+    p = lambda t: ctypes.c_void_p(t.data_ptr())  # noqa: E731
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    lib = pisa.load()
+    for pyr_old, pyr_new in ((None, p(po)), (p(po), p(po))):
+        st = lib.pisa_cache_grow(ctypes.byref(old), p(Kc), p(Vc), pyr_old, ctypes.byref(new), p(Kn), p(Vn),
+                                 pyr_new, stream)
+        torch.cuda.synchronize()
+        assert st == -1
+        assert bool((Kn == 3.0).all()) and bool((Vn == 3.0).all()), "a failed call wrote the new caches"

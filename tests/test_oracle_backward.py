@@ -117,3 +117,27 @@ def test_sampled_backward_equals_the_full_backward(G, causal):
         np.testing.assert_allclose(sK[li, :n], fK[leaf * C:leaf * C + n], rtol=1e-12, atol=1e-12)
         np.testing.assert_allclose(sV[li, :n], fV[leaf * C:leaf * C + n], rtol=1e-12, atol=1e-12)
         assert not sK[li, n:].any() and not sV[li, n:].any()
+
+
+@pytest.mark.parametrize("G,causal", [(1, True), (3, True), (2, False)])
+def test_leaf_backward_equals_the_full_backward(G, causal):
+    # the batched per-leaf form (normaliser and output from attn_rows, every
+    # user of the leaf at once) against the rows of the pinned full backward,
+    # on every leaf, the ragged last one included
+    N, C, d, K = 300, 16, 8, 5
+    rng = np.random.default_rng(41 + G)
+    Q, Kh, Vh, dO = _rand((G, N, d), 42), _rand((N, d), 43), _rand((N, d), 44), _rand((G, N, d), 45)
+    M1 = (N + C - 1) // C
+    idx = np.full((N, K), -1, np.int64)
+    for t in range(N):
+        c = t // C
+        pick = {0, c} | set(rng.choice(max(c, 1), size=min(K - 2, max(c, 1)), replace=False).tolist())
+        pick = sorted(x for x in pick if x <= (c if causal else M1 - 1))[:K]
+        idx[t, :len(pick)] = pick
+    _, fK, fV = oracle.attn_backward_rows(Q, Kh, Vh, idx, dO, C=C, causal=causal)
+    for leaf in range(M1):
+        lK, lV = oracle.attn_backward_leaf(Q, Kh, Vh, idx, dO, leaf, C=C, causal=causal)
+        n = min(C, N - leaf * C)
+        np.testing.assert_allclose(lK[:n], fK[leaf * C:leaf * C + n], rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(lV[:n], fV[leaf * C:leaf * C + n], rtol=1e-10, atol=1e-12)
+        assert not lK[n:].any() and not lV[n:].any()
