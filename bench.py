@@ -160,7 +160,9 @@ _CS = "hierarchical_block_sparse_b200/csrc/"
 _BMF = _CS + "blockmajor.cu"
 _TILE = [(_BMF, "tile plumbing"), _CS + "tc.cuh", _CS + "pisa_internal.h"]
 KERNEL_SOURCES = {
-    "stage1": [(_BMF, "stage 1"), _CS + "pisa_stage1.cuh", _CS + "pisa_walk.cuh", _CS + "pisa_device.cuh"],
+    "stage1": [_CS + "walk_tc.cu", _CS + "tc.cuh", _CS + "pisa_walk.cuh", _CS + "pisa_device.cuh"],
+    "stage1_per_query": [(_BMF, "stage 1"), _CS + "pisa_stage1.cuh", _CS + "pisa_walk.cuh", _CS + "pisa_device.cuh"],
+    "bsa_tc": [_CS + "bsa_tc.cu", _CS + "tc.cuh", _CS + "pisa_walk.cuh", _CS + "pisa_device.cuh"],
     "leaf_scores": [(_BMF, "stage 2: leaf LSEs")] + _TILE,
     "topk": [(_BMF, "final Top-K"), _CS + "pisa_walk.cuh", _CS + "pisa_device.cuh"],
     "attn_tiles": [(_BMF, "attention tiles")] + _TILE,
@@ -361,6 +363,11 @@ def dominant_roofline(w, phase_ms, alg, pk, fma_peak, fma_note, tc_peak):
         roof = {"kernel": "leaf_score_kernel", "bound": "tensor", "achieved": alg["leaf_flops"] / t_dom / 1e12,
                 "peak": tc_peak, "unit": "TFLOP/s", "algorithmic_per_launch": alg["leaf_flops"],
                 "peak_note": tc_note}
+    elif dom == "stage1" and walk_on_tensor_cores(w):
+        roof = {"kernel": "walk_tc_kernel", "bound": "tensor", "achieved": alg["internal_flops"] / t_dom / 1e12,
+                "peak": tc_peak, "unit": "TFLOP/s", "algorithmic_per_launch": alg["internal_flops"],
+                "peak_note": tc_note + "; achieved counts the walk's own child dots (the union's extra dots and "
+                                       "the second bf16 part are not counted)"}
     elif dom == "stage1":
         roof = {"kernel": "stage1_kernel", "bound": "alu", "achieved": alg["internal_flops"] / t_dom / 1e12,
                 "peak": fma_peak, "unit": "TFLOP/s", "algorithmic_per_launch": alg["internal_flops"],
@@ -375,24 +382,43 @@ def dominant_roofline(w, phase_ms, alg, pk, fma_peak, fma_note, tc_peak):
     return roof
 
 
+def walk_on_tensor_cores(w) -> bool:
+    """The block-major selection walks on the tensor cores while the level
+    above the finest ranked one has at most 8192 nodes (N <= 2M at C = 64)."""
+    M1 = -(-w.N // w.C)
+    M3 = -(-(-(-M1 // 2)) // 2)
+    return M1 <= 2 or M3 <= 8192
+
+
 SELECTION_PHASES = ("pyramid", "stage1", "group_candidates", "leaf_scores", "topk")
 
 
-def time_bsa(cfg, Qd, Kd, pyr, idx, stream):
-    """Flat BSA selection (pyramid + Eq.1 scan over every eligible leaf), ms."""
+def time_bsa(cfg, Qd, Kd, pyr, idx, stream, work=None, reps: int = 3):
+    """Flat BSA selection (pyramid + Eq.1 over every eligible leaf), ms: on the
+    tensor cores (pisa_bsa_select_ws) when a workspace is given, else the
+    per-query CUDA-core scan (pisa_bsa_select)."""
     import torch
     from hierarchical_block_sparse_b200 import pisa
     bidx = torch.empty_like(idx)
-    pisa.pisa_build_pyramid(cfg, Kd, pyr)
-    pisa.pisa_bsa_select(cfg, Qd, pyr, bidx)
+
+    def run():
+        pisa.pisa_build_pyramid(cfg, Kd, pyr)
+        if work is None:
+            pisa.pisa_bsa_select(cfg, Qd, pyr, bidx)
+        else:
+            pisa.pisa_bsa_select_ws(cfg, Qd, pyr, bidx, work)
+
+    run()
     torch.cuda.synchronize()
     b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     b0.record(stream)
-    pisa.pisa_build_pyramid(cfg, Kd, pyr)
-    pisa.pisa_bsa_select(cfg, Qd, pyr, bidx)
+    for _ in range(reps):
+        run()
     b1.record(stream)
     torch.cuda.synchronize()
-    return b0.elapsed_time(b1)
+    if work is not None and pisa.pisa_workspace_status(cfg, work) != 0:
+        raise RuntimeError("a tensor-core BSA tile timed out")
+    return b0.elapsed_time(b1) / reps
 
 
 def prefill_config_line(w, dev, stream, steps, warmup, pk, fma_peak, fma_note, tc_peak, bsa=True):
@@ -438,7 +464,8 @@ def prefill_config_line(w, dev, stream, steps, warmup, pk, fma_peak, fma_note, t
            "work": {"internal_tflop": alg["internal_flops"] / 1e12, "leaf_tflop": alg["leaf_flops"] / 1e12,
                     "attn_tflop": alg["attn_flops"] / 1e12}}
     if bsa:
-        out["bsa_selection_ms"] = time_bsa(cfg, Qd, Kd, pyr, idx, stream)
+        out["bsa_selection_ms"] = time_bsa(cfg, Qd, Kd, pyr, idx, stream, work)
+        out["bsa_cuda_core_ms"] = time_bsa(cfg, Qd, Kd, pyr, idx, stream, reps=1)
         out["pisa_vs_bsa_selection_speedup"] = out["bsa_selection_ms"] / sel
     del Qd, Kd, Vd, pyr, idx, O, work
     torch.cuda.empty_cache()
@@ -519,9 +546,10 @@ def main():
     stream = torch.cuda.current_stream()
     nph = len(pisa.PHASES)
     pool_launches = 2 if pisa.pisa_num_levels(cfg) >= 6 else 1
-    # our kernels per step: pyramid, stage 1, 3 grouping kernels, leaf scores,
-    # Top-K, 3 grouping kernels, forced tiles, attention tiles, output conversion
-    launches_per_step = pool_launches + 1 + 3 + 1 + 1 + 3 + 1 + 1 + 1
+    # our kernels per step: pyramid, stage 1 (pyramid split + tile walk, or the
+    # one-warp walk), 3 grouping kernels, leaf scores, Top-K, 3 grouping
+    # kernels, forced tiles, attention tiles, output conversion
+    launches_per_step = pool_launches + (2 if walk_on_tensor_cores(w) else 1) + 3 + 1 + 1 + 3 + 1 + 1 + 1
 
     def step(ev=None):
         if ev is None:
@@ -659,8 +687,9 @@ def main():
 
     # ---- flat BSA selection, the quadratic comparison ----
     if not args.no_bsa:
-        out["bsa_selection_ms"] = time_bsa(cfg, Qd, Kd, pyr, idx, stream)
-        out["bsa_kernel"] = "per-query CUDA-core flat scan (bsa_kernel)"
+        out["bsa_selection_ms"] = time_bsa(cfg, Qd, Kd, pyr, idx, stream, work)
+        out["bsa_kernel"] = "tensor-core flat Eq.(1) contraction with a streaming Top-K (bsa_tc_kernel)"
+        out["bsa_cuda_core_ms"] = time_bsa(cfg, Qd, Kd, pyr, idx, stream, reps=1)
         out["pisa_vs_bsa_selection_speedup"] = out["bsa_selection_ms"] / sel_total
 
     # ---- the same step ranking by the PISA-1 / PISA-2 scores (Eq.8-9 ablations) ----

@@ -260,6 +260,25 @@ int pisa_bsa_select(const pisa_cfg* cfg, const void* Q, const float* pyr, int32_
     return cuda_status(launch_bsa(cfg->dtype, cfg->d, Q, pyr, idx, select_params(cfg, g), (cudaStream_t)stream));
 }
 
+int pisa_bsa_select_ws(const pisa_cfg* cfg, const void* Q, const float* pyr, int32_t* idx, void* workspace,
+                       size_t workspace_bytes, void* stream) {
+    int s = check_bm(cfg);
+    if (s) return s;
+    if (cfg->N == 0) return PISA_OK;
+    if (!Q || !pyr || !idx) return PISA_E_INVALID;
+    if (!aligned16(Q) || !aligned16(pyr) || !aligned16(idx)) return PISA_E_ALIGNMENT;
+    s = check_ws(cfg, workspace, workspace_bytes);
+    if (s) return s;
+    const BmLayout L = blockmajor_layout(bm_shape(cfg));
+    uint8_t* ws = (uint8_t*)workspace;
+    cudaStream_t st = (cudaStream_t)stream;
+    if (cudaMemsetAsync(ws + L.misc, 0, 256, st) != cudaSuccess) return PISA_E_CUDA;
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    return cuda_status(launch_bsa_tc(Q, pyr, ws + L.phl, idx, (int*)(ws + L.misc) + 1, select_params_of(cfg),
+                                     cfg->Hq / cfg->Hkv, sms, st));
+}
+
 int64_t pisa_workspace_bytes(const pisa_cfg* cfg) {
     int s = check_bm(cfg);
     if (s) return s;

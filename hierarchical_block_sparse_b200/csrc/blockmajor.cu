@@ -63,16 +63,24 @@ constexpr int kORowStride = kD * 4 + 16;  // staged fp32 output row: 16-byte pad
 // Grid: x = blocks of 8 query positions, y = b * Hkv + kvh. Besides the
 // candidates, each lane adds its non-forced candidate to the leaf's bucket
 // count (the grouping of stage 2).
-template <int G, class W>
+// RESUME: the tensor-core tile walk (walk_tc.cu) has done the coarse levels;
+// resume[unit] is 0 for a position it finished, else (resume level << 8 |
+// count) with the kept nodes in cand_out's row, which this kernel reads
+// before it overwrites the row with the level-1 candidates.
+template <int G, class W, bool RESUME = false>
 __global__ void __launch_bounds__(256, PISA_STAGE1_MINBLOCKS) stage1_kernel(const __nv_bfloat16* __restrict__ Q,
                                                      const float* __restrict__ pyr, int32_t* __restrict__ cand_out,
                                                      int32_t* __restrict__ counts, int32_t* __restrict__ slots,
-                                                     int64_t M1, int* __restrict__ err, SelectParams p) {
+                                                     int64_t M1, int* __restrict__ err, SelectParams p,
+                                                     const int32_t* __restrict__ resume = nullptr) {
     const int lane = threadIdx.x & 31;
     const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     if (t >= p.N) return;
     const int64_t bh = blockIdx.y;
     const int64_t unit = bh * p.N + t;
+    if constexpr (RESUME) {
+        if (resume[unit] == 0) return;  // the tile walk finished this position
+    }
     const int64_t b = bh / p.Hkv;
     const int kvh = (int)(bh - b * p.Hkv);
     W w;
@@ -87,7 +95,21 @@ __global__ void __launch_bounds__(256, PISA_STAGE1_MINBLOCKS) stage1_kernel(cons
     const float* P = pyr + bh * p.geom.rows * kD;
     const Forced F(t, p.C, p.causal, p.forced_mask);
     int cand = lane == 0 ? 0 : -1;
-    for (int l = p.geom.L; l >= 2; --l) {
+    int lstart = p.geom.L;
+    if constexpr (RESUME) {
+        const int meta = resume[unit];
+        const int nk = meta & 0xff;
+        lstart = meta >> 8;
+        if (lstart < 1 || lstart >= p.geom.L || nk > p.K) {  // self-check: never expected
+            if (lane == 0 && err) atomicCAS(err, 0, 18);
+            lstart = 1;
+        }
+        const int par = lane < nk ? cand_out[unit * kSlots + lane] : -1;
+        const int pp = __shfl_sync(kFull, par, lane >> 1);
+        cand = lane < 2 * nk && pp >= 0 ? 2 * pp + (lane & 1) : -1;
+        __syncwarp();
+    }
+    for (int l = lstart; l >= 2; --l) {
         const LevelState s = level_state(cand, l, p.C, p.N, t, p.causal, F);
         int parent;
         if (s.n <= p.K) {
@@ -1654,6 +1676,8 @@ BmLayout blockmajor_layout(const BmShape& s) {
     L.entries = take(units * kSlots * 4);
     L.tiles = take(max_tiles * 16);
     L.bsum = take(((nb + kScanBlock - 1) / kScanBlock) * 16);
+    L.phl = take(walk_tc_pyramid_bytes((int64_t)s.B * s.Hkv, s.rows));  // bf16 high / low parts of the pyramid
+    L.resume = take(units * 4);  // where the one-warp walk resumes after the tile walk
     L.misc = take(256);  // [0] tile count, [1] error word
     L.oacc = take((int64_t)s.B * s.Hq * s.N * kD * 4);
     L.total = off;
@@ -1764,14 +1788,27 @@ static cudaError_t select_bm_t(const void* Q, const void* K, const float* pyr, i
     e = zero_counts(s, ws, L, st);
     if (e != cudaSuccess) return e;
     using W = typename std::conditional<(G <= 2), Walk4S<(G <= 2 ? G : 1)>, Walk<__nv_bfloat16, kD, G>>::type;
+    if (walk_tc_fits(sp)) {
+        // the coarse levels in tiles of consecutive positions on the tensor cores,
+        // the fine ones (little reuse across positions) one warp per position
+        e = launch_walk_tc(Q, pyr, ws + L.phl, cand, (int32_t*)(ws + L.resume), (int32_t*)(ws + L.counts),
+                           (int32_t*)(ws + L.slots), (int*)(ws + L.misc) + 1, sp, G, sm_count(), st);
+        if (e != cudaSuccess) return e;
+        stage1_kernel<G, W, true><<<unit_grid(s), 256, 0, st>>>((const __nv_bfloat16*)Q, pyr, cand,
+                                                                (int32_t*)(ws + L.counts), (int32_t*)(ws + L.slots),
+                                                                s.M1, (int*)(ws + L.misc) + 1, sp,
+                                                                (const int32_t*)(ws + L.resume));
+    } else {
 #if PISA_STAGE1_CARVEOUT >= 0
-    // the walk lives on L1 hits of pyramid rows and needs little shared memory
-    e = cudaFuncSetAttribute(stage1_kernel<G, W>, cudaFuncAttributePreferredSharedMemoryCarveout,
-                             PISA_STAGE1_CARVEOUT);
-    if (e != cudaSuccess) return e;
+        // the walk lives on L1 hits of pyramid rows and needs little shared memory
+        e = cudaFuncSetAttribute(stage1_kernel<G, W>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 PISA_STAGE1_CARVEOUT);
+        if (e != cudaSuccess) return e;
 #endif
-    stage1_kernel<G, W><<<unit_grid(s), 256, 0, st>>>((const __nv_bfloat16*)Q, pyr, cand, (int32_t*)(ws + L.counts),
-                                                      (int32_t*)(ws + L.slots), s.M1, (int*)(ws + L.misc) + 1, sp);
+        stage1_kernel<G, W><<<unit_grid(s), 256, 0, st>>>((const __nv_bfloat16*)Q, pyr, cand,
+                                                          (int32_t*)(ws + L.counts), (int32_t*)(ws + L.slots), s.M1,
+                                                          (int*)(ws + L.misc) + 1, sp);
+    }
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     mark(ev, 2, st);

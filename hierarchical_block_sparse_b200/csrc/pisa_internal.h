@@ -45,7 +45,7 @@ struct BmShape {
     int variant;   // enum pisa_score (the ranking scores need their own region unless 0)
 };
 struct BmLayout {  // byte offsets of the workspace regions
-    size_t cand, lse, vscore, z2, counts, slots, offsets, entries, tiles, bsum, misc, oacc, total;
+    size_t cand, lse, vscore, z2, counts, slots, offsets, entries, tiles, bsum, phl, resume, misc, oacc, total;
 };
 struct PhaseEvents {  // optional caller events recorded at phase boundaries
     void* const* events;
@@ -84,6 +84,25 @@ inline BmShape bm_shape_of(const pisa_cfg* c) {
     s.variant = c->score_variant;
     return s;
 }
+
+// Stage 1 on the tensor cores (walk_tc.cu): tiles of consecutive positions
+// walk the coarse levels, scoring the union of their kept parents'
+// grandchildren. A tile that finishes every level writes the level-1
+// candidates and bucket counts itself (resume[unit] = 0); otherwise each
+// position's kept nodes go to the candidate region (slots 0..15) and
+// resume[unit] = resume level << 8 | count, for the one-warp walk to finish.
+// pyr_hl holds the bf16 high and low parts of the pyramid (walk_tc_pyramid_bytes).
+bool walk_tc_fits(const SelectParams& sp);
+size_t walk_tc_pyramid_bytes(int64_t units_bh, int64_t rows);
+cudaError_t launch_walk_tc(const void* Q, const float* pyr, void* pyr_hl, int32_t* cand, int32_t* resume,
+                           int32_t* counts, int32_t* slots, int* err, const SelectParams& sp, int G, int sms,
+                           cudaStream_t st);
+
+// the bf16 high / low parts of the fp32 pyramid (elems floats -> 2 x elems bf16 at pyr_hl)
+cudaError_t launch_split_pyramid(const float* pyr, void* pyr_hl, int64_t elems, int sms, cudaStream_t st);
+// flat Eq.(1) selection on the tensor cores (bsa_tc.cu); pyr_hl as for the tile walk
+cudaError_t launch_bsa_tc(const void* Q, const float* pyr, void* pyr_hl, int32_t* idx, int* err,
+                          const SelectParams& sp, int G, int sms, cudaStream_t st);
 
 cudaError_t launch_pool(int dtype, int d, const void* K, float* pyr, const PoolParams& p, cudaStream_t st);
 cudaError_t launch_attn_bwd(int dtype, int d, const void* Q, const void* K, const void* V, const int32_t* idx,

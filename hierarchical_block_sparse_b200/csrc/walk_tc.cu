@@ -1,0 +1,601 @@
+// walk_tc.cu -- the internal levels of the pyramid walk (Stage 1 of close
+// reading §05 Algorithm 1; Eq.(5)-(7), (11); §5.3 forced and causal rules)
+// for a tile of consecutive query positions on the tensor cores.
+//
+// A CTA takes 128 MMA rows: 128/G consecutive positions of one (b, kv-head)
+// times the G query heads of the group. Every position walks the pyramid by
+// the same rules as the one-warp-per-query walk (pisa_stage1.cuh): at each
+// level its candidates are the children of the nodes it kept one level up;
+// when it has more than K of them it keeps the forced ones and the best by
+// the LSE over each candidate's two children (summed over the G heads), ties
+// to the lower index. Consecutive positions keep mostly the same nodes, so
+// the dot products are taken for the union of the tile's kept parents: each
+// kept parent p at level l+1 contributes its four grandchildren (rows 4p..4p+3
+// of level l-1, the children of its candidates 2p and 2p+1), in chunks of 32
+// parents (128 columns). S = Q_tile x rows^T runs on tcgen05 into TMEM; the
+// fp32 summaries enter as two bf16 parts (hi = bf16(x), lo = bf16(x - hi)),
+// and q is bf16 already, so both products are exact and S carries the
+// summaries to about 2^-16 of their size (about 1e-5 on a logit). Each row
+// then reads the four columns of each of its own kept parents and writes its
+// candidates' pair scores to shared memory; one warp per position ranks them
+// with the walk's own keep rule. After level 2 the level-1 candidates are
+// written exactly as the one-warp walk writes them (slots, sibling-pair
+// bucket counts), so the rest of the block-major selection is unchanged.
+//
+// Per chunk, the gather of the next chunk's rows (cp.async) runs while the
+// current chunk's MMAs and row pick-up run: two B buffers and two 128-column
+// TMEM accumulators. Warps 0-3 pick up column groups 0-1 of a chunk, warps
+// 4-7 groups 2-3 (warp w reads TMEM lanes 32 (w % 4) ..).
+#include <cmath>
+
+#include "pisa_internal.h"
+#include "pisa_walk.cuh"
+#include "tc.cuh"
+
+namespace pisa {
+namespace {
+
+constexpr int kTwThreads = 256;
+constexpr int kTwPar = 32;            // union parents per chunk
+constexpr int kTwMaxWords = 256;      // bitmap words: parent levels of up to 8192 nodes
+constexpr int kTwMaxUnion = 2048;     // 128 positions x 16 kept nodes
+constexpr int kTwHandoff = 4 * kTwPar; // a level whose union needs more chunks goes to the one-warp walk
+constexpr int kD = 128;
+constexpr int kSlots = 32;
+constexpr int kPairs = 16;
+constexpr int kBig = 0x7fffffff;
+
+constexpr int kRow = 17;  // padded row of the per-position lists (one thread per position reads its own row)
+
+struct TwSmem {
+    uint8_t q[32768];        // A: 128 rows x 128 bf16, K-major canonical layout
+    uint8_t b[2][2][32768];  // B[buffer][hi, lo]: 128 rows x 128 bf16
+    float score[128 * kSlots + 128];  // position p, slot c, head h at p * (32 G + 1) + c * G + h
+    int32_t kept[128][kRow];  // kept nodes of the level above, ascending
+    int32_t keptu[128][kRow]; // their index in the union
+    int32_t uni[kTwMaxUnion];
+    uint32_t bits[kTwMaxWords];
+    int32_t pre[kTwMaxWords];
+    int32_t nkept[128];
+    int32_t need[128];
+    int32_t scan[8];
+    uint64_t mbar[2];
+    uint32_t tmem_base;
+};
+
+// exclusive scan of one int per thread over the 256 threads; returns the total
+__device__ __forceinline__ int block_exscan(int& v, int32_t* scan) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(kFull, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) scan[warp] = x;
+    __syncthreads();
+    int before = 0, total = 0;
+#pragma unroll
+    for (int w = 0; w < kTwThreads / 32; ++w) {
+        const int s = scan[w];
+        before += w < warp ? s : 0;
+        total += s;
+    }
+    v = before + x - v;
+    __syncthreads();
+    return total;
+}
+
+__device__ __forceinline__ uint32_t idesc_n(int n) {  // kind::f16, bf16 x bf16 -> fp32, both K-major, M = 128
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+}
+
+// One position's candidates at level l are held by two adjacent lanes: lane
+// half h owns slots 16 h .. 16 h + 15, the children of its kept nodes 8 h ..
+// 8 h + 7 one level up (the root alone in slot 0 at l = L), so the slots
+// ascend with the node index. Bit i of v: slot 16 h + i exists and is
+// eligible (causal: its first key is not after t); of f: it is on a forced
+// path (close reading §5.3).
+struct HalfCands {
+    int node[16];
+    uint32_t v, f;
+};
+
+__device__ __forceinline__ void half_cands(const TwSmem& S, int pos, int l, int L, int64_t t, const SelectParams& p,
+                                           int h, bool live, HalfCands& hc) {
+    const Forced F(t, p.C, p.causal, p.forced_mask);
+    const int nk = (!live || l == L) ? 0 : S.nkept[pos];
+    const int64_t span = (int64_t)p.C << (l - 1);
+    hc.v = hc.f = 0u;
+#pragma unroll
+    for (int jj = 0; jj < 8; ++jj) {
+        const int j = 8 * h + jj;
+        const int par = !live ? -1 : l == L ? (j == 0 ? 0 : -1) : (j < nk ? S.kept[pos][j] : -1);
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int i = 2 * jj + e;
+            const int node = l == L ? (par == 0 && e == 0 ? 0 : -1) : (par >= 0 ? 2 * par + e : -1);
+            hc.node[i] = node;
+            const int64_t first = (int64_t)node * span;
+            const bool valid = node >= 0 && first < p.N && (!p.causal || first <= t);
+            hc.v |= (valid ? 1u : 0u) << i;
+            hc.f |= (valid && F.has(node, l) ? 1u : 0u) << i;
+        }
+    }
+}
+
+// the 32-slot mask of a position from its two lanes' 16-slot halves
+__device__ __forceinline__ uint32_t pair_mask(uint32_t m16, int h) {
+    const uint32_t o = __shfl_xor_sync(kFull, m16, 1);
+    return h == 0 ? (m16 | (o << 16)) : (o | (m16 << 16));
+}
+
+// the kept candidates (bit c of `keep`) in slot order, i.e. ascending node
+// order; each lane writes its own half
+__device__ __forceinline__ void write_kept(TwSmem& S, int pos, const HalfCands& hc, uint32_t keep, int h) {
+    int n = h == 0 ? 0 : __popc(keep & 0xffffu);
+    const uint32_t mine = (keep >> (16 * h)) & 0xffffu;
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+        if ((mine >> i) & 1u) S.kept[pos][n++] = hc.node[i];
+    if (h == 0) S.nkept[pos] = __popc(keep);
+}
+
+// the lowest k set bits of m
+__device__ __forceinline__ uint32_t lowest_bits(uint32_t m, int k) {
+    uint32_t r = 0u;
+    for (int i = 0; i < k && m; ++i) {
+        const uint32_t b = m & (0u - m);
+        r |= b;
+        m ^= b;
+    }
+    return r;
+}
+
+// order-preserving map of a float onto uint32 (larger float -> larger integer)
+__device__ __forceinline__ uint32_t ordered(float x) {
+    const uint32_t u = __float_as_uint(x);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ void cex(uint64_t& x, uint64_t& y, bool desc) {
+    const uint64_t big = x > y ? x : y, small = x > y ? y : x;
+    x = desc ? big : small;
+    y = desc ? small : big;
+}
+
+// The keep rule of a ranked level (close reading §04 4.2; Eq.(6)): forced
+// candidates first, then the best scores, ties to the lower node (= lower
+// slot). Each candidate's key packs (score, 31 - slot) into 64 bits, so the
+// keys are distinct and their order is the rank order. The two lanes of a
+// position sort their 16 keys in opposite directions (a bitonic sequence of
+// 32), exchange once, and lane half 0 ends with the 16 largest, descending;
+// the top K are kept. Returns the 32-slot keep mask on both lanes.
+__device__ __forceinline__ uint32_t rank_keep(const float (&score)[16], const HalfCands& hc, uint32_t vfull,
+                                              uint32_t ffull, int K, int h) {
+    uint64_t a[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const int c = 16 * h + i;
+        const bool v = (vfull >> c) & 1u, f = (ffull >> c) & 1u;
+        const uint32_t hi = !v ? 0u : f ? 0xffffffffu : ordered(score[i]);
+        a[i] = ((uint64_t)hi << 32) | (uint32_t)(kSlots - 1 - c);
+    }
+#pragma unroll
+    for (int k = 2; k <= 16; k <<= 1)
+#pragma unroll
+        for (int j = k >> 1; j > 0; j >>= 1)
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const int m = i ^ j;
+                if (m > i) cex(a[i], a[m], k == 16 ? h == 0 : (i & k) == 0);
+            }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {  // the cross-lane step of the 32-key merge
+        const uint32_t lo = __shfl_xor_sync(kFull, (uint32_t)a[i], 1);
+        const uint32_t hi = __shfl_xor_sync(kFull, (uint32_t)(a[i] >> 32), 1);
+        const uint64_t o = ((uint64_t)hi << 32) | lo;
+        a[i] = h == 0 ? (a[i] > o ? a[i] : o) : (a[i] > o ? o : a[i]);
+    }
+#pragma unroll
+    for (int j = 8; j > 0; j >>= 1)
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const int m = i ^ j;
+            if (m > i) cex(a[i], a[m], true);
+        }
+    uint32_t keep = 0u;
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+        if (i < K) keep |= 1u << (kSlots - 1 - (int)(a[i] & 31u));
+    keep = __shfl_sync(kFull, keep, (threadIdx.x & 31) & ~1);
+    return keep & vfull;
+}
+
+template <int G>
+__global__ void __launch_bounds__(kTwThreads, 1) walk_tc_kernel(
+    const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ pyr_hi,
+    const __nv_bfloat16* __restrict__ pyr_lo, int32_t* __restrict__ cand_out, int32_t* __restrict__ resume,
+    int32_t* __restrict__ counts, int32_t* __restrict__ slots, int tiles_per_head, int* __restrict__ err,
+    SelectParams p) {
+    constexpr int P = 128 / G;  // positions per tile
+    extern __shared__ __align__(1024) uint8_t dsm[];
+    TwSmem& S = *reinterpret_cast<TwSmem*>(dsm);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+    // heaviest tiles (latest positions: the largest unions) first
+    const int64_t nbh = (int64_t)p.B * p.Hkv;
+    const int64_t bh = blockIdx.x % nbh;
+    const int tile = tiles_per_head - 1 - (int)(blockIdx.x / nbh);
+    const int64_t b = bh / p.Hkv;
+    const int kvh = (int)(bh - b * p.Hkv);
+    const int t0 = tile * P;
+    const int L = p.geom.L;
+
+    if (warp == 0) tc::tmem_alloc(&S.tmem_base, 256);
+    if (tid == 0) {
+        tc::mbar_init(&S.mbar[0], 1);
+        tc::mbar_init(&S.mbar[1], 1);
+        tc::fence_mbar_init();
+    }
+    // the tile's query rows (row r = position r / G, head r % G) into the A tile
+    const uint32_t q_smem = tc::smem_u32(S.q);
+    for (int i = tid; i < 128 * 16; i += kTwThreads) {
+        const int r = (i >> 7) * 8 + (i & 7), c = (i >> 3) & 15;  // 8 rows x 16-byte chunk: 128 contiguous bytes
+        const int t = t0 + r / G;
+        const __nv_bfloat16* src = Q + (((b * p.Hq + (int64_t)kvh * G + (r % G)) * p.N) + (t < p.N ? t : 0)) * kD + c * 8;
+        if (t < p.N) tc::cp_async16(q_smem + tc::kmajor128_off(r, c), src);
+        else tc::cp_async_zero16(q_smem + tc::kmajor128_off(r, c), src);
+    }
+    tc::cp_async_commit();
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    const uint32_t tmem = S.tmem_base;
+    uint32_t parity[2] = {0u, 0u};
+    bool ok = true;
+
+    const __nv_bfloat16* Hh = pyr_hi + bh * p.geom.rows * kD;
+    const __nv_bfloat16* Hl = pyr_lo + bh * p.geom.rows * kD;
+
+    // Above the first level where some position of the tile has more than K
+    // eligible nodes, every position keeps every eligible node: its kept list
+    // one level below that is simply all of its eligible nodes there.
+    const int t_hi = min(t0 + P, p.N) - 1;
+    int lstart = L;
+    while (lstart >= 2) {
+        const int64_t span = (int64_t)p.C << (lstart - 1);
+        const int64_t n_elig = p.causal ? min(p.geom.M[lstart], (int64_t)t_hi / span + 1) : p.geom.M[lstart];
+        if (n_elig > p.K) break;
+        --lstart;
+    }
+    if (lstart < L) {  // kept lists at level lstart + 1 (at most K nodes each)
+        const int64_t span = (int64_t)p.C << lstart;
+        for (int i = tid; i < P * 16; i += kTwThreads) {
+            const int pos = i >> 4, j = i & 15;
+            const int64_t t = min(t0 + pos, p.N - 1);
+            const int64_t n_elig = p.causal ? min(p.geom.M[lstart + 1], t / span + 1) : p.geom.M[lstart + 1];
+            if (j < n_elig) S.kept[pos][j] = j;
+            if (j == 0) S.nkept[pos] = (int)n_elig;
+        }
+        __syncthreads();
+    }
+    int lstop = 1;  // the level the one-warp walk resumes at (1: only the leaf candidates are left)
+
+    for (int l = lstart; l >= 2 && ok; --l) {
+        // ---- level state of every position; those that must rank flag their kept parents
+        const int64_t span_par = (int64_t)p.C << l;  // tokens under a node of level l + 1
+        const int t_last = min(t0 + P, p.N) - 1;
+        // kept parents are eligible nodes: under causal masking none starts after the tile's last position
+        const int64_t wnodes = l == L ? 1 : p.causal ? min(p.geom.M[l + 1], (int64_t)t_last / span_par + 1)
+                                                      : p.geom.M[l + 1];
+        const int words = (int)((wnodes + 31) >> 5);
+        for (int i = tid; i < words; i += kTwThreads) S.bits[i] = 0u;
+        __syncthreads();
+        int any = 0;
+        if (warp * 32 < 2 * P) {  // two lanes per position
+            const int pos = tid >> 1, h = tid & 1;
+            const bool live = pos < P && t0 + pos < p.N;
+            const int64_t t = live ? t0 + pos : 0;
+            HalfCands hc;
+            half_cands(S, pos, l, L, t, p, h, live, hc);
+            const uint32_t vfull = pair_mask(hc.v, h), ffull = pair_mask(hc.f, h);
+            const int n = __popc(vfull), nf = __popc(ffull);
+            const bool rank = live && n > p.K && nf < p.K;
+            const int nk = live && l < L ? S.nkept[pos] : 0;
+            __syncwarp();  // both lanes have read the kept nodes they expand
+            if (live && !rank)  // all of them, or the forced ones fill the budget: no scores needed
+                write_kept(S, pos, hc, n <= p.K ? vfull : lowest_bits(ffull, p.K), h);
+            if (rank) {  // flag the parents whose grandchildren are needed
+                for (int j = 8 * h; j < min(nk, 8 * h + 8); ++j) {
+                    const int par = S.kept[pos][j];
+                    if (par >= 0 && par < wnodes) atomicOr(&S.bits[par >> 5], 1u << (par & 31));
+                    else if (err) atomicCAS(err, 0, 16);  // self-check: a kept node past the tile's reach
+                }
+            }
+            if (pos < P && h == 0) S.need[pos] = rank ? 1 : 0;
+            any = rank ? 1 : 0;
+        }
+        if (!__syncthreads_or(any)) continue;
+
+        // ---- the union of the kept parents (sorted), and each parent's index in it
+        int cnt = tid < words ? __popc(S.bits[tid]) : 0;
+        const int nU = block_exscan(cnt, S.scan);
+        if (tid < words) {
+            S.pre[tid] = cnt;
+            uint32_t wbits = S.bits[tid];
+            int at = cnt;
+            while (wbits) {
+                const int bit = __ffs(wbits) - 1;
+                wbits &= wbits - 1;
+                S.uni[at++] = tid * 32 + bit;
+            }
+        }
+        __syncthreads();
+        if ((tid >> 1) < P && S.need[tid >> 1]) {
+            const int pos = tid >> 1, h = tid & 1;
+            const int nk = S.nkept[pos];
+            for (int j = 8 * h; j < min(nk, 8 * h + 8); ++j) {
+                const int par = S.kept[pos][j];
+                const uint32_t below = S.bits[par >> 5] & ((1u << (par & 31)) - 1u);
+                S.keptu[pos][j] = S.pre[par >> 5] + __popc(below);
+            }
+        }
+        __syncthreads();
+
+        // ---- chunks of 32 union parents: gather, MMA, pick-up
+        const int64_t child_off = p.geom.off[l - 1];
+        const int64_t child_M = p.geom.M[l - 1];
+        const int64_t span_child = (int64_t)p.C << (l - 2);
+        if (nU > kTwHandoff) {  // low reuse from here down: the one-warp walk continues at level l
+            lstop = l;
+            break;
+        }
+        const int nch = (nU + kTwPar - 1) / kTwPar;
+        auto gather = [&](int k, int buf) {
+            const int n = min(kTwPar, nU - k * kTwPar);
+            const uint32_t dst_hi = tc::smem_u32(S.b[buf][0]), dst_lo = tc::smem_u32(S.b[buf][1]);
+            for (int i = tid; i < ((4 * n + 7) & ~7) * 32; i += kTwThreads) {
+                // 8 rows of one core-matrix group per 16-byte chunk: each 8 lanes fill 128 contiguous bytes
+                const int row = (i >> 8) * 8 + (i & 7), part = (i >> 3) & 31, c = part & 15;
+                if (row >= 4 * n) continue;
+                const int64_t node = 4 * (int64_t)S.uni[k * kTwPar + (row >> 2)] + (row & 3);
+                const bool exists = node < child_M;
+                const __nv_bfloat16* base = part < 16 ? Hh : Hl;
+                const __nv_bfloat16* src = base + (child_off + (exists ? node : 0)) * kD + c * 8;
+                const uint32_t dst = (part < 16 ? dst_hi : dst_lo) + tc::kmajor128_off(row, c);
+                if (exists) tc::cp_async16(dst, src);
+                else tc::cp_async_zero16(dst, src);
+            }
+            tc::cp_async_commit();
+        };
+        // this thread's row and its walk over its position's kept parents
+        const int r = tid & 127, wg = tid >> 7;
+        const int pos = r / G, h = r % G;
+        const bool mine = pos < P && t0 + pos < p.N && S.need[pos];
+        const int nk = mine ? S.nkept[pos] : 0;
+        int jptr = 0;
+        int ucur = nk > 0 ? S.keptu[pos][0] : kBig;
+        gather(0, 0);
+        for (int k = 0; k < nch; ++k) {
+            const int buf = k & 1;
+            tc::cp_async_wait_all();
+            tc::fence_async_smem();
+            __syncthreads();
+            if (tid == 0) {
+                tc::tc_fence_after();
+                const int n = min(kTwPar, nU - k * kTwPar);
+                const uint32_t idesc = idesc_n((4 * n + 15) & ~15);
+                const uint32_t dt = tmem + (uint32_t)(buf * 128);
+                const uint32_t bh_s = tc::smem_u32(S.b[buf][0]), bl_s = tc::smem_u32(S.b[buf][1]);
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks)
+                    tc::mma_bf16(dt, tc::smem_desc(q_smem + ks * 256, 128, 2048),
+                                 tc::smem_desc(bh_s + ks * 256, 128, 2048), idesc, ks > 0);
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks)
+                    tc::mma_bf16(dt, tc::smem_desc(q_smem + ks * 256, 128, 2048),
+                                 tc::smem_desc(bl_s + ks * 256, 128, 2048), idesc, 1u);
+                tc::mma_commit(&S.mbar[buf]);
+            }
+            // the other buffer was read by chunk k - 1's MMAs, which completed before its pick-up
+            if (k + 1 < nch) gather(k + 1, buf ^ 1);
+            ok = __syncthreads_and(tc::mbar_wait(&S.mbar[buf], parity[buf], err, 15)) != 0;
+            parity[buf] ^= 1u;
+            if (!ok) break;
+            tc::tc_fence_after();
+#pragma unroll
+            for (int gi = 0; gi < 2; ++gi) {
+                const int g = 2 * wg + gi;
+                const int g0 = k * kTwPar + g * 8;  // union index of the group's first parent
+                while (ucur < g0) {  // parents of the other warpgroup's groups
+                    ++jptr;
+                    ucur = jptr < nk ? S.keptu[pos][jptr] : kBig;
+                }
+                if (!__any_sync(kFull, ucur < g0 + 8)) continue;
+                __syncwarp();
+                float v[32];
+                tc::tmem_ld32(tmem + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)(buf * 128 + g * 32), v);
+                tc::tmem_ld_wait();
+                while (ucur < g0 + 8) {
+                    const int dlt = ucur - g0;
+                    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        if (dlt == i) {
+                            a0 = v[4 * i];
+                            a1 = v[4 * i + 1];
+                            a2 = v[4 * i + 2];
+                            a3 = v[4 * i + 3];
+                        }
+                    const int64_t par = S.kept[pos][jptr];
+                    // children 4 par + 1 and 4 par + 3 (the second child of each candidate) may not exist
+                    const bool has1 = (4 * par + 1) * span_child < p.N;
+                    const bool has3 = (4 * par + 3) * span_child < p.N;
+                    const float z0 = a0 * p.qscale, z1 = a1 * p.qscale, z2 = a2 * p.qscale, z3 = a3 * p.qscale;
+                    float* sc = S.score + pos * (kSlots * G + 1) + 2 * jptr * G + h;
+                    sc[0] = pair_score(z0, has1 ? z1 : -INFINITY, p.variant);
+                    sc[G] = pair_score(z2, has3 ? z3 : -INFINITY, p.variant);
+                    ++jptr;
+                    ucur = jptr < nk ? S.keptu[pos][jptr] : kBig;
+                }
+            }
+            tc::tc_fence_before();
+        }
+        tc::cp_async_wait_all();
+        __syncthreads();
+        if (!ok) break;
+
+        // ---- two lanes per ranking position: forced first, then the best by score (lower index on ties)
+        if (warp * 32 < 2 * P) {
+            const int pos = tid >> 1, h = tid & 1;
+            const bool live = pos < P && S.need[pos];
+            HalfCands hc;
+            half_cands(S, pos, l, L, live ? t0 + pos : 0, p, h, live, hc);
+            const uint32_t vfull = pair_mask(hc.v, h), ffull = pair_mask(hc.f, h);
+            float score[16];
+            const float* sc = S.score + pos * (kSlots * G + 1) + 16 * h * G;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                float x = 0.f;
+#pragma unroll
+                for (int hh = 0; hh < G; ++hh) x += live ? sc[i * G + hh] : 0.f;  // Eq.(11): summed over the group
+                score[i] = x;
+            }
+            const uint32_t keep = rank_keep(score, hc, vfull, ffull, p.K, h);
+            __syncwarp();  // both lanes have read the kept nodes they expand
+            if (live) write_kept(S, pos, hc, keep, h);
+        }
+        __syncthreads();
+    }
+
+    if (ok && lstop == 1) {
+        // ---- every level done: the level-1 candidates and the sibling-pair
+        // bucket counts, as the one-warp walk writes them
+        if (warp * 32 < 2 * P) {
+            const int pos = tid >> 1, h = tid & 1;
+            const bool live = pos < P && t0 + pos < p.N;
+            const int64_t t = live ? t0 + pos : 0;
+            const int64_t M1 = p.geom.M[1];
+            HalfCands hc;
+            half_cands(S, pos, 1, L, t, p, h, live, hc);
+            if (live) {
+                const int64_t unit = bh * p.N + t;
+                int last = -1;
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const bool valid = (hc.v >> i) & 1u;
+                    const int cand = hc.node[i];
+                    const bool in_range = cand >= 0 && cand < M1;
+                    if (valid && !in_range && err) atomicCAS(err, 0, 10);  // self-check: never expected
+                    if (valid && last >= 0 && last >= cand && err) atomicCAS(err, 0, 14);  // slots ascend
+                    if (valid) last = cand;
+                    hc.node[i] = valid && in_range ? cand : -1;
+                    cand_out[unit * kSlots + 16 * h + i] = hc.node[i];
+                }
+#pragma unroll
+                for (int i = 0; i < 16; i += 2) {  // a sibling pair with at least one leaf that is not forced
+                    const int c0 = hc.node[i], c1 = hc.node[i + 1];
+                    const bool free0 = c0 >= 0 && !((hc.f >> i) & 1u);
+                    const bool free1 = c1 >= 0 && !((hc.f >> (i + 1)) & 1u);
+                    if (c0 >= 0 && (free0 || free1))
+                        slots[unit * kPairs + 8 * h + i / 2] = atomicAdd(&counts[bh * ((M1 + 1) / 2) + (c0 >> 1)], 1);
+                }
+                if (h == 0) resume[unit] = 0;
+            }
+        }
+    } else if (ok) {
+        // ---- hand each position's walk over to the one-warp walk: its kept
+        // nodes one level above the level it resumes at
+        const int pos = tid >> 1, h = tid & 1;
+        if (pos < P && t0 + pos < p.N) {
+            const int64_t unit = bh * p.N + t0 + pos;
+            // positions that ranked at the level handed over still hold that level's parents
+            const int level = S.need[pos] ? lstop : lstop - 1;
+            const int nk = S.nkept[pos];
+            for (int j = 8 * h; j < min(nk, 8 * h + 8); ++j) cand_out[unit * kSlots + j] = S.kept[pos][j];
+            if (h == 0) resume[unit] = (level << 8) | nk;
+        }
+    }
+    tc::cp_async_wait_all();
+    tc::tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc::tc_fence_after();
+        tc::tmem_dealloc(tmem, 256);
+    }
+}
+
+// fp32 summaries -> bf16 high and low parts: hi = bf16(x), lo = bf16(x - hi)
+__global__ void split_pyramid_kernel(const float4* __restrict__ pyr, uint2* __restrict__ hi, uint2* __restrict__ lo,
+                                     int64_t n4) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (int64_t)gridDim.x * blockDim.x) {
+        const float4 x = pyr[i];
+        const __nv_bfloat162 h01 = __floats2bfloat162_rn(x.x, x.y), h23 = __floats2bfloat162_rn(x.z, x.w);
+        const float2 f01 = __bfloat1622float2(h01), f23 = __bfloat1622float2(h23);
+        const __nv_bfloat162 l01 = __floats2bfloat162_rn(x.x - f01.x, x.y - f01.y);
+        const __nv_bfloat162 l23 = __floats2bfloat162_rn(x.z - f23.x, x.w - f23.y);
+        uint2 uh, ul;
+        uh.x = *reinterpret_cast<const uint32_t*>(&h01);
+        uh.y = *reinterpret_cast<const uint32_t*>(&h23);
+        ul.x = *reinterpret_cast<const uint32_t*>(&l01);
+        ul.y = *reinterpret_cast<const uint32_t*>(&l23);
+        hi[i] = uh;
+        lo[i] = ul;
+    }
+}
+
+cudaError_t launch_split_pyramid_impl(const float* pyr, void* pyr_hl, int64_t elems, int sms, cudaStream_t st) {
+    __nv_bfloat16* hi = (__nv_bfloat16*)pyr_hl;
+    split_pyramid_kernel<<<sms * 8, 256, 0, st>>>((const float4*)pyr, (uint2*)hi, (uint2*)(hi + elems), elems / 4);
+    return cudaGetLastError();
+}
+
+template <int G>
+cudaError_t walk_tc_t(const void* Q, const float* pyr, void* pyr_hl, int32_t* cand, int32_t* resume, int32_t* counts,
+                      int32_t* slots, int* err, const SelectParams& sp, int sms, cudaStream_t st) {
+    const int64_t elems = (int64_t)sp.B * sp.Hkv * sp.geom.rows * kD;
+    cudaError_t e = launch_split_pyramid(pyr, pyr_hl, elems, sms, st);
+    if (e != cudaSuccess) return e;
+    const __nv_bfloat16* hi = (const __nv_bfloat16*)pyr_hl;
+    const __nv_bfloat16* lo = hi + elems;
+    constexpr int P = 128 / G;
+    const int tiles_per_head = (sp.N + P - 1) / P;
+    const size_t smem = sizeof(TwSmem);
+    auto kern = walk_tc_kernel<G>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int64_t grid = (int64_t)sp.B * sp.Hkv * tiles_per_head;
+    kern<<<(unsigned)grid, kTwThreads, smem, st>>>((const __nv_bfloat16*)Q, hi, lo, cand, resume, counts, slots,
+                                                   tiles_per_head, err, sp);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_split_pyramid(const float* pyr, void* pyr_hl, int64_t elems, int sms, cudaStream_t st) {
+    return launch_split_pyramid_impl(pyr, pyr_hl, elems, sms, st);
+}
+
+bool walk_tc_fits(const SelectParams& sp) {
+    // at least one ranked level below the root's children, and a union bitmap
+    // that covers the parent level of every ranked level (at most 8192 nodes)
+    return sp.geom.L >= 3 && sp.geom.M[3] <= (int64_t)kTwMaxWords * 32;
+}
+
+size_t walk_tc_pyramid_bytes(int64_t units_bh, int64_t rows) { return (size_t)units_bh * rows * kD * 2 * 2; }
+
+cudaError_t launch_walk_tc(const void* Q, const float* pyr, void* pyr_hl, int32_t* cand, int32_t* resume,
+                           int32_t* counts, int32_t* slots, int* err, const SelectParams& sp, int G, int sms,
+                           cudaStream_t st) {
+    switch (G) {
+        case 1: return walk_tc_t<1>(Q, pyr, pyr_hl, cand, resume, counts, slots, err, sp, sms, st);
+        case 2: return walk_tc_t<2>(Q, pyr, pyr_hl, cand, resume, counts, slots, err, sp, sms, st);
+        case 4: return walk_tc_t<4>(Q, pyr, pyr_hl, cand, resume, counts, slots, err, sp, sms, st);
+        case 8: return walk_tc_t<8>(Q, pyr, pyr_hl, cand, resume, counts, slots, err, sp, sms, st);
+        case 16: return walk_tc_t<16>(Q, pyr, pyr_hl, cand, resume, counts, slots, err, sp, sms, st);
+    }
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace pisa

@@ -70,6 +70,7 @@ def load(path: str | None = None):
             "pisa_sparse_attn": (ctypes.c_int, [cfgp, P, P, P, P, P, P]),
             "pisa_forward": (ctypes.c_int, [cfgp, P, P, P, P, P, P, P]),
             "pisa_bsa_select": (ctypes.c_int, [cfgp, P, P, P, P]),
+            "pisa_bsa_select_ws": (ctypes.c_int, [cfgp, P, P, P, P, ctypes.c_size_t, P]),
             "pisa_workspace_bytes": (ctypes.c_int64, [cfgp]),
             "pisa_workspace_status": (ctypes.c_int, [cfgp, P, P]),
             "pisa_select_ws": (ctypes.c_int, [cfgp, P, P, P, P, P, ctypes.c_size_t, P]),
@@ -192,6 +193,12 @@ def pisa_forward(cfg, Q, K, V, pyr, idx, O):
 
 def pisa_bsa_select(cfg, Q, pyr, idx):
     _check("pisa_bsa_select", load().pisa_bsa_select(ctypes.byref(cfg), _ptr(Q), _ptr(pyr), _ptr(idx), _stream()))
+
+
+def pisa_bsa_select_ws(cfg, Q, pyr, idx, ws):
+    """Flat BSA selection (Eq.1) on the tensor cores, in the block-major workspace."""
+    _check("pisa_bsa_select_ws", load().pisa_bsa_select_ws(ctypes.byref(cfg), _ptr(Q), _ptr(pyr), _ptr(idx),
+                                                           _ptr(ws), ws.numel(), _stream()))
 
 
 # ---- block-major tensor-core prefill (workspace) -----------------------------------

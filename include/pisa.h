@@ -153,6 +153,18 @@ int pisa_forward(const pisa_cfg *cfg, const void *Q, const void *K, const void *
  * Q: [B, Hq, N, d]; idx: int32 [B, Hkv, N, K] (written). */
 int pisa_bsa_select(const pisa_cfg *cfg, const void *Q, const float *pyr, int32_t *idx,
                     void *stream);
+/* Flat BSA selection (close reading §02, Eq.(1)) on the tensor cores: the
+ * same selection as pisa_bsa_select (forced leaves first, the best eligible
+ * leaves by the mean-summary dot summed over the group, ties to the lower
+ * leaf; idx sorted ascending, -1 padded), computed as S = Q x leaves^T per tile
+ * of 128 (position, head) rows with a streaming Top-K. Rows whose K-th and
+ * (K+1)-th scores differ by less than about 1e-5 may differ from the CUDA-core
+ * call (the summaries enter as bf16 high and low parts). Limits and workspace
+ * as pisa_select_ws (bf16, d = 128, C = 64; pisa_workspace_bytes bytes,
+ * 256-byte aligned; it uses the workspace's pyramid-split region);
+ * pisa_workspace_status reports a tile that gave up a bounded wait. */
+int pisa_bsa_select_ws(const pisa_cfg *cfg, const void *Q, const float *pyr, int32_t *idx, void *workspace,
+                       size_t workspace_bytes, void *stream);
 
 /* ---- block-major tensor-core prefill (close reading §05 Algorithm 1, §5.1) ------
  * The pages' two-stage form: Stage 1 walks the internal levels per query;
