@@ -512,9 +512,9 @@ __global__ void __launch_bounds__(128) leaf_score_kernel(const __nv_bfloat16* __
                 float s = 0.f;
 #pragma unroll
                 for (int j = 0; j < 64; ++j)
-                    if (j < nvalid) s += exp2f(v[j] * p.qscale - m);
+                    if (j < nvalid) s += ex2_approx(v[j] * p.qscale - m);
                 const int64_t unit = bh * p.N + t;
-                lse[(unit * kSlots + slot) * G + (tid % G)] = m + log2f(s);
+                lse[(unit * kSlots + slot) * G + (tid % G)] = m + lg2_approx(s);
                 if constexpr (VSCORE) {  // PISA-1 / PISA-2 ranking score: two-pass mean and variance of the logits
                     float sum = 0.f;
 #pragma unroll
@@ -715,8 +715,8 @@ __global__ void __launch_bounds__(128) attn_tile_kernel(const __nv_bfloat16* __r
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
                     const int j = c * 8 + q * 2;
-                    const float p0 = j < nvalid ? exp2f(v[j] * p.qscale - z) : 0.f;
-                    const float p1 = j + 1 < nvalid ? exp2f(v[j + 1] * p.qscale - z) : 0.f;
+                    const float p0 = j < nvalid ? ex2_approx(v[j] * p.qscale - z) : 0.f;
+                    const float p1 = j + 1 < nvalid ? ex2_approx(v[j + 1] * p.qscale - z) : 0.f;
                     __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
                     w4[q] = *reinterpret_cast<uint32_t*>(&h2);
                 }
@@ -919,8 +919,8 @@ __global__ void __launch_bounds__(128) forced_tile_kernel(const __nv_bfloat16* _
                 float sum = 0.f;
 #pragma unroll
                 for (int j = 0; j < 64; ++j)
-                    if (j < nvalid) sum += exp2f(v[j] * p.qscale - m);
-                lse_f = logaddexp2f(lse_f, m + log2f(sum));
+                    if (j < nvalid) sum += ex2_approx(v[j] * p.qscale - m);
+                lse_f = logaddexp2f(lse_f, m + lg2_approx(sum));
             }
             tc::tc_fence_before();
             __syncthreads();
@@ -962,8 +962,8 @@ __global__ void __launch_bounds__(128) forced_tile_kernel(const __nv_bfloat16* _
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
                         const int j = c * 8 + q * 2;
-                        const float p0 = j < nvalid ? exp2f(v[j] * p.qscale - z) : 0.f;
-                        const float p1 = j + 1 < nvalid ? exp2f(v[j + 1] * p.qscale - z) : 0.f;
+                        const float p0 = j < nvalid ? ex2_approx(v[j] * p.qscale - z) : 0.f;
+                        const float p1 = j + 1 < nvalid ? ex2_approx(v[j + 1] * p.qscale - z) : 0.f;
                         __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
                         w4[q] = *reinterpret_cast<uint32_t*>(&h2);
                     }
@@ -1303,13 +1303,13 @@ __global__ void __launch_bounds__(128) bwd_stats_kernel(
                     if (c * 32 + j < nvalid) mc = fmaxf(mc, sv[j] * p.qscale);
                 const float mn = fmaxf(m, mc);
                 if (mn != -INFINITY) {
-                    const float sc = exp2f(m - mn);
+                    const float sc = ex2_approx(m - mn);
                     l *= sc;
                     dd *= sc;
 #pragma unroll
                     for (int j = 0; j < 32; ++j)
                         if (c * 32 + j < nvalid) {
-                            const float w = exp2f(sv[j] * p.qscale - mn);
+                            const float w = ex2_approx(sv[j] * p.qscale - mn);
                             l += w;
                             dd = fmaf(w, dp[j], dd);
                         }
@@ -1318,7 +1318,7 @@ __global__ void __launch_bounds__(128) bwd_stats_kernel(
             }
             if (t >= 0) {
                 const int64_t o = ((bh * p.N + t) * p.K + rk[tid]) * G + (tid % G);
-                lse_s[o] = l > 0.f ? m + log2f(l) : -INFINITY;
+                lse_s[o] = l > 0.f ? m + lg2_approx(l) : -INFINITY;
                 dbar_s[o] = l > 0.f ? dd / l : 0.f;
             }
         }
@@ -1556,8 +1556,8 @@ __global__ void __launch_bounds__(256, 1) bwd_tile_kernel(
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
                     const int i = c * 8 + q * 2, j = half * 32 + i;
-                    const float p0 = j < nvalid ? exp2f(sv[i] * p.qscale - z) : 0.f;
-                    const float p1 = j + 1 < nvalid ? exp2f(sv[i + 1] * p.qscale - z) : 0.f;
+                    const float p0 = j < nvalid ? ex2_approx(sv[i] * p.qscale - z) : 0.f;
+                    const float p1 = j + 1 < nvalid ? ex2_approx(sv[i + 1] * p.qscale - z) : 0.f;
                     __nv_bfloat162 hp = __floats2bfloat162_rn(p0, p1);
                     __nv_bfloat162 hs = __floats2bfloat162_rn(p0 * (dp[i] - dd), p1 * (dp[i + 1] - dd));
                     wp[q] = *reinterpret_cast<uint32_t*>(&hp);

@@ -103,9 +103,15 @@ struct HalfCands {
 
 __device__ __forceinline__ void half_cands(const TwSmem& S, int pos, int l, int L, int64_t t, const SelectParams& p,
                                            int h, bool live, HalfCands& hc) {
-    const Forced F(t, p.C, p.causal, p.forced_mask);
-    const int nk = (!live || l == L) ? 0 : S.nkept[pos];
+    // node i of level l exists and is eligible iff 0 <= i <= vmax (M_l = ceil(N / span))
     const int64_t span = (int64_t)p.C << (l - 1);
+    const int64_t lastn = p.geom.M[l] - 1;
+    const int vmax = (int)(p.causal ? min(lastn, t / span) : lastn);
+    // the forced leaves' ancestors at level l (-2: none)
+    const Forced F(t, p.C, p.causal, p.forced_mask);
+    const int s = l - 1;
+    const int fa = F.f0 >= 0 ? F.f0 >> s : -2, fb = F.f1 >= 0 ? F.f1 >> s : -2, fc = F.f2 >= 0 ? F.f2 >> s : -2;
+    const int nk = (!live || l == L) ? 0 : S.nkept[pos];
     hc.v = hc.f = 0u;
 #pragma unroll
     for (int jj = 0; jj < 8; ++jj) {
@@ -116,10 +122,9 @@ __device__ __forceinline__ void half_cands(const TwSmem& S, int pos, int l, int 
             const int i = 2 * jj + e;
             const int node = l == L ? (par == 0 && e == 0 ? 0 : -1) : (par >= 0 ? 2 * par + e : -1);
             hc.node[i] = node;
-            const int64_t first = (int64_t)node * span;
-            const bool valid = node >= 0 && first < p.N && (!p.causal || first <= t);
+            const bool valid = (unsigned)node <= (unsigned)vmax;
             hc.v |= (valid ? 1u : 0u) << i;
-            hc.f |= (valid && F.has(node, l) ? 1u : 0u) << i;
+            hc.f |= (valid && (node == fa || node == fb || node == fc) ? 1u : 0u) << i;
         }
     }
 }
@@ -158,29 +163,21 @@ __device__ __forceinline__ uint32_t ordered(float x) {
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-__device__ __forceinline__ void cex(uint64_t& x, uint64_t& y, bool desc) {
-    const uint64_t big = x > y ? x : y, small = x > y ? y : x;
-    x = desc ? big : small;
-    y = desc ? small : big;
-}
-
 // The keep rule of a ranked level (close reading §04 4.2; Eq.(6)): forced
 // candidates first, then the best scores, ties to the lower node (= lower
-// slot). Each candidate's key packs (score, 31 - slot) into 64 bits, so the
-// keys are distinct and their order is the rank order. The two lanes of a
-// position sort their 16 keys in opposite directions (a bitonic sequence of
-// 32), exchange once, and lane half 0 ends with the 16 largest, descending;
-// the top K are kept. Returns the 32-slot keep mask on both lanes.
-__device__ __forceinline__ uint32_t rank_keep(const float (&score)[16], const HalfCands& hc, uint32_t vfull,
-                                              uint32_t ffull, int K, int h) {
-    uint64_t a[16];
+// slot). Keys are the scores mapped order-preservingly onto uint32 (forced:
+// the maximum, not eligible: 0). The two lanes of a position sort their 16
+// keys in opposite directions (a bitonic sequence of 32), exchange once, and
+// lane half 0 ends with the 16 largest, descending, so the K-th largest key
+// tau is known; the kept set is every key above tau and, of the keys equal to
+// tau, the lowest slots that fill K. Returns the 32-slot keep mask on both lanes.
+__device__ __forceinline__ uint32_t rank_keep(const float* score, int stride, uint32_t vfull, uint32_t ffull,
+                                              int K, int h) {
+    const uint32_t vm = (vfull >> (16 * h)) & 0xffffu, fm = (ffull >> (16 * h)) & 0xffffu;
+    uint32_t a[16];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-        const int c = 16 * h + i;
-        const bool v = (vfull >> c) & 1u, f = (ffull >> c) & 1u;
-        const uint32_t hi = !v ? 0u : f ? 0xffffffffu : ordered(score[i]);
-        a[i] = ((uint64_t)hi << 32) | (uint32_t)(kSlots - 1 - c);
-    }
+    for (int i = 0; i < 16; ++i)
+        a[i] = !((vm >> i) & 1u) ? 0u : ((fm >> i) & 1u) ? 0xffffffffu : ordered(score[i * stride]);
 #pragma unroll
     for (int k = 2; k <= 16; k <<= 1)
 #pragma unroll
@@ -188,28 +185,42 @@ __device__ __forceinline__ uint32_t rank_keep(const float (&score)[16], const Ha
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
                 const int m = i ^ j;
-                if (m > i) cex(a[i], a[m], k == 16 ? h == 0 : (i & k) == 0);
+                if (m > i) {
+                    const bool desc = k == 16 ? h == 0 : (i & k) == 0;
+                    const uint32_t x = a[i], y = a[m];
+                    a[i] = desc ? max(x, y) : min(x, y);
+                    a[m] = desc ? min(x, y) : max(x, y);
+                }
             }
 #pragma unroll
     for (int i = 0; i < 16; ++i) {  // the cross-lane step of the 32-key merge
-        const uint32_t lo = __shfl_xor_sync(kFull, (uint32_t)a[i], 1);
-        const uint32_t hi = __shfl_xor_sync(kFull, (uint32_t)(a[i] >> 32), 1);
-        const uint64_t o = ((uint64_t)hi << 32) | lo;
-        a[i] = h == 0 ? (a[i] > o ? a[i] : o) : (a[i] > o ? o : a[i]);
+        const uint32_t o = __shfl_xor_sync(kFull, a[i], 1);
+        a[i] = h == 0 ? max(a[i], o) : min(a[i], o);
     }
 #pragma unroll
     for (int j = 8; j > 0; j >>= 1)
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
             const int m = i ^ j;
-            if (m > i) cex(a[i], a[m], true);
+            if (m > i) {
+                const uint32_t x = a[i], y = a[m];
+                a[i] = max(x, y);
+                a[m] = min(x, y);
+            }
         }
-    uint32_t keep = 0u;
+    uint32_t tau = 0u;  // a[K - 1], picked with masks (an indexed read would put a[] in local memory)
 #pragma unroll
-    for (int i = 0; i < 16; ++i)
-        if (i < K) keep |= 1u << (kSlots - 1 - (int)(a[i] & 31u));
-    keep = __shfl_sync(kFull, keep, (threadIdx.x & 31) & ~1);
-    return keep & vfull;
+    for (int i = 0; i < 16; ++i) tau |= a[i] & (0u - (uint32_t)(i == K - 1));
+    tau = __shfl_sync(kFull, tau, (threadIdx.x & 31) & ~1);
+    uint32_t gt = 0u, eq = 0u;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const uint32_t k = !((vm >> i) & 1u) ? 0u : ((fm >> i) & 1u) ? 0xffffffffu : ordered(score[i * stride]);
+        gt |= (k > tau ? 1u : 0u) << i;
+        eq |= (k == tau ? 1u : 0u) << i;
+    }
+    const uint32_t gt_full = pair_mask(gt, h), eq_full = pair_mask(eq, h);
+    return (gt_full | lowest_bits(eq_full, K - __popc(gt_full))) & vfull;
 }
 
 template <int G>
@@ -346,7 +357,7 @@ __global__ void __launch_bounds__(kTwThreads, 1) walk_tc_kernel(
         // ---- chunks of 32 union parents: gather, MMA, pick-up
         const int64_t child_off = p.geom.off[l - 1];
         const int64_t child_M = p.geom.M[l - 1];
-        const int64_t span_child = (int64_t)p.C << (l - 2);
+        const int child_rows = (int)child_M;  // rows of level l - 1 (a row exists iff its first key is before N)
         if (nU > kTwHandoff) {  // low reuse from here down: the one-warp walk continues at level l
             lstop = l;
             break;
@@ -374,8 +385,9 @@ __global__ void __launch_bounds__(kTwThreads, 1) walk_tc_kernel(
         const int pos = r / G, h = r % G;
         const bool mine = pos < P && t0 + pos < p.N && S.need[pos];
         const int nk = mine ? S.nkept[pos] : 0;
-        int jptr = 0;
-        int ucur = nk > 0 ? S.keptu[pos][0] : kBig;
+        int uj[16];  // union index of each of its kept parents (ascending; kBig past the count)
+#pragma unroll
+        for (int j = 0; j < 16; ++j) uj[j] = j < nk ? S.keptu[pos][j] : kBig;
         gather(0, 0);
         for (int k = 0; k < nch; ++k) {
             const int buf = k & 1;
@@ -404,40 +416,45 @@ __global__ void __launch_bounds__(kTwThreads, 1) walk_tc_kernel(
             parity[buf] ^= 1u;
             if (!ok) break;
             tc::tc_fence_after();
+            // bit i: union parent k * 32 + i is one of this row's kept parents;
+            // `base`: how many of its kept parents lie in earlier chunks
+            const int c0u = k * kTwPar;
+            uint32_t mask = 0u;
+            int base = 0;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const int dlt = uj[j] - c0u;
+                mask |= (dlt >= 0 && dlt < kTwPar) ? (1u << dlt) : 0u;
+                base += uj[j] < c0u ? 1 : 0;
+            }
 #pragma unroll
             for (int gi = 0; gi < 2; ++gi) {
-                const int g = 2 * wg + gi;
-                const int g0 = k * kTwPar + g * 8;  // union index of the group's first parent
-                while (ucur < g0) {  // parents of the other warpgroup's groups
-                    ++jptr;
-                    ucur = jptr < nk ? S.keptu[pos][jptr] : kBig;
-                }
-                if (!__any_sync(kFull, ucur < g0 + 8)) continue;
+                const int g = 2 * wg + gi;  // 8 parents: columns 32 g .. 32 g + 31
+                const uint32_t m8 = (mask >> (8 * g)) & 0xffu;
+                if (!__any_sync(kFull, m8 != 0u)) continue;
                 __syncwarp();
                 float v[32];
                 tc::tmem_ld32(tmem + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)(buf * 128 + g * 32), v);
                 tc::tmem_ld_wait();
-                while (ucur < g0 + 8) {
-                    const int dlt = ucur - g0;
-                    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+                const int before = base + __popc(mask & ((1u << (8 * g)) - 1u));
 #pragma unroll
-                    for (int i = 0; i < 8; ++i)
-                        if (dlt == i) {
-                            a0 = v[4 * i];
-                            a1 = v[4 * i + 1];
-                            a2 = v[4 * i + 2];
-                            a3 = v[4 * i + 3];
+                for (int i = 0; i < 8; ++i) {
+                    if ((m8 >> i) & 1u) {
+                        const int j = before + __popc(m8 & ((1u << i) - 1u));  // its place in the kept list
+                        const int par = S.uni[c0u + 8 * g + i];
+                        // children 4 par + 1 and 4 par + 3 (the second child of each candidate) may not exist
+                        const bool has1 = 4 * par + 1 < child_rows, has3 = 4 * par + 3 < child_rows;
+                        const float z0 = v[4 * i] * p.qscale, z1 = has1 ? v[4 * i + 1] * p.qscale : -INFINITY;
+                        const float z2 = v[4 * i + 2] * p.qscale, z3 = has3 ? v[4 * i + 3] * p.qscale : -INFINITY;
+                        float* sc = S.score + pos * (kSlots * G + 1) + 2 * j * G + h;
+                        if (p.variant == 0) {  // Eq.(7): the LSE over the two children
+                            sc[0] = lse2_pair(z0, z1);
+                            sc[G] = lse2_pair(z2, z3);
+                        } else {
+                            sc[0] = pair_score(z0, z1, p.variant);
+                            sc[G] = pair_score(z2, z3, p.variant);
                         }
-                    const int64_t par = S.kept[pos][jptr];
-                    // children 4 par + 1 and 4 par + 3 (the second child of each candidate) may not exist
-                    const bool has1 = (4 * par + 1) * span_child < p.N;
-                    const bool has3 = (4 * par + 3) * span_child < p.N;
-                    const float z0 = a0 * p.qscale, z1 = a1 * p.qscale, z2 = a2 * p.qscale, z3 = a3 * p.qscale;
-                    float* sc = S.score + pos * (kSlots * G + 1) + 2 * jptr * G + h;
-                    sc[0] = pair_score(z0, has1 ? z1 : -INFINITY, p.variant);
-                    sc[G] = pair_score(z2, has3 ? z3 : -INFINITY, p.variant);
-                    ++jptr;
-                    ucur = jptr < nk ? S.keptu[pos][jptr] : kBig;
+                    }
                 }
             }
             tc::tc_fence_before();
@@ -453,16 +470,17 @@ __global__ void __launch_bounds__(kTwThreads, 1) walk_tc_kernel(
             HalfCands hc;
             half_cands(S, pos, l, L, live ? t0 + pos : 0, p, h, live, hc);
             const uint32_t vfull = pair_mask(hc.v, h), ffull = pair_mask(hc.f, h);
-            float score[16];
-            const float* sc = S.score + pos * (kSlots * G + 1) + 16 * h * G;
+            float* sc = S.score + pos * (kSlots * G + 1) + 16 * h * G;
+            if (G > 1 && live) {  // Eq.(11): summed over the group, into the first head's entry
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                float x = 0.f;
+                for (int i = 0; i < 16; ++i) {
+                    float x = 0.f;
 #pragma unroll
-                for (int hh = 0; hh < G; ++hh) x += live ? sc[i * G + hh] : 0.f;  // Eq.(11): summed over the group
-                score[i] = x;
+                    for (int hh = 0; hh < G; ++hh) x += sc[i * G + hh];
+                    sc[i * G] = x;
+                }
             }
-            const uint32_t keep = rank_keep(score, hc, vfull, ffull, p.K, h);
+            const uint32_t keep = rank_keep(sc, G, vfull, ffull, p.K, h);
             __syncwarp();  // both lanes have read the kept nodes they expand
             if (live) write_kept(S, pos, hc, keep, h);
         }
