@@ -442,7 +442,10 @@ __global__ void __launch_bounds__(128) leaf_score_kernel(const __nv_bfloat16* __
     extern __shared__ __align__(1024) uint8_t dsm[];
     uint8_t* sA = dsm;           // 32 KB gathered query rows
     uint8_t* sB = dsm + 32768;   // NK x 256 B key rows
-    __shared__ TileRows tr;
+    // Two row tables: while tile i's logits are turned into LSEs, tile i + 1's
+    // metadata is read and its query and key rows are gathered into the
+    // operand buffers (free once tile i's MMA has completed).
+    __shared__ TileRows trs[2];
     __shared__ __align__(8) uint64_t mbar;
     __shared__ uint32_t tmem_base;
     const int tid = threadIdx.x, warp = tid >> 5;
@@ -459,34 +462,65 @@ __global__ void __launch_bounds__(128) leaf_score_kernel(const __nv_bfloat16* __
     const int ntiles = min(*ntiles_ptr, p.max_tiles);
     const int64_t nkeys = PAIR ? (p.M1 + 1) / 2 : p.M1;
     uint32_t phase = 0;
-    bool ok;
-    for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
-        const int4 td = tiles[tile];
-        const int64_t bh = td.x, key = td.y;
-        const int64_t b = bh / p.Hkv;
-        const int kvh = (int)(bh - b * p.Hkv);
+    bool ok = true;
+    // tile descriptor + the row table; false for a tile past the list or a malformed one
+    auto fetch = [&](int tile, int buf, int4& td) {
+        if (tile >= ntiles) return false;
+        td = tiles[tile];
         if (!tile_sane(td, (int64_t)p.B * p.Hkv, nkeys, 128 / G)) {  // self-check: never expected
             if (tid == 0) atomicCAS(err, 0, 12);
-            continue;
+            return false;
         }
-        tile_rows<G>(tr, entries, td.z, td.w, p.N, err, tid);
-        __syncthreads();
-        gather_q<G>(a_smem, tr, Q, b, kvh, p.Hq, p.N, tid);
-        load_kblock<NK>(b_smem, Kmat + bh * p.N * kD, key * NK, p.N, tid);
+        tile_rows<G>(trs[buf], entries, td.z, td.w, p.N, err, tid);
+        return true;
+    };
+    // Consecutive tiles of a bucket share their key block, so each CTA takes
+    // runs of kRun consecutive tiles (run r of CTA c is r * gridDim.x + c) and
+    // reloads the keys only when the bucket changes.
+    constexpr int kRun = 8;
+    auto tile_of = [&](int it) { return ((it / kRun) * (int)gridDim.x + (int)blockIdx.x) * kRun + it % kRun; };
+    int2 kb_loaded = make_int2(-1, -1);  // (b * Hkv + kvh, key) of the key block in sB
+    auto gather = [&](const int4& td, int buf) {
+        const int64_t bh = td.x;
+        const int64_t b = bh / p.Hkv;
+        gather_q<G>(a_smem, trs[buf], Q, b, (int)(bh - b * p.Hkv), p.Hq, p.N, tid);
+        if (kb_loaded.x != td.x || kb_loaded.y != td.y) {
+            load_kblock<NK>(b_smem, Kmat + bh * p.N * kD, (int64_t)td.y * NK, p.N, tid);
+            kb_loaded = make_int2(td.x, td.y);
+        }
         tc::cp_async_commit();
+    };
+    int4 td_next;
+    bool have_next = fetch(tile_of(0), 0, td_next);
+    __syncthreads();
+    if (have_next) gather(td_next, 0);
+    int buf = 0;
+    for (int it = 0, tile = tile_of(0); tile < ntiles; tile = tile_of(++it), buf ^= 1) {
+        const int4 td = td_next;
+        const bool have = have_next;
+        const int64_t bh = td.x, key = td.y;
         tc::cp_async_wait_all();
         tc::fence_async_smem();
         __syncthreads();
-        if (tid == 0) {
+        if (have && tid == 0) {
             tc::tc_fence_after();
             issue_qk<NK>(tmem, a_smem, b_smem);
             tc::mma_commit(&mbar);
         }
+        // the next tile's row table goes to the other buffer (read last by tile i - 1's epilogue)
+        have_next = fetch(tile_of(it + 1), buf ^ 1, td_next);
         // a CTA-uniform verdict: every thread polls, all agree before moving on
-        ok = __syncthreads_and(tc::mbar_wait(&mbar, phase, err, 1)) != 0;
-        phase ^= 1;
+        if (have) {
+            ok = __syncthreads_and(tc::mbar_wait(&mbar, phase, err, 1)) != 0;
+            phase ^= 1;
+        } else {
+            __syncthreads();
+        }
         if (!ok) break;
+        if (have_next) gather(td_next, buf ^ 1);  // the operand buffers are free: this tile's MMA is done
+        if (!have) continue;
         tc::tc_fence_after();
+        const TileRows& tr = trs[buf];
         const int t = tr.t[tid];
         const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16);
 #pragma unroll
@@ -532,8 +566,8 @@ __global__ void __launch_bounds__(128) leaf_score_kernel(const __nv_bfloat16* __
             }
         }
         tc::tc_fence_before();
-        __syncthreads();
     }
+    tc::cp_async_wait_all();
     __syncthreads();
     if (warp == 0) {
         tc::tc_fence_after();

@@ -1,6 +1,6 @@
-// walk_tc.cu -- the internal levels of the pyramid walk (Stage 1 of close
-// reading §05 Algorithm 1; Eq.(5)-(7), (11); §5.3 forced and causal rules)
-// for a tile of consecutive query positions on the tensor cores.
+// walk_tc.cu -- the coarse internal levels of the pyramid walk (Stage 1 of
+// close reading §05 Algorithm 1; Eq.(5)-(7), (11); §5.3 forced and causal
+// rules) for a tile of consecutive query positions on the tensor cores.
 //
 // A CTA takes 128 MMA rows: 128/G consecutive positions of one (b, kv-head)
 // times the G query heads of the group. Every position walks the pyramid by
@@ -16,11 +16,18 @@
 // fp32 summaries enter as two bf16 parts (hi = bf16(x), lo = bf16(x - hi)),
 // and q is bf16 already, so both products are exact and S carries the
 // summaries to about 2^-16 of their size (about 1e-5 on a logit). Each row
-// then reads the four columns of each of its own kept parents and writes its
-// candidates' pair scores to shared memory; one warp per position ranks them
-// with the walk's own keep rule. After level 2 the level-1 candidates are
-// written exactly as the one-warp walk writes them (slots, sibling-pair
-// bucket counts), so the rest of the block-major selection is unchanged.
+// reads the four columns of each of its own kept parents (found with a
+// bitmask per chunk) and writes its candidates' pair scores to shared memory;
+// two adjacent lanes per position then rank them with the walk's keep rule.
+//
+// The levels above the first one where some position of the tile has more
+// than K eligible nodes are not walked: there every eligible node is kept.
+// Reuse across positions falls towards the leaves (the union grows), so a
+// level whose union needs more chunks than tw_handoff_parents allows is left
+// to the one-warp walk: each position's kept nodes go to the candidate region
+// and its resume level to `resume` (stage1_kernel<..., RESUME> continues). A
+// tile that finishes every level writes the level-1 candidates and the
+// sibling-pair bucket counts itself, exactly as the one-warp walk does.
 //
 // Per chunk, the gather of the next chunk's rows (cp.async) runs while the
 // current chunk's MMAs and row pick-up run: two B buffers and two 128-column
@@ -39,7 +46,10 @@ constexpr int kTwThreads = 256;
 constexpr int kTwPar = 32;            // union parents per chunk
 constexpr int kTwMaxWords = 256;      // bitmap words: parent levels of up to 8192 nodes
 constexpr int kTwMaxUnion = 2048;     // 128 positions x 16 kept nodes
-constexpr int kTwHandoff = 4 * kTwPar; // a level whose union needs more chunks goes to the one-warp walk
+// a level whose union needs more chunks than this goes to the one-warp walk:
+// a chunk's MMAs serve all 128 rows, so tiles of fewer positions (GQA groups)
+// afford fewer chunks per position
+__host__ __device__ constexpr int tw_handoff_parents(int positions) { return (positions >= 128 ? 8 : 4) * kTwPar; }
 constexpr int kD = 128;
 constexpr int kSlots = 32;
 constexpr int kPairs = 16;
@@ -358,7 +368,7 @@ __global__ void __launch_bounds__(kTwThreads, 1) walk_tc_kernel(
         const int64_t child_off = p.geom.off[l - 1];
         const int64_t child_M = p.geom.M[l - 1];
         const int child_rows = (int)child_M;  // rows of level l - 1 (a row exists iff its first key is before N)
-        if (nU > kTwHandoff) {  // low reuse from here down: the one-warp walk continues at level l
+        if (nU > tw_handoff_parents(P)) {  // low reuse from here down: the one-warp walk continues at level l
             lstop = l;
             break;
         }
