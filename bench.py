@@ -364,10 +364,12 @@ def dominant_roofline(w, phase_ms, alg, pk, fma_peak, fma_note, tc_peak):
                 "peak": tc_peak, "unit": "TFLOP/s", "algorithmic_per_launch": alg["leaf_flops"],
                 "peak_note": tc_note}
     elif dom == "stage1" and walk_on_tensor_cores(w):
-        roof = {"kernel": "walk_tc_kernel", "bound": "tensor", "achieved": alg["internal_flops"] / t_dom / 1e12,
-                "peak": tc_peak, "unit": "TFLOP/s", "algorithmic_per_launch": alg["internal_flops"],
-                "peak_note": tc_note + "; achieved counts the walk's own child dots (the union's extra dots and "
-                                       "the second bf16 part are not counted)"}
+        roof = {"kernel": "stage 1: walk_tc_kernel (coarse levels, tensor cores) + stage1_kernel (fine levels, "
+                          "one warp per query)",
+                "bound": "alu", "achieved": alg["internal_flops"] / t_dom / 1e12,
+                "peak": fma_peak, "unit": "TFLOP/s", "algorithmic_per_launch": alg["internal_flops"],
+                "peak_note": fma_note + "; the fine levels, which take most of the phase, run on the CUDA cores; "
+                                        "achieved counts the walk's own child dots over the whole phase"}
     elif dom == "stage1":
         roof = {"kernel": "stage1_kernel", "bound": "alu", "achieved": alg["internal_flops"] / t_dom / 1e12,
                 "peak": fma_peak, "unit": "TFLOP/s", "algorithmic_per_launch": alg["internal_flops"],
