@@ -865,8 +865,10 @@ def bench_decode(w, dev, stream, steps: int = 8, batch: int = 0, cache: int = 0)
     # compulsory bytes per step (per sequence and KV head): the scored levels'
     # child summaries (fp32), the raw keys of every level-1 candidate (scored or
     # forced), the attended values, the new q/k/v rows and the updated leaf
-    # and ancestor summaries. The kernel also reads the attended keys a second
-    # time (gathered bytes).
+    # and ancestor summaries. With one head per group and leaves of at most 64
+    # keys the kernel keeps the scoring pass's logits and streams only the
+    # attended values; otherwise it reads the attended keys a second time
+    # (gathered bytes).
     internal, leafkeys, attended = walk_counts(prefix + 8, w.C, w.K, w.forced_mask)
     tlast = prefix + 4
     G = w.Hq // w.Hkv
@@ -879,7 +881,8 @@ def bench_decode(w, dev, stream, steps: int = 8, batch: int = 0, cache: int = 0)
     per_unit = internal[tlast] * w.d * 4 + (leafkeys[tlast] + walk_counts.forced_keys[tlast]) * w.d * e + \
         attended[tlast] * w.d * e + (G + 2) * w.d * e + L * w.d * 4
     step_bytes = per_unit * B * w.Hkv
-    gathered = step_bytes + attended[tlast] * w.d * e * B * w.Hkv
+    rereads_keys = not (G == 1 and w.C <= 64)
+    gathered = step_bytes + (attended[tlast] * w.d * e * B * w.Hkv if rereads_keys else 0)
     pk = peaks()
     del Kc, Vc, pyr
     return {"batch": B, "cache_keys": prefix, "call": "pisa_decode_step", "us_per_step": fused,

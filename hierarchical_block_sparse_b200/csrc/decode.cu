@@ -131,7 +131,6 @@ __global__ void __launch_bounds__(128) append_kernel(T* __restrict__ Kc, T* __re
 // Tile rows keep their 16-byte chunks XOR-swizzled so that the 8 threads of a
 // shared-memory access phase hit distinct banks.
 constexpr int kDecStageBytes = 16384;
-constexpr int kDecStages = 3;
 
 template <typename T, int D>
 struct DecLayout {
@@ -193,6 +192,17 @@ __device__ __forceinline__ void lse_merge(float& m, float& s, float m2, float s2
 template <int G>
 constexpr int decode_min_blocks() { return G <= 2 ? 4 : (G <= 4 ? 2 : 1); }
 
+// With one head per group (G = 1) and leaves of at most kDecCacheKeys keys, the
+// scoring pass keeps every candidate key's logit in shared memory
+// ([32 leaves][kDecCacheKeys]), so the attention streams only the values of
+// the kept leaves; that variant runs a 2-stage pipeline to make room (still
+// 8 stages of 16 KB in flight per SM).
+constexpr int kDecCacheKeys = 64;
+template <int G>
+constexpr bool decode_caches() { return G == 1; }
+template <int G>
+constexpr int decode_stages() { return decode_caches<G>() ? 2 : 3; }
+
 template <typename T, int D, int G>
 __global__ void __launch_bounds__(256, decode_min_blocks<G>()) decode_kernel(
     const T* __restrict__ q_new, T* __restrict__ Kc, T* __restrict__ Vc, float* __restrict__ pyr,
@@ -200,6 +210,7 @@ __global__ void __launch_bounds__(256, decode_min_blocks<G>()) decode_kernel(
     const T* __restrict__ v_new, DecodeParams p) {
     using Lo = DecLayout<T, D>;
     constexpr int NW = 8;
+    constexpr int kDecStages = decode_stages<G>();
     constexpr int EPC = Lo::EPC, TPR = Lo::TPR, TPRC = Lo::TPRC, TPRW = Lo::TPRW;
     extern __shared__ __align__(16) uint8_t dsm[];  // pipeline stages, then [NW][G][D] partial outputs
     __shared__ __align__(16) float s_q[G][D];       // scaled queries of the group
@@ -220,6 +231,10 @@ __global__ void __launch_bounds__(256, decode_min_blocks<G>()) decode_kernel(
     Part& s_vn = *reinterpret_cast<Part*>(dsm + kDecStages * kDecStageBytes + 2 * sizeof(Part));
     Part& s_vmean = *reinterpret_cast<Part*>(dsm + kDecStages * kDecStageBytes + 3 * sizeof(Part));
     Part& s_vm2 = *reinterpret_cast<Part*>(dsm + kDecStages * kDecStageBytes + 4 * sizeof(Part));
+    // cached logits [32][kDecCacheKeys] (G = 1, C <= kDecCacheKeys), after the leaf states
+    float* s_logit = reinterpret_cast<float*>(dsm + kDecStages * kDecStageBytes + 5 * sizeof(Part));
+    const bool cached = decode_caches<G>() && p.C <= kDecCacheKeys;
+    __shared__ int s_kj[32];  // for each kept leaf, its index in the scored list
     const int64_t unit = blockIdx.x;  // b * Hkv + kvh
     const int64_t b = unit / p.Hkv;
     const int kvh = (int)(unit - b * p.Hkv);
@@ -413,6 +428,7 @@ __global__ void __launch_bounds__(256, decode_min_blocks<G>()) decode_kernel(
             for (int o = 1; o < TPR; o <<= 1)
 #pragma unroll
                 for (int h = 0; h < G; ++h) acc[h] += __shfl_xor_sync(kFull, acc[h], o);
+            if (cached && sl == 0 && r < nrows) s_logit[j * kDecCacheKeys + (tile % tpl) * Lo::RowsB + r] = acc[0];
             // this warp's rows: max and sum of 2^(z - max) per head, one lane per row counting
 #pragma unroll
             for (int h = 0; h < G; ++h) {
@@ -494,6 +510,8 @@ __global__ void __launch_bounds__(256, decode_min_blocks<G>()) decode_kernel(
         }
         const int out_id = lane < kept ? id : -1;
         if (lane < p.K) idx[unit * p.K + lane] = out_id;
+        if ((kmask >> lane) & 1u)  // kept candidate lane -> (its rank among the kept, among the scored)
+            s_kj[__popc(kmask & ((1u << lane) - 1u))] = __popc(s.vmask & ((1u << lane) - 1u));
         s_sel[lane] = lane < p.K ? out_id : -1;
         if (lane == 0) s_nlist = min(kept, p.K);
 #pragma unroll
@@ -538,7 +556,7 @@ __global__ void __launch_bounds__(256, decode_min_blocks<G>()) decode_kernel(
                 int64_t lo;
                 const int n = rows_of(tile, lo);
                 const uint32_t dst = stage0 + (tile % kDecStages) * kDecStageBytes;
-                stage_rows<T, D>(dst, Kh + lo * D, n, TPRC, tid);
+                if (!cached) stage_rows<T, D>(dst, Kh + lo * D, n, TPRC, tid);
                 stage_rows<T, D>(dst + kDecStageBytes / 2, Vh + lo * D, n, TPRC, tid);
             }
             tc::cp_async_commit();
@@ -557,7 +575,9 @@ __global__ void __launch_bounds__(256, decode_min_blocks<G>()) decode_kernel(
 #pragma unroll
             for (int h = 0; h < G; ++h) acc[h] = 0.f;
             const bool live = rc < nrows;
-            if (live) {
+            if (cached) {  // the logit from the scoring pass (every lane of the row reads it)
+                if (live) acc[0] = s_logit[s_kj[tile / tpl] * kDecCacheKeys + (tile % tpl) * Lo::RowsC + rc];
+            } else if (live) {
 #pragma unroll
                 for (int k = 0; k < 2; ++k) {
                     float x[EPC];
@@ -572,10 +592,12 @@ __global__ void __launch_bounds__(256, decode_min_blocks<G>()) decode_kernel(
                         }
                 }
             }
+            if (!cached) {
 #pragma unroll
-            for (int o2 = 1; o2 < TPRC; o2 <<= 1)
+                for (int o2 = 1; o2 < TPRC; o2 <<= 1)
 #pragma unroll
-                for (int h = 0; h < G; ++h) acc[h] += __shfl_xor_sync(kFull, acc[h], o2);
+                    for (int h = 0; h < G; ++h) acc[h] += __shfl_xor_sync(kFull, acc[h], o2);
+            }
             if (live) {
                 float pr[G];
 #pragma unroll
@@ -656,8 +678,9 @@ static cudaError_t launch_decode_t(const void* q, void* Kc, void* Vc, float* pyr
                                    void* o, const void* k_new, const void* v_new, const DecodeParams& p,
                                    cudaStream_t st) {
     const size_t out_bytes = sizeof(float) * 8 * G * (D + 1);
-    // pipeline stages + five per-warp arrays [32][8][G] of leaf states
-    const size_t stage_bytes = (size_t)kDecStages * kDecStageBytes + 5 * sizeof(float) * 32 * 8 * G;
+    // pipeline stages + five per-warp arrays [32][8][G] of leaf states (+ the cached logits)
+    const size_t stage_bytes = (size_t)decode_stages<G>() * kDecStageBytes + 5 * sizeof(float) * 32 * 8 * G +
+                               (decode_caches<G>() ? sizeof(float) * 32 * kDecCacheKeys : 0);
     const size_t smem = out_bytes > stage_bytes ? out_bytes : stage_bytes;
     auto kern = decode_kernel<T, D, G>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
