@@ -497,6 +497,8 @@ def main():
     ap.add_argument("--decode-batch", type=int, default=0, help="override the decode batch (profiling)")
     ap.add_argument("--decode-cache", type=int, default=0, help="override the cached keys per sequence")
     ap.add_argument("--decode-only", action="store_true", help="skip the prefill measurement (profiling)")
+    ap.add_argument("--seq", type=int, default=0,
+                    help="override the workload's sequence length (smaller cases for counter captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         print("warning: --warmup raised to 3", file=sys.stderr)
@@ -507,6 +509,8 @@ def main():
     from hierarchical_block_sparse_b200.workloads import WORKLOADS, make_inputs
 
     w = WORKLOADS[args.workload]
+    if args.seq:
+        w = w.replace(N=args.seq, name=f"{w.name}_seq{args.seq}")
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))

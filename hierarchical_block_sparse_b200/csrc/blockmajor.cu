@@ -582,11 +582,14 @@ __global__ void __launch_bounds__(128) leaf_score_kernel(const __nv_bfloat16* __
 // lower leaf: valid candidates arrive in ascending order, so the lane order is
 // the index order and the kept leaves come out sorted), writes idx and the
 // per-head partial normaliser z2[unit * G + h] = log2 sum 2^lse over the kept
-// leaves that are not forced (forced_tile_kernel adds the forced ones). The
-// slot-returning atomics that place each kept free leaf in its attention
-// bucket are issued for all of the warp's positions together, so their round
-// trips overlap.
+// leaves that are not forced (forced_tile_kernel adds the forced ones).
+// Each kept free leaf also gets its slot in the attention bucket of its leaf.
+// Consecutive positions keep many of the same leaves, so a CTA (8 warps, 32
+// positions) first counts its own entries per leaf in a shared-memory hash
+// table (local slots), then reserves each leaf's range with one global atomic
+// (its base), and an entry's slot is base + local slot.
 constexpr int kTopkQ = 4;
+constexpr int kTopkHash = 1024;  // > the at most 32 x 16 distinct leaves of a CTA
 
 template <int G>
 __global__ void __launch_bounds__(256) topk_kernel(const int32_t* __restrict__ cand, const float* __restrict__ lse,
@@ -594,11 +597,19 @@ __global__ void __launch_bounds__(256) topk_kernel(const int32_t* __restrict__ c
                                                    int32_t* __restrict__ idx, float* __restrict__ z2,
                                                    int32_t* __restrict__ counts, int32_t* __restrict__ slots,
                                                    int64_t M1, SelectParams p) {
+    __shared__ int s_key[kTopkHash], s_cnt[kTopkHash], s_base[kTopkHash];
+    for (int e = threadIdx.x; e < kTopkHash; e += blockDim.x) {
+        s_key[e] = -1;
+        s_cnt[e] = 0;
+    }
+    __syncthreads();
     const int lane = threadIdx.x & 31;
     const int t0 = (blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * kTopkQ;
-    if (t0 >= p.N) return;
     const int64_t bh = blockIdx.y;
     int out_leaf[kTopkQ];  // lane < K: the lane-th kept leaf that needs a bucket slot, else -1
+#pragma unroll
+    for (int i = 0; i < kTopkQ; ++i) out_leaf[i] = -1;
+    if (t0 < p.N) {  // (warps past the end still take part in the CTA's barriers)
     // all positions' candidates and LSEs are loaded first (independent requests in flight)
     int leaves[kTopkQ];
     float l2s[kTopkQ][G], rank_score[kTopkQ];
@@ -655,14 +666,34 @@ __global__ void __launch_bounds__(256) topk_kernel(const int32_t* __restrict__ c
         if (lane < p.K) idx[unit * p.K + lane] = v;
         if (lane < p.K && v >= 0 && !F.has(v, 1)) out_leaf[i] = v;
     }
-    // bucket count (and slot) of the attention grouping, by position in idx
-    int slot[kTopkQ];
+    }  // t0 < p.N
+    // bucket slots of the kept free leaves: local slots per leaf in the CTA's
+    // hash table, one global reservation per distinct leaf, slot = base + local
+    int hslot[kTopkQ], local[kTopkQ];
+#pragma unroll
+    for (int i = 0; i < kTopkQ; ++i) {
+        hslot[i] = -1;
+        local[i] = 0;
+        const int leaf = out_leaf[i];
+        if (leaf < 0) continue;
+        int h = (int)(((uint32_t)leaf * 2654435761u) >> 22);  // 10 bits
+        for (int probe = 0; probe < kTopkHash; ++probe) {
+            const int k = atomicCAS(&s_key[h], -1, leaf);
+            if (k == -1 || k == leaf) break;
+            h = (h + 1) & (kTopkHash - 1);
+        }
+        hslot[i] = h;
+        local[i] = atomicAdd(&s_cnt[h], 1);
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < kTopkHash; e += blockDim.x) {
+        const int leaf = s_key[e];
+        if (leaf >= 0) s_base[e] = atomicAdd(&counts[bh * M1 + leaf], s_cnt[e]);
+    }
+    __syncthreads();
 #pragma unroll
     for (int i = 0; i < kTopkQ; ++i)
-        slot[i] = out_leaf[i] >= 0 ? atomicAdd(&counts[bh * M1 + out_leaf[i]], 1) : 0;
-#pragma unroll
-    for (int i = 0; i < kTopkQ; ++i)
-        if (out_leaf[i] >= 0) slots[(bh * p.N + t0 + i) * kPairs + lane] = slot[i];
+        if (hslot[i] >= 0) slots[(bh * p.N + t0 + i) * kPairs + lane] = s_base[hslot[i]] + local[i];
 }
 
 // ------------------------------------------------------ attention tiles ----
