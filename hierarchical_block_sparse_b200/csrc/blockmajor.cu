@@ -708,11 +708,15 @@ __global__ void __launch_bounds__(128) attn_tile_kernel(const __nv_bfloat16* __r
                                                         const uint32_t* __restrict__ entries,
                                                         const float* __restrict__ z2, float* __restrict__ oacc,
                                                         int* __restrict__ err, TileParams p) {
+    // Shared memory (72 KB): gathered Q rows [0, 32K), later the probabilities P
+    // [0, 16K) and the staged output rows (two rounds of 64, [0, 33.8K)); the
+    // leaf's value block [40K, 56K) and key block [56K, 72K) outlive a tile, so
+    // a run of consecutive tiles of one bucket loads them once.
     extern __shared__ __align__(1024) uint8_t dsm[];
     uint8_t* sA = dsm;                 // 32 KB gathered Q rows
-    uint8_t* sK = dsm + 32768;         // 16 KB key block
-    uint8_t* sV = dsm + 49152;         // 16 KB value block (MN-major)
-    uint8_t* sP = sK;                  // 16 KB probabilities (K-major), over the keys once S has landed
+    uint8_t* sP = dsm;                 // 16 KB probabilities (K-major), over Q once S has landed
+    uint8_t* sV = dsm + 40960;         // 16 KB value block (MN-major)
+    uint8_t* sK = dsm + 57344;         // 16 KB key block
     __shared__ TileRows tr;
     __shared__ __align__(8) uint64_t mbar;
     __shared__ uint32_t tmem_base;
@@ -731,9 +735,13 @@ __global__ void __launch_bounds__(128) attn_tile_kernel(const __nv_bfloat16* __r
     const uint32_t a_smem = tc::smem_u32(sA), k_smem = tc::smem_u32(sK), v_smem = tc::smem_u32(sV),
                    p_smem = tc::smem_u32(sP);
     const int ntiles = min(*ntiles_ptr, p.max_tiles);
+    // runs of kRun consecutive tiles (mostly one bucket: one leaf) per CTA
+    constexpr int kRun = 8;
+    auto tile_of = [&](int it) { return ((it / kRun) * (int)gridDim.x + (int)blockIdx.x) * kRun + it % kRun; };
+    int2 kv_loaded = make_int2(-1, -1);  // (b * Hkv + kvh, leaf) of the blocks in sK / sV
     uint32_t phase = 0;
     bool ok;
-    for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+    for (int it = 0, tile = tile_of(0); tile < ntiles; tile = tile_of(++it)) {
         const int4 td = tiles[tile];
         const int64_t bh = td.x, leaf = td.y;
         const int64_t b = bh / p.Hkv;
@@ -745,8 +753,11 @@ __global__ void __launch_bounds__(128) attn_tile_kernel(const __nv_bfloat16* __r
         tile_rows<G>(tr, entries, td.z, td.w, p.N, err, tid);
         __syncthreads();
         gather_q<G>(a_smem, tr, Q, b, kvh, p.Hq, p.N, tid);
-        load_kblock(k_smem, Kmat + bh * p.N * kD, leaf * kBlk, p.N, tid);
-        load_vblock(v_smem, Vmat + bh * p.N * kD, leaf * kBlk, p.N, tid);
+        if (kv_loaded.x != td.x || kv_loaded.y != td.y) {
+            load_kblock(k_smem, Kmat + bh * p.N * kD, leaf * kBlk, p.N, tid);
+            load_vblock(v_smem, Vmat + bh * p.N * kD, leaf * kBlk, p.N, tid);
+            kv_loaded = make_int2(td.x, td.y);
+        }
         tc::cp_async_commit();
         tc::cp_async_wait_all();
         tc::fence_async_smem();
@@ -760,7 +771,7 @@ __global__ void __launch_bounds__(128) attn_tile_kernel(const __nv_bfloat16* __r
         phase ^= 1;
         if (!ok) break;
         tc::tc_fence_after();
-        // P = 2^(S*scale - z), masked, packed to bf16 in the K-major P tile
+        // P = 2^(S*scale - z), masked, packed to bf16 in the K-major P tile (over the Q rows, which the MMA has read)
         {
             float v[64];
             const uint32_t taddr = tmem_s + ((uint32_t)(warp * 32) << 16);
@@ -805,32 +816,39 @@ __global__ void __launch_bounds__(128) attn_tile_kernel(const __nv_bfloat16* __r
         if (!ok) break;
         tc::tc_fence_after();
         {
-            // Row tid of the output tile is staged in shared memory (the tile's
-            // buffers are free once the PV product has landed) and added to the
-            // accumulator with one 512-byte bulk reduction: whole-line
-            // operations at L2 instead of 32 scattered 16-byte ones.
+            // Each output row is staged in shared memory (over Q and P, both
+            // read by now) and added to the accumulator with one 512-byte bulk
+            // reduction: whole-line operations at L2 instead of 32 scattered
+            // 16-byte ones. Two rounds of 64 rows leave the K and V blocks intact.
             const int t = tr.t[tid];
             const uint32_t taddr = tmem_o + ((uint32_t)(warp * 32) << 16);
-            uint8_t* srow = dsm + tid * kORowStride;
 #pragma unroll
-            for (int part = 0; part < 4; ++part) {
-                float v[32];
-                tc::tmem_ld32(taddr + part * 32, v);
-                tc::tmem_ld_wait();
+            for (int round = 0; round < 2; ++round) {
+                const bool mine = (tid >> 6) == round;
+                uint8_t* srow = dsm + (tid & 63) * kORowStride;
+                if (mine) {
 #pragma unroll
-                for (int q = 0; q < 32; q += 4)
-                    *reinterpret_cast<float4*>(srow + (part * 32 + q) * 4) = make_float4(v[q], v[q + 1], v[q + 2], v[q + 3]);
-            }
-            if (t >= 0) {
-                tc::fence_async_smem();
-                tc::bulk_reduce_add_f32(oacc + (((b * p.Hq + (int64_t)kvh * G + (tid % G)) * p.N) + t) * kD,
-                                        tc::smem_u32(srow), kD * 4);
-                tc::bulk_commit();
+                    for (int part = 0; part < 4; ++part) {
+                        float v[32];
+                        tc::tmem_ld32(taddr + part * 32, v);
+                        tc::tmem_ld_wait();
+#pragma unroll
+                        for (int q = 0; q < 32; q += 4)
+                            *reinterpret_cast<float4*>(srow + (part * 32 + q) * 4) =
+                                make_float4(v[q], v[q + 1], v[q + 2], v[q + 3]);
+                    }
+                    if (t >= 0) {
+                        tc::fence_async_smem();
+                        tc::bulk_reduce_add_f32(oacc + (((b * p.Hq + (int64_t)kvh * G + (tid % G)) * p.N) + t) * kD,
+                                                tc::smem_u32(srow), kD * 4);
+                        tc::bulk_commit();
+                    }
+                }
+                tc::bulk_wait_read_all();  // the staged rows have been read: the buffer may be refilled
+                __syncthreads();
             }
         }
         tc::tc_fence_before();
-        tc::bulk_wait_read_all();  // the staged row has been read: the buffers may be refilled
-        __syncthreads();
     }
     tc::bulk_wait_all();
     __syncthreads();
@@ -1811,10 +1829,12 @@ static int sm_count() {
     return n;
 }
 
-// Q 32 KB + K (then P) 16 KB + V 16 KB, rounded up so that the staged output
-// tile fits: three CTAs per SM
+// attention tiles: Q (then P, then two rounds of 64 staged output rows) 33.8 KB,
+// V 16 KB at 40 KB, K 16 KB at 56 KB: three CTAs per SM. The forced tiles stage
+// all 128 rows at once over their Q, K and V buffers.
 constexpr size_t kAttnSmem = 72 * 1024;
-static_assert(128 * kORowStride <= kAttnSmem, "the staged output tile fits in the attention tile's buffers");
+static_assert(64 * kORowStride <= 40960, "half the staged output tile fits below the value block");
+static_assert(128 * kORowStride <= kAttnSmem, "the staged output tile fits in the forced tile's buffers");
 constexpr int kAttnCtasPerSm = 3;
 
 template <int G, bool PAIR, bool VSCORE>
