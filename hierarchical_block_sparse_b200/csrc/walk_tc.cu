@@ -100,19 +100,22 @@ __device__ __forceinline__ uint32_t idesc_n(int n) {  // kind::f16, bf16 x bf16 
     return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
 }
 
-// One position's candidates at level l are held by two adjacent lanes: lane
-// half h owns slots 16 h .. 16 h + 15, the children of its kept nodes 8 h ..
-// 8 h + 7 one level up (the root alone in slot 0 at l = L), so the slots
-// ascend with the node index. Bit i of v: slot 16 h + i exists and is
-// eligible (causal: its first key is not after t); of f: it is on a forced
-// path (close reading §5.3).
-struct HalfCands {
-    int node[16];
+// One position's candidates at level l are held by LPP = 2G adjacent lanes
+// (all 256 threads serve the tile's 128/G positions): lane q of the group owns
+// the SPL = 16/G slots q*SPL .. q*SPL + SPL - 1, slot c being child c & 1 of
+// the position's (c >> 1)-th kept node one level up (the root alone in slot 0
+// at l = L), so the slots ascend with the node index. Bit i of v: slot
+// q*SPL + i exists and is eligible (causal: its first key is not after t); of
+// f: it is on a forced path (close reading §5.3).
+template <int SPL>
+struct LaneCands {
+    int node[SPL];
     uint32_t v, f;
 };
 
-__device__ __forceinline__ void half_cands(const TwSmem& S, int pos, int l, int L, int64_t t, const SelectParams& p,
-                                           int h, bool live, HalfCands& hc) {
+template <int SPL>
+__device__ __forceinline__ void lane_cands(const TwSmem& S, int pos, int l, int L, int64_t t, const SelectParams& p,
+                                           int q, bool live, LaneCands<SPL>& lc) {
     // node i of level l exists and is eligible iff 0 <= i <= vmax (M_l = ceil(N / span))
     const int64_t span = (int64_t)p.C << (l - 1);
     const int64_t lastn = p.geom.M[l] - 1;
@@ -122,38 +125,53 @@ __device__ __forceinline__ void half_cands(const TwSmem& S, int pos, int l, int 
     const int s = l - 1;
     const int fa = F.f0 >= 0 ? F.f0 >> s : -2, fb = F.f1 >= 0 ? F.f1 >> s : -2, fc = F.f2 >= 0 ? F.f2 >> s : -2;
     const int nk = (!live || l == L) ? 0 : S.nkept[pos];
-    hc.v = hc.f = 0u;
+    lc.v = lc.f = 0u;
+    if constexpr (SPL >= 2) {  // parents q * SPL / 2 .. + SPL / 2 - 1, two slots each
 #pragma unroll
-    for (int jj = 0; jj < 8; ++jj) {
-        const int j = 8 * h + jj;
-        const int par = !live ? -1 : l == L ? (j == 0 ? 0 : -1) : (j < nk ? S.kept[pos][j] : -1);
+        for (int jj = 0; jj < SPL / 2; ++jj) {
+            const int j = q * (SPL / 2) + jj;
+            const int par = !live ? -1 : l == L ? (j == 0 ? 0 : -1) : (j < nk ? S.kept[pos][j] : -1);
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-            const int i = 2 * jj + e;
-            const int node = l == L ? (par == 0 && e == 0 ? 0 : -1) : (par >= 0 ? 2 * par + e : -1);
-            hc.node[i] = node;
-            const bool valid = (unsigned)node <= (unsigned)vmax;
-            hc.v |= (valid ? 1u : 0u) << i;
-            hc.f |= (valid && (node == fa || node == fb || node == fc) ? 1u : 0u) << i;
+            for (int e = 0; e < 2; ++e) {
+                const int i = 2 * jj + e;
+                const int node = l == L ? (par == 0 && e == 0 ? 0 : -1) : (par >= 0 ? 2 * par + e : -1);
+                lc.node[i] = node;
+                const bool valid = (unsigned)node <= (unsigned)vmax;
+                lc.v |= (valid ? 1u : 0u) << i;
+                lc.f |= (valid && (node == fa || node == fb || node == fc) ? 1u : 0u) << i;
+            }
         }
+    } else {  // one slot: child q & 1 of parent q >> 1
+        const int j = q >> 1, e = q & 1;
+        const int par = !live ? -1 : l == L ? (j == 0 ? 0 : -1) : (j < nk ? S.kept[pos][j] : -1);
+        const int node = l == L ? (par == 0 && e == 0 ? 0 : -1) : (par >= 0 ? 2 * par + e : -1);
+        lc.node[0] = node;
+        const bool valid = (unsigned)node <= (unsigned)vmax;
+        lc.v = valid ? 1u : 0u;
+        lc.f = valid && (node == fa || node == fb || node == fc) ? 1u : 0u;
     }
 }
 
-// the 32-slot mask of a position from its two lanes' 16-slot halves
-__device__ __forceinline__ uint32_t pair_mask(uint32_t m16, int h) {
-    const uint32_t o = __shfl_xor_sync(kFull, m16, 1);
-    return h == 0 ? (m16 | (o << 16)) : (o | (m16 << 16));
+// the 32-slot mask of a position from its lanes' SPL-slot parts
+template <int SPL>
+__device__ __forceinline__ uint32_t group_mask(uint32_t m, int q) {
+    constexpr int LPP = kSlots / SPL;
+    uint32_t full = m << (q * SPL);
+#pragma unroll
+    for (int o = 1; o < LPP; o <<= 1) full |= __shfl_xor_sync(kFull, full, o);
+    return full;
 }
 
 // the kept candidates (bit c of `keep`) in slot order, i.e. ascending node
-// order; each lane writes its own half
-__device__ __forceinline__ void write_kept(TwSmem& S, int pos, const HalfCands& hc, uint32_t keep, int h) {
-    int n = h == 0 ? 0 : __popc(keep & 0xffffu);
-    const uint32_t mine = (keep >> (16 * h)) & 0xffffu;
+// order; each lane writes its own slots
+template <int SPL>
+__device__ __forceinline__ void write_kept(TwSmem& S, int pos, const LaneCands<SPL>& lc, uint32_t keep, int q) {
+    int n = __popc(keep & ((1u << (q * SPL)) - 1u));
+    const uint32_t mine = (keep >> (q * SPL)) & (SPL == 32 ? 0xffffffffu : ((1u << SPL) - 1u));
 #pragma unroll
-    for (int i = 0; i < 16; ++i)
-        if ((mine >> i) & 1u) S.kept[pos][n++] = hc.node[i];
-    if (h == 0) S.nkept[pos] = __popc(keep);
+    for (int i = 0; i < SPL; ++i)
+        if ((mine >> i) & 1u) S.kept[pos][n++] = lc.node[i];
+    if (q == 0) S.nkept[pos] = __popc(keep);
 }
 
 // the lowest k set bits of m
@@ -176,60 +194,61 @@ __device__ __forceinline__ uint32_t ordered(float x) {
 // The keep rule of a ranked level (close reading §04 4.2; Eq.(6)): forced
 // candidates first, then the best scores, ties to the lower node (= lower
 // slot). Keys are the scores mapped order-preservingly onto uint32 (forced:
-// the maximum, not eligible: 0). The two lanes of a position sort their 16
-// keys in opposite directions (a bitonic sequence of 32), exchange once, and
-// lane half 0 ends with the 16 largest, descending, so the K-th largest key
-// tau is known; the kept set is every key above tau and, of the keys equal to
-// tau, the lowest slots that fill K. Returns the 32-slot keep mask on both lanes.
+// the maximum, not eligible: 0). A bitonic network sorts the 32 keys of a
+// position descending, element e = q*SPL + i held by lane q of its group:
+// compare-exchanges with partners less than SPL apart are in registers, the
+// others exchange with lane q ^ (j / SPL). The K-th largest key tau is then
+// known; the kept set is every key above tau and, of the keys equal to tau,
+// the lowest slots that fill K. Returns the 32-slot keep mask on every lane.
+template <int SPL>
 __device__ __forceinline__ uint32_t rank_keep(const float* score, int stride, uint32_t vfull, uint32_t ffull,
-                                              int K, int h) {
-    const uint32_t vm = (vfull >> (16 * h)) & 0xffffu, fm = (ffull >> (16 * h)) & 0xffffu;
-    uint32_t a[16];
+                                              int K, int q) {
+    constexpr uint32_t kMaskSpl = SPL == 32 ? 0xffffffffu : ((1u << SPL) - 1u);
+    const uint32_t vm = (vfull >> (q * SPL)) & kMaskSpl, fm = (ffull >> (q * SPL)) & kMaskSpl;
+    uint32_t a[SPL];
 #pragma unroll
-    for (int i = 0; i < 16; ++i)
+    for (int i = 0; i < SPL; ++i)
         a[i] = !((vm >> i) & 1u) ? 0u : ((fm >> i) & 1u) ? 0xffffffffu : ordered(score[i * stride]);
 #pragma unroll
-    for (int k = 2; k <= 16; k <<= 1)
+    for (int k = 2; k <= kSlots; k <<= 1)
 #pragma unroll
-        for (int j = k >> 1; j > 0; j >>= 1)
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            if (j < SPL) {
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const int m = i ^ j;
-                if (m > i) {
-                    const bool desc = k == 16 ? h == 0 : (i & k) == 0;
-                    const uint32_t x = a[i], y = a[m];
-                    a[i] = desc ? max(x, y) : min(x, y);
-                    a[m] = desc ? min(x, y) : max(x, y);
+                for (int i = 0; i < SPL; ++i) {
+                    const int m = i ^ j;
+                    if (m > i) {
+                        // (q * SPL + i) & k: the lane's part is a multiple of SPL
+                        const bool desc = k < SPL ? (i & k) == 0 : ((q * SPL) & k) == 0;
+                        const uint32_t x = a[i], y = a[m];
+                        a[i] = desc ? max(x, y) : min(x, y);
+                        a[m] = desc ? min(x, y) : max(x, y);
+                    }
+                }
+            } else {
+                const int lo_lane = (q & (j / SPL)) == 0;  // this lane holds the lower elements of its pairs
+#pragma unroll
+                for (int i = 0; i < SPL; ++i) {
+                    const uint32_t o = __shfl_xor_sync(kFull, a[i], j / SPL);
+                    const bool desc = k < SPL ? (i & k) == 0 : ((q * SPL) & k) == 0;
+                    a[i] = (desc == (lo_lane != 0)) ? max(a[i], o) : min(a[i], o);
                 }
             }
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {  // the cross-lane step of the 32-key merge
-        const uint32_t o = __shfl_xor_sync(kFull, a[i], 1);
-        a[i] = h == 0 ? max(a[i], o) : min(a[i], o);
-    }
-#pragma unroll
-    for (int j = 8; j > 0; j >>= 1)
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const int m = i ^ j;
-            if (m > i) {
-                const uint32_t x = a[i], y = a[m];
-                a[i] = max(x, y);
-                a[m] = min(x, y);
-            }
         }
-    uint32_t tau = 0u;  // a[K - 1], picked with masks (an indexed read would put a[] in local memory)
+    // element K - 1: lane (K - 1) / SPL of the group, register (K - 1) % SPL
+    uint32_t tau = 0u;  // picked with masks (an indexed read would put a[] in local memory)
 #pragma unroll
-    for (int i = 0; i < 16; ++i) tau |= a[i] & (0u - (uint32_t)(i == K - 1));
-    tau = __shfl_sync(kFull, tau, (threadIdx.x & 31) & ~1);
+    for (int i = 0; i < SPL; ++i) tau |= a[i] & (0u - (uint32_t)(i == (K - 1) % SPL));
+    constexpr int LPP = kSlots / SPL;
+    tau = __shfl_sync(kFull, tau, ((threadIdx.x & 31) & ~(LPP - 1)) + (K - 1) / SPL);
     uint32_t gt = 0u, eq = 0u;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
+    for (int i = 0; i < SPL; ++i) {
         const uint32_t k = !((vm >> i) & 1u) ? 0u : ((fm >> i) & 1u) ? 0xffffffffu : ordered(score[i * stride]);
         gt |= (k > tau ? 1u : 0u) << i;
         eq |= (k == tau ? 1u : 0u) << i;
     }
-    const uint32_t gt_full = pair_mask(gt, h), eq_full = pair_mask(eq, h);
+    const uint32_t gt_full = group_mask<SPL>(gt, q), eq_full = group_mask<SPL>(eq, q);
     return (gt_full | lowest_bits(eq_full, K - __popc(gt_full))) & vfull;
 }
 
@@ -239,7 +258,9 @@ __global__ void __launch_bounds__(kTwThreads, 1) walk_tc_kernel(
     const __nv_bfloat16* __restrict__ pyr_lo, int32_t* __restrict__ cand_out, int32_t* __restrict__ resume,
     int32_t* __restrict__ counts, int32_t* __restrict__ slots, int tiles_per_head, int* __restrict__ err,
     SelectParams p) {
-    constexpr int P = 128 / G;  // positions per tile
+    constexpr int P = 128 / G;       // positions per tile
+    constexpr int LPP = 2 * G;       // lanes per position in the per-position phases (LPP * P = 256)
+    constexpr int SPL = kSlots / LPP;  // candidate slots per lane
     extern __shared__ __align__(1024) uint8_t dsm[];
     TwSmem& S = *reinterpret_cast<TwSmem*>(dsm);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -314,27 +335,27 @@ __global__ void __launch_bounds__(kTwThreads, 1) walk_tc_kernel(
         for (int i = tid; i < words; i += kTwThreads) S.bits[i] = 0u;
         __syncthreads();
         int any = 0;
-        if (warp * 32 < 2 * P) {  // two lanes per position
-            const int pos = tid >> 1, h = tid & 1;
-            const bool live = pos < P && t0 + pos < p.N;
+        {  // LPP lanes per position
+            const int pos = tid / LPP, q = tid % LPP;
+            const bool live = t0 + pos < p.N;
             const int64_t t = live ? t0 + pos : 0;
-            HalfCands hc;
-            half_cands(S, pos, l, L, t, p, h, live, hc);
-            const uint32_t vfull = pair_mask(hc.v, h), ffull = pair_mask(hc.f, h);
+            LaneCands<SPL> lc;
+            lane_cands<SPL>(S, pos, l, L, t, p, q, live, lc);
+            const uint32_t vfull = group_mask<SPL>(lc.v, q), ffull = group_mask<SPL>(lc.f, q);
             const int n = __popc(vfull), nf = __popc(ffull);
             const bool rank = live && n > p.K && nf < p.K;
             const int nk = live && l < L ? S.nkept[pos] : 0;
-            __syncwarp();  // both lanes have read the kept nodes they expand
+            __syncwarp();  // the group's lanes have read the kept nodes they expand
             if (live && !rank)  // all of them, or the forced ones fill the budget: no scores needed
-                write_kept(S, pos, hc, n <= p.K ? vfull : lowest_bits(ffull, p.K), h);
+                write_kept<SPL>(S, pos, lc, n <= p.K ? vfull : lowest_bits(ffull, p.K), q);
             if (rank) {  // flag the parents whose grandchildren are needed
-                for (int j = 8 * h; j < min(nk, 8 * h + 8); ++j) {
+                for (int j = q * SPL / 2; j < min(nk, (q + 1) * SPL / 2); ++j) {
                     const int par = S.kept[pos][j];
                     if (par >= 0 && par < wnodes) atomicOr(&S.bits[par >> 5], 1u << (par & 31));
                     else if (err) atomicCAS(err, 0, 16);  // self-check: a kept node past the tile's reach
                 }
             }
-            if (pos < P && h == 0) S.need[pos] = rank ? 1 : 0;
+            if (q == 0) S.need[pos] = rank ? 1 : 0;
             any = rank ? 1 : 0;
         }
         if (!__syncthreads_or(any)) continue;
@@ -353,10 +374,10 @@ __global__ void __launch_bounds__(kTwThreads, 1) walk_tc_kernel(
             }
         }
         __syncthreads();
-        if ((tid >> 1) < P && S.need[tid >> 1]) {
-            const int pos = tid >> 1, h = tid & 1;
+        if (S.need[tid / LPP]) {
+            const int pos = tid / LPP, q = tid % LPP;
             const int nk = S.nkept[pos];
-            for (int j = 8 * h; j < min(nk, 8 * h + 8); ++j) {
+            for (int j = q * SPL / 2; j < min(nk, (q + 1) * SPL / 2); ++j) {
                 const int par = S.kept[pos][j];
                 const uint32_t below = S.bits[par >> 5] & ((1u << (par & 31)) - 1u);
                 S.keptu[pos][j] = S.pre[par >> 5] + __popc(below);
@@ -473,26 +494,26 @@ __global__ void __launch_bounds__(kTwThreads, 1) walk_tc_kernel(
         __syncthreads();
         if (!ok) break;
 
-        // ---- two lanes per ranking position: forced first, then the best by score (lower index on ties)
-        if (warp * 32 < 2 * P) {
-            const int pos = tid >> 1, h = tid & 1;
-            const bool live = pos < P && S.need[pos];
-            HalfCands hc;
-            half_cands(S, pos, l, L, live ? t0 + pos : 0, p, h, live, hc);
-            const uint32_t vfull = pair_mask(hc.v, h), ffull = pair_mask(hc.f, h);
-            float* sc = S.score + pos * (kSlots * G + 1) + 16 * h * G;
+        // ---- LPP lanes per ranking position: forced first, then the best by score (lower index on ties)
+        {
+            const int pos = tid / LPP, q = tid % LPP;
+            const bool live = S.need[pos] != 0;
+            LaneCands<SPL> lc;
+            lane_cands<SPL>(S, pos, l, L, live ? t0 + pos : 0, p, q, live, lc);
+            const uint32_t vfull = group_mask<SPL>(lc.v, q), ffull = group_mask<SPL>(lc.f, q);
+            float* sc = S.score + pos * (kSlots * G + 1) + q * SPL * G;
             if (G > 1 && live) {  // Eq.(11): summed over the group, into the first head's entry
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
+                for (int i = 0; i < SPL; ++i) {
                     float x = 0.f;
 #pragma unroll
                     for (int hh = 0; hh < G; ++hh) x += sc[i * G + hh];
                     sc[i * G] = x;
                 }
             }
-            const uint32_t keep = rank_keep(sc, G, vfull, ffull, p.K, h);
-            __syncwarp();  // both lanes have read the kept nodes they expand
-            if (live) write_kept(S, pos, hc, keep, h);
+            const uint32_t keep = rank_keep<SPL>(sc, G, vfull, ffull, p.K, q);
+            __syncwarp();  // the group's lanes have read the kept nodes they expand
+            if (live) write_kept<SPL>(S, pos, lc, keep, q);
         }
         __syncthreads();
     }
@@ -500,49 +521,54 @@ __global__ void __launch_bounds__(kTwThreads, 1) walk_tc_kernel(
     if (ok && lstop == 1) {
         // ---- every level done: the level-1 candidates and the sibling-pair
         // bucket counts, as the one-warp walk writes them
-        if (warp * 32 < 2 * P) {
-            const int pos = tid >> 1, h = tid & 1;
-            const bool live = pos < P && t0 + pos < p.N;
-            const int64_t t = live ? t0 + pos : 0;
-            const int64_t M1 = p.geom.M[1];
-            HalfCands hc;
-            half_cands(S, pos, 1, L, t, p, h, live, hc);
-            if (live) {
-                const int64_t unit = bh * p.N + t;
-                int last = -1;
+        const int pos = tid / LPP, q = tid % LPP;
+        const bool live = t0 + pos < p.N;
+        const int64_t t = live ? t0 + pos : 0;
+        const int64_t M1 = p.geom.M[1];
+        LaneCands<SPL> lc;
+        lane_cands<SPL>(S, pos, 1, L, t, p, q, live, lc);
+        uint32_t okm = 0u;  // slots holding a candidate (valid, in range)
+        int last = -1;
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const bool valid = (hc.v >> i) & 1u;
-                    const int cand = hc.node[i];
-                    const bool in_range = cand >= 0 && cand < M1;
-                    if (valid && !in_range && err) atomicCAS(err, 0, 10);  // self-check: never expected
-                    if (valid && last >= 0 && last >= cand && err) atomicCAS(err, 0, 14);  // slots ascend
-                    if (valid) last = cand;
-                    hc.node[i] = valid && in_range ? cand : -1;
-                    cand_out[unit * kSlots + 16 * h + i] = hc.node[i];
-                }
+        for (int i = 0; i < SPL; ++i) {
+            const bool valid = (lc.v >> i) & 1u;
+            const int cand = lc.node[i];
+            const bool in_range = cand >= 0 && cand < M1;
+            if (live && valid && !in_range && err) atomicCAS(err, 0, 10);  // self-check: never expected
+            if (live && valid && last >= 0 && last >= cand && err) atomicCAS(err, 0, 14);  // slots ascend
+            if (valid) last = cand;
+            okm |= (valid && in_range ? 1u : 0u) << i;
+        }
+        const uint32_t ok_full = group_mask<SPL>(okm, q);
+        const uint32_t free_full = ok_full & ~group_mask<SPL>(lc.f, q);
+        // a sibling pair (slots 2i, 2i + 1) whose first slot holds a candidate and
+        // has at least one leaf that is not forced counts once in its bucket
+        int pnode[SPL];  // the even slots' nodes (odd slots' lanes leave them unused)
 #pragma unroll
-                for (int i = 0; i < 16; i += 2) {  // a sibling pair with at least one leaf that is not forced
-                    const int c0 = hc.node[i], c1 = hc.node[i + 1];
-                    const bool free0 = c0 >= 0 && !((hc.f >> i) & 1u);
-                    const bool free1 = c1 >= 0 && !((hc.f >> (i + 1)) & 1u);
-                    if (c0 >= 0 && (free0 || free1))
-                        slots[unit * kPairs + 8 * h + i / 2] = atomicAdd(&counts[bh * ((M1 + 1) / 2) + (c0 >> 1)], 1);
-                }
-                if (h == 0) resume[unit] = 0;
+        for (int i = 0; i < SPL; ++i) pnode[i] = ((okm >> i) & 1u) ? lc.node[i] : -1;
+        if (live) {
+            const int64_t unit = bh * p.N + t;
+#pragma unroll
+            for (int i = 0; i < SPL; ++i) cand_out[unit * kSlots + q * SPL + i] = pnode[i];
+#pragma unroll
+            for (int i = 0; i < SPL; ++i) {
+                const int c = q * SPL + i;
+                if ((c & 1) == 0 && ((ok_full >> c) & 1u) && ((free_full >> c) & 3u))
+                    slots[unit * kPairs + c / 2] = atomicAdd(&counts[bh * ((M1 + 1) / 2) + (pnode[i] >> 1)], 1);
             }
+            if (q == 0) resume[unit] = 0;
         }
     } else if (ok) {
         // ---- hand each position's walk over to the one-warp walk: its kept
         // nodes one level above the level it resumes at
-        const int pos = tid >> 1, h = tid & 1;
-        if (pos < P && t0 + pos < p.N) {
+        const int pos = tid / LPP, q = tid % LPP;
+        if (t0 + pos < p.N) {
             const int64_t unit = bh * p.N + t0 + pos;
             // positions that ranked at the level handed over still hold that level's parents
             const int level = S.need[pos] ? lstop : lstop - 1;
             const int nk = S.nkept[pos];
-            for (int j = 8 * h; j < min(nk, 8 * h + 8); ++j) cand_out[unit * kSlots + j] = S.kept[pos][j];
-            if (h == 0) resume[unit] = (level << 8) | nk;
+            for (int j = q * SPL / 2; j < min(nk, (q + 1) * SPL / 2); ++j) cand_out[unit * kSlots + j] = S.kept[pos][j];
+            if (q == 0) resume[unit] = (level << 8) | nk;
         }
     }
     tc::cp_async_wait_all();
