@@ -11,11 +11,14 @@
 // heads (lanes of one position are adjacent, so the sum is a butterfly of
 // shuffles). The forced leaves (first, previous, current) count against K and
 // are kept; the other eligible leaves compete for the rest by score, ties to
-// the lower leaf. Every row keeps a sorted top list in registers and inserts
-// only what beats its current K-th key; warps 0-3 take the first 64 columns of
-// each chunk and warps 4-7 the last 64, and one warp per position merges the
-// two lists at the end. Output rows are sorted ascending, -1 padded, as from
-// the per-query kernel (bsa.cu).
+// the lower leaf. Every row keeps its best keys in a sorted list in registers
+// (the list's top slots hold +inf placeholders for the forced leaves, so the
+// entry to beat is always the last slot); a 32-column slice of scores marks
+// the columns that beat it, and the lanes insert their marked columns in
+// lockstep, a branch-free shift per insertion. Warps 0-3 take the first 64
+// columns of each chunk and warps 4-7 the last 64, and one warp per position
+// merges the two lists at the end. Output rows are sorted ascending, -1
+// padded, as from the per-query kernel (bsa.cu).
 #include <cmath>
 
 #include "pisa_internal.h"
@@ -29,16 +32,37 @@ constexpr int kBtThreads = 256;
 constexpr int kBtCols = 128;  // leaves per chunk
 constexpr int kD = 128;
 constexpr int kTop = 16;      // K <= 16
+constexpr int kTopPad = 17;   // stride of the lists handed to the merge
+constexpr int kZPad = 33;     // stride of a lane's staged scores: a column's 32 lanes hit 32 banks
 constexpr int kNone = 0x7fffffff;
 
 struct BtSmem {
     uint8_t q[32768];              // A: 128 rows x 128 bf16, K-major
-    uint8_t b[2][2][32768];        // B[buffer][hi, lo]: 128 leaf rows x 128 bf16
-    float key[2][128][kTop];       // per warpgroup and position: its best keys, descending
-    int32_t id[2][128][kTop];
+    uint8_t b[2][2][32768];        // B[buffer][hi, lo]: 128 leaf rows x 128 bf16; after the
+                                   // scan, each warpgroup's lists (BtLists)
+    float zs[8][32][kZPad];        // per warp and lane: one slice of scores, for the insertions
     uint64_t mbar[2];
     uint32_t tmem_base;
 };
+struct BtLists {
+    float key[2][128][kTopPad];    // per warpgroup and position: its best keys, descending
+    int32_t id[2][128][kTopPad];
+};
+static_assert(sizeof(BtLists) <= sizeof(BtSmem::b), "the lists fit in the tile buffers");
+
+// z into a descending list (ties: the earlier entry stays first), no branches
+__device__ __forceinline__ void top_insert(float (&k)[kTop], int (&id)[kTop], float z, int leaf) {
+    bool c[kTop];
+#pragma unroll
+    for (int i = 0; i < kTop; ++i) c[i] = z > k[i];
+#pragma unroll
+    for (int i = kTop - 1; i > 0; --i) {
+        k[i] = c[i - 1] ? k[i - 1] : (c[i] ? z : k[i]);
+        id[i] = c[i - 1] ? id[i - 1] : (c[i] ? leaf : id[i]);
+    }
+    k[0] = c[0] ? z : k[0];
+    id[0] = c[0] ? leaf : id[0];
+}
 
 __device__ __forceinline__ uint32_t idesc_n(int n) {  // kind::f16, bf16 x bf16 -> fp32, both K-major, M = 128
     return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
@@ -120,30 +144,25 @@ __global__ void __launch_bounds__(kBtThreads, 1) bsa_tc_kernel(const __nv_bfloat
         }
     }
     const int Kp = p.K - nf;  // places for the ranked leaves
-    // this row's best keys so far, descending (ties: the lower leaf first), in
-    // shared memory: an insertion is rare, and a list in registers would be
-    // indexed by a runtime position
-    float* lk = S.key[wg][pos];
-    int32_t* li = S.id[wg][pos];
-    if (live) {
+    // this row's list: kTop - Kp placeholders (+inf, never displaced), then
+    // Kp places for the ranked leaves; the entry to beat is k[kTop - 1]
+    float lk[kTop];
+    int li[kTop];
 #pragma unroll
-        for (int i = 0; i < kTop; ++i) {
-            lk[i] = -INFINITY;
-            li[i] = kNone;
-        }
+    for (int i = 0; i < kTop; ++i) {
+        lk[i] = i < kTop - Kp ? INFINITY : -INFINITY;
+        li[i] = kNone;
     }
-    float thr = Kp > 0 ? -INFINITY : INFINITY;  // the Kp-th best key so far
 
     uint32_t parity[2] = {0u, 0u};
     bool ok = true;
-    gather(0, 0);
-    for (int k = 0; k < nch; ++k) {
-        const int buf = k & 1;
-        tc::cp_async_wait_all();
-        tc::fence_async_smem();
-        __syncthreads();
+    // Chunk k's B tile sits in buffer k & 1 of shared memory and its scores in
+    // TMEM columns (k & 1) * 128. The MMAs of chunk k + 1 and the gather of
+    // chunk k + 2 run while the threads scan chunk k.
+    auto issue_mma = [&](int k) {
         if (tid == 0) {
             tc::tc_fence_after();
+            const int buf = k & 1;
             const int n = (int)min((int64_t)kBtCols, n_tile - (int64_t)k * kBtCols);
             const uint32_t idesc = idesc_n((n + 15) & ~15);
             const uint32_t dt = tmem + (uint32_t)(buf * 128);
@@ -158,10 +177,27 @@ __global__ void __launch_bounds__(kBtThreads, 1) bsa_tc_kernel(const __nv_bfloat
                              idesc, 1u);
             tc::mma_commit(&S.mbar[buf]);
         }
-        if (k + 1 < nch) gather(k + 1, buf ^ 1);  // the other buffer's MMAs completed before chunk k - 1's scan
+    };
+    gather(0, 0);  // the Q tile went out in the group before this one
+    if (nch > 1) gather(1, 1);
+    if (nch > 1) tc::cp_async_wait_group<1>();
+    else tc::cp_async_wait_all();
+    tc::fence_async_smem();
+    __syncthreads();
+    issue_mma(0);
+    for (int k = 0; k < nch; ++k) {
+        const int buf = k & 1;
         ok = __syncthreads_and(tc::mbar_wait(&S.mbar[buf], parity[buf], err, 17)) != 0;
         parity[buf] ^= 1u;
         if (!ok) break;
+        if (k + 2 < nch) gather(k + 2, buf);  // chunk k's MMAs have read this buffer
+        if (k + 1 < nch) {
+            if (k + 2 < nch) tc::cp_async_wait_group<1>();
+            else tc::cp_async_wait_all();
+            tc::fence_async_smem();
+            __syncthreads();  // chunk k + 1's tile is in place, and chunk k - 1's scan has left TMEM buffer buf ^ 1
+            issue_mma(k + 1);
+        }
         tc::tc_fence_after();
 #pragma unroll
         for (int gi = 0; gi < 2; ++gi) {
@@ -171,30 +207,54 @@ __global__ void __launch_bounds__(kBtThreads, 1) bsa_tc_kernel(const __nv_bfloat
             float v[32];
             tc::tmem_ld32(tmem + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)(buf * 128 + c0), v);
             tc::tmem_ld_wait();
+            // eligible columns of this slice: causal, not forced
+            const int64_t lim = c_max - leaf0 + 1;
+            uint32_t elig = lim >= 32 ? 0xffffffffu : (lim <= 0 ? 0u : (1u << lim) - 1u);
+            {
+                const int f[3] = {F.f0, F.f1, F.f2};
+#pragma unroll
+                for (int i = 0; i < 3; ++i)
+                    if (f[i] >= leaf0 && f[i] < leaf0 + 32) elig &= ~(1u << (f[i] - leaf0));
+            }
+            const float thr = lk[kTop - 1];
+            uint32_t cm = 0;
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
                 float z = v[j] * p.qscale;
 #pragma unroll
                 for (int o = 1; o < G; o <<= 1) z += __shfl_xor_sync(kFull, z, o);  // Eq.(11)-style sum over the group
-                if (live && z > thr) {  // rare once the list is full
-                    const int64_t leaf = leaf0 + j;
-                    if (leaf <= c_max && !F.has((int)leaf, 1)) {
-                        int i = Kp - 1;
-                        while (i > 0 && z > lk[i - 1]) {
-                            lk[i] = lk[i - 1];
-                            li[i] = li[i - 1];
-                            --i;
-                        }
-                        lk[i] = z;
-                        li[i] = (int)leaf;
-                        thr = lk[Kp - 1];
-                    }
+                v[j] = z;
+                cm |= (z > thr ? 1u : 0u) << j;
+            }
+            cm = live ? cm & elig : 0u;
+            if (__any_sync(kFull, cm != 0u)) {  // rare once the lists are full
+                float* zrow = S.zs[warp][lane];
+                if (cm) {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) zrow[j] = v[j];
                 }
+                while (cm) {  // the lanes with marked columns take one each per round
+                    const int j = __ffs(cm) - 1;
+                    cm &= cm - 1u;
+                    const float z = zrow[j];
+                    if (z > lk[kTop - 1]) top_insert(lk, li, z, (int)(leaf0 + j));
+                }
+                __syncwarp();
             }
         }
         tc::tc_fence_before();
     }
     tc::cp_async_wait_all();
+    __syncthreads();  // every MMA has completed (or the tile gave up): the tile buffers are free
+    BtLists& Ls = *reinterpret_cast<BtLists*>(S.b);
+    if (ok && live) {
+#pragma unroll
+        for (int i = 0; i < kTop; ++i) {
+            const bool real = lk[i] != INFINITY;  // placeholders rank below every leaf
+            Ls.key[wg][pos][i] = real ? lk[i] : -INFINITY;
+            Ls.id[wg][pos][i] = real ? li[i] : kNone;
+        }
+    }
     __syncthreads();
     if (ok) {
         // one warp per position: merge the two lists, add the forced leaves, sort ascending
@@ -203,8 +263,8 @@ __global__ void __launch_bounds__(kBtThreads, 1) bsa_tc_kernel(const __nv_bfloat
             if (tq >= p.N) continue;
             const Forced Fq(tq, p.C, p.causal, p.forced_mask);
             const int64_t cq = p.causal ? min(M1 - 1, (int64_t)tq / p.C) : M1 - 1;
-            float key = S.key[lane >> 4][q][lane & 15];
-            int id = S.id[lane >> 4][q][lane & 15];
+            float key = Ls.key[lane >> 4][q][lane & 15];
+            int id = Ls.id[lane >> 4][q][lane & 15];
             warp_sort_desc(key, id, lane);
             // the eligible forced leaves, each once
             int fl[3], nfq = 0;
