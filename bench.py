@@ -475,6 +475,49 @@ def prefill_config_line(w, dev, stream, steps, warmup, pk, fma_peak, fma_note, t
 
 
 PER_CONFIG = ("mha16_n16k", "needle_mha16_n64k", "gqa32x8_n128k")
+SWEEP_N = (262144, 524288, 1048576)
+
+
+def selection_sweep(w, dev, stream, ns=SWEEP_N, reps: int = 3):
+    """PISA's selection against flat BSA's on the headline workload's shape at
+    growing N (both from the keys: the pyramid, then the selection; PISA
+    through pisa_select_ws, BSA on the tensor cores), to locate where the
+    log-linear walk overtakes the quadratic contraction on this GPU. Inputs
+    are i.i.d. N(0, 1) in bf16, drawn on the device (seeded) to keep the
+    sweep's host time short."""
+    import torch
+    from hierarchical_block_sparse_b200 import pisa
+    out = {}
+    gen = torch.Generator(device=dev)
+    for n in ns:
+        gen.manual_seed(1000 + n)
+        Qd = torch.randn((w.B, w.Hq, n, w.d), generator=gen, device=dev, dtype=torch.float32).to(torch.bfloat16)
+        Kd = torch.randn((w.B, w.Hkv, n, w.d), generator=gen, device=dev, dtype=torch.float32).to(torch.bfloat16)
+        cfg = pisa.cfg_for(Qd, Kd, C=w.C, K_=w.K, causal=w.causal, forced_mask=w.forced_mask)
+        pyr = torch.empty((w.B, w.Hkv, pisa.pisa_pyramid_rows(cfg), w.d), dtype=torch.float32, device=dev)
+        idx = torch.empty((w.B, w.Hkv, n, w.K), dtype=torch.int32, device=dev)
+        work = pisa.alloc_workspace(cfg, dev)
+
+        def run():
+            pisa.pisa_build_pyramid(cfg, Kd, pyr)
+            pisa.pisa_select_ws(cfg, Qd, Kd, pyr, idx, work)
+
+        run()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            run()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if pisa.pisa_workspace_status(cfg, work) != 0:
+            raise RuntimeError(f"a tensor-core tile timed out (selection sweep, N = {n})")
+        p_ms = e0.elapsed_time(e1) / reps
+        b_ms = time_bsa(cfg, Qd, Kd, pyr, idx, stream, work, reps=reps)
+        out[str(n)] = {"pisa_selection_ms": p_ms, "bsa_selection_ms": b_ms, "pisa_vs_bsa_selection_speedup": b_ms / p_ms}
+        del Qd, Kd, pyr, idx, work
+        torch.cuda.empty_cache()
+    return out
 
 
 # -------------------------------------------------------------------- main ----
@@ -492,6 +535,7 @@ def main():
     ap.add_argument("--no-backward", action="store_true", help="skip timing the attention backward")
     ap.add_argument("--no-per-query", action="store_true")
     ap.add_argument("--no-per-config", action="store_true", help="skip the 16K / 64K / 128K workloads")
+    ap.add_argument("--no-sweep", action="store_true", help="skip the PISA vs BSA selection sweep over N")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=16.0)
     ap.add_argument("--decode-batch", type=int, default=0, help="override the decode batch (profiling)")
@@ -802,6 +846,11 @@ def main():
         out["per_config"] = per
         out["selection_ms_by_n"] = {str(v["N"]): v["selection_ms"] for v in per.values()}
         out["selection_ms_by_n"][str(w.N)] = sel_total
+
+    # ---- PISA vs flat BSA selection beyond the headline N (the crossover) ----
+    if not args.no_bsa and not args.no_sweep and world == 1 and w.name == "mha8_n256k":
+        out["selection_sweep"] = {"workload": "mha8 shape (B 1, 8 heads, d 128, C 64, K 16), N varied",
+                                  "by_n": selection_sweep(w, dev, stream)}
 
     if dist:
         dist.barrier()
