@@ -810,18 +810,26 @@ def main():
         g1.record(stream)
         torch.cuda.synchronize()
         pq_ms = max_over_ranks(g0.elapsed_time(g1), dist, dev)
-        out["backward"] = {"ms": bms, "tokens_per_s": job_tokens_per_s(w.B * w.N, world, bms),
-                           "call": "pisa_sparse_attn_backward_ws",
-                           "kernel": "bwd_tile_kernel (key-major tcgen05 tiles; dK, dV in TMEM per leaf) after "
-                                     "the statistics pass (bwd_stats_kernel: per-leaf LSE and P-weighted dP)",
-                           "phase_ms": {name: float(np.mean([e[i].elapsed_time(e[i + 1]) for e in bev]))
-                                        for i, name in enumerate(pisa.BWD_PHASES)},
-                           "algorithmic_tflop": bflops / 1e12, "achieved_tflops": bflops / (bms / 1e3) / 1e12,
+        # Training keeps the forward's workspace: the backward then starts from
+        # the normaliser and fp32 output the forward left there (the headline
+        # figure); the standalone call recomputes them from Q, K, V, dO and idx.
+        sflops = alg["attn_flops"] * 10.0 / 4.0  # logits, dP, dQ, dK, dV: 10d per (query head, key)
+        out["backward"] = {"ms": saved_ms, "tokens_per_s": job_tokens_per_s(w.B * w.N, world, saved_ms),
+                           "call": "pisa_sparse_attn_backward_saved_ws (after pisa_forward_ws, whose workspace "
+                                   "keeps the normaliser and the fp32 output)",
+                           "kernel": "bwd_tile_kernel (key-major tcgen05 tiles; dK, dV in TMEM per leaf; dQ rows "
+                                     "by bulk reductions)",
+                           "algorithmic_tflop": sflops / 1e12, "achieved_tflops": sflops / (saved_ms / 1e3) / 1e12,
                            "bf16_tensor_peak_tflops": tc_peak,
-                           "frac": bflops / (bms / 1e3) / 1e12 / tc_peak,
+                           "frac": sflops / (saved_ms / 1e3) / 1e12 / tc_peak,
                            "tiles_dram_bytes": measured_traffic("backward_tiles", w.name),
-                           "saved_state_ms": saved_ms,
-                           "saved_state_call": "pisa_sparse_attn_backward_saved_ws (after pisa_forward_ws)",
+                           "standalone_ms": bms,
+                           "standalone_call": "pisa_sparse_attn_backward_ws (statistics recomputed: bwd_stats_kernel, "
+                                              "per-leaf LSE and P-weighted dP)",
+                           "standalone_phase_ms": {name: float(np.mean([e[i].elapsed_time(e[i + 1]) for e in bev]))
+                                                   for i, name in enumerate(pisa.BWD_PHASES)},
+                           "standalone_algorithmic_tflop": bflops / 1e12,
+                           "standalone_frac": bflops / (bms / 1e3) / 1e12 / tc_peak,
                            "per_query_cuda_core_ms": pq_ms,
                            "per_query_cuda_core_frac_of_fp32_fma": bflops / (pq_ms / 1e3) / 1e12 / fma_peak}
         del dOd, dQ, dK, dV
