@@ -263,7 +263,7 @@ __global__ void __launch_bounds__(kTwThreads, 1) walk_tc_kernel(
     constexpr int SPL = kSlots / LPP;  // candidate slots per lane
     extern __shared__ __align__(1024) uint8_t dsm[];
     TwSmem& S = *reinterpret_cast<TwSmem*>(dsm);
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int tid = threadIdx.x, warp = tid >> 5;
 
     // heaviest tiles (latest positions: the largest unions) first
     const int64_t nbh = (int64_t)p.B * p.Hkv;
@@ -458,32 +458,41 @@ __global__ void __launch_bounds__(kTwThreads, 1) walk_tc_kernel(
                 mask |= (dlt >= 0 && dlt < kTwPar) ? (1u << dlt) : 0u;
                 base += uj[j] < c0u ? 1 : 0;
             }
-#pragma unroll
-            for (int gi = 0; gi < 2; ++gi) {
-                const int g = 2 * wg + gi;  // 8 parents: columns 32 g .. 32 g + 31
-                const uint32_t m8 = (mask >> (8 * g)) & 0xffu;
-                if (!__any_sync(kFull, m8 != 0u)) continue;
-                __syncwarp();
-                float v[32];
-                tc::tmem_ld32(tmem + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)(buf * 128 + g * 32), v);
+            // this warp's two column groups (8 parents each: columns 32 g .. 32 g + 31):
+            // both loads go out before the one wait
+            const uint32_t m2[2] = {(mask >> (16 * wg)) & 0xffu, (mask >> (16 * wg + 8)) & 0xffu};
+            const bool need[2] = {__any_sync(kFull, m2[0] != 0u) != 0, __any_sync(kFull, m2[1] != 0u) != 0};
+            if (need[0] || need[1]) {
+                float v[2][32];
+                const uint32_t ta = tmem + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)(buf * 128 + 64 * wg);
+                if (need[0]) tc::tmem_ld32(ta, v[0]);
+                if (need[1]) tc::tmem_ld32(ta + 32u, v[1]);
                 tc::tmem_ld_wait();
-                const int before = base + __popc(mask & ((1u << (8 * g)) - 1u));
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    if ((m8 >> i) & 1u) {
-                        const int j = before + __popc(m8 & ((1u << i) - 1u));  // its place in the kept list
-                        const int par = S.uni[c0u + 8 * g + i];
-                        // children 4 par + 1 and 4 par + 3 (the second child of each candidate) may not exist
-                        const bool has1 = 4 * par + 1 < child_rows, has3 = 4 * par + 3 < child_rows;
-                        const float z0 = v[4 * i] * p.qscale, z1 = has1 ? v[4 * i + 1] * p.qscale : -INFINITY;
-                        const float z2 = v[4 * i + 2] * p.qscale, z3 = has3 ? v[4 * i + 3] * p.qscale : -INFINITY;
-                        float* sc = S.score + pos * (kSlots * G + 1) + 2 * j * G + h;
-                        if (p.variant == 0) {  // Eq.(7): the LSE over the two children
-                            sc[0] = lse2_pair(z0, z1);
-                            sc[G] = lse2_pair(z2, z3);
-                        } else {
-                            sc[0] = pair_score(z0, z1, p.variant);
-                            sc[G] = pair_score(z2, z3, p.variant);
+                for (int gi = 0; gi < 2; ++gi) {
+                    const int g = 2 * wg + gi;
+                    const uint32_t m8 = m2[gi];
+                    if (!need[gi]) continue;
+                    const int before = base + __popc(mask & ((1u << (8 * g)) - 1u));
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        if ((m8 >> i) & 1u) {
+                            const int j = before + __popc(m8 & ((1u << i) - 1u));  // its place in the kept list
+                            const int par = S.uni[c0u + 8 * g + i];
+                            // children 4 par + 1 and 4 par + 3 (the second child of each candidate) may not exist
+                            const bool has1 = 4 * par + 1 < child_rows, has3 = 4 * par + 3 < child_rows;
+                            const float z0 = v[gi][4 * i] * p.qscale;
+                            const float z1 = has1 ? v[gi][4 * i + 1] * p.qscale : -INFINITY;
+                            const float z2 = v[gi][4 * i + 2] * p.qscale;
+                            const float z3 = has3 ? v[gi][4 * i + 3] * p.qscale : -INFINITY;
+                            float* sc = S.score + pos * (kSlots * G + 1) + 2 * j * G + h;
+                            if (p.variant == 0) {  // Eq.(7): the LSE over the two children
+                                sc[0] = lse2_pair(z0, z1);
+                                sc[G] = lse2_pair(z2, z3);
+                            } else {
+                                sc[0] = pair_score(z0, z1, p.variant);
+                                sc[G] = pair_score(z2, z3, p.variant);
+                            }
                         }
                     }
                 }

@@ -48,9 +48,14 @@ def test_blockmajor_small_every_row(name):
     _report("ws:" + name, stats)
 
 
-@pytest.mark.parametrize("name", ["mha16_n16k", "needle_mha16_n64k", "gqa32x8_n128k", "mha8_n256k"])
+# a group of 16 query heads per KV head (8 positions per tile) at a size where
+# the tile walk hands its fine levels to the one-warp walk
+LARGE = {"gqa32x2_n64k": Workload("gqa32x2_n64k", 136, B=1, Hq=32, Hkv=2, N=65536, d=128, C=64, K=16)}
+
+
+@pytest.mark.parametrize("name", ["mha16_n16k", "needle_mha16_n64k", "gqa32x8_n128k", "mha8_n256k", "gqa32x2_n64k"])
 def test_blockmajor_named_workload_full_size(name):
-    w = WORKLOADS[name]
+    w = WORKLOADS[name] if name in WORKLOADS else LARGE[name]
     Q, K, V, _ = make_inputs(w)
     res = parity.gpu_prefill(w, Q, K, V, ws=True)
     idx = res["idx"]
