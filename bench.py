@@ -904,6 +904,9 @@ def bench_decode(w, dev, stream, steps: int = 8, batch: int = 0, cache: int = 0)
         pos += 1
     torch.cuda.synchronize()
     evf = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
+    # a short device-side wait first, so the host enqueues the steps while the
+    # stream is busy and the events bracket the kernels, not the launch latency
+    torch.cuda._sleep(10_000_000)
     for s in range(steps):
         q, k, v = ins[3 + s]
         evf[s][0].record(stream)
@@ -911,6 +914,7 @@ def bench_decode(w, dev, stream, steps: int = 8, batch: int = 0, cache: int = 0)
         evf[s][1].record(stream)
         pos += 1
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    torch.cuda._sleep(10_000_000)
     for s in range(steps):
         q, k, v = ins[3 + steps + s]
         ev[s][0].record(stream)
