@@ -18,7 +18,7 @@
 // summaries to about 2^-16 of their size (about 1e-5 on a logit). Each row
 // reads the four columns of each of its own kept parents (found with a
 // bitmask per chunk) and writes its candidates' pair scores to shared memory;
-// two adjacent lanes per position then rank them with the walk's keep rule.
+// 2G adjacent lanes per position then rank them with the walk's keep rule.
 //
 // The levels above the first one where some position of the tile has more
 // than K eligible nodes are not walked: there every eligible node is kept.
@@ -60,7 +60,7 @@ constexpr int kRow = 17;  // padded row of the per-position lists (one thread pe
 struct TwSmem {
     uint8_t q[32768];        // A: 128 rows x 128 bf16, K-major canonical layout
     uint8_t b[2][2][32768];  // B[buffer][hi, lo]: 128 rows x 128 bf16
-    float score[128 * kSlots + 128];  // position p, slot c, head h at p * (32 G + 1) + c * G + h
+    float score[128 * kSlots];  // slot c, MMA row r at score_at<G>(c, r)
     int32_t kept[128][kRow];  // kept nodes of the level above, ascending
     int32_t keptu[128][kRow]; // their index in the union
     int32_t uni[kTwMaxUnion];
@@ -72,6 +72,21 @@ struct TwSmem {
     uint64_t mbar[2];
     uint32_t tmem_base;
 };
+
+// Place of (slot c, MMA row r = position * G + head) in TwSmem::score: slot
+// major, the row XOR-swizzled by the slot's lane group q = c / SPL (2G lanes
+// per position, SPL = 32 / 2G slots per lane). A warp's pick-up stores (32
+// consecutive rows, any slots) land in distinct banks but for pairs of rows
+// 16 apart; a warp's ranking reads (16 consecutive rows, for a fixed head and
+// slot index the 2G lanes of each position in different groups q) flip the
+// head bits and bit 4 of the row by q, so they meet 32 distinct banks.
+template <int G>
+__device__ __forceinline__ int score_swz(int q) { return (q & (G - 1)) | ((q / G) << 4); }
+template <int G>
+__device__ __forceinline__ int score_at(int c, int r) {
+    constexpr int SPL = kSlots / (2 * G);
+    return c * 128 + (r ^ score_swz<G>(c / SPL));
+}
 
 // exclusive scan of one int per thread over the 256 threads; returns the total
 __device__ __forceinline__ int block_exscan(int& v, int32_t* scan) {
@@ -413,7 +428,7 @@ __global__ void __launch_bounds__(kTwThreads, 1) walk_tc_kernel(
         };
         // this thread's row and its walk over its position's kept parents
         const int r = tid & 127, wg = tid >> 7;
-        const int pos = r / G, h = r % G;
+        const int pos = r / G;
         const bool mine = pos < P && t0 + pos < p.N && S.need[pos];
         const int nk = mine ? S.nkept[pos] : 0;
         int uj[16];  // union index of each of its kept parents (ascending; kBig past the count)
@@ -485,13 +500,14 @@ __global__ void __launch_bounds__(kTwThreads, 1) walk_tc_kernel(
                             const float z1 = has1 ? v[gi][4 * i + 1] * p.qscale : -INFINITY;
                             const float z2 = v[gi][4 * i + 2] * p.qscale;
                             const float z3 = has3 ? v[gi][4 * i + 3] * p.qscale : -INFINITY;
-                            float* sc = S.score + pos * (kSlots * G + 1) + 2 * j * G + h;
+                            float* sc0 = S.score + score_at<G>(2 * j, r);
+                            float* sc1 = S.score + score_at<G>(2 * j + 1, r);
                             if (p.variant == 0) {  // Eq.(7): the LSE over the two children
-                                sc[0] = lse2_pair(z0, z1);
-                                sc[G] = lse2_pair(z2, z3);
+                                *sc0 = lse2_pair(z0, z1);
+                                *sc1 = lse2_pair(z2, z3);
                             } else {
-                                sc[0] = pair_score(z0, z1, p.variant);
-                                sc[G] = pair_score(z2, z3, p.variant);
+                                *sc0 = pair_score(z0, z1, p.variant);
+                                *sc1 = pair_score(z2, z3, p.variant);
                             }
                         }
                     }
@@ -510,17 +526,19 @@ __global__ void __launch_bounds__(kTwThreads, 1) walk_tc_kernel(
             LaneCands<SPL> lc;
             lane_cands<SPL>(S, pos, l, L, live ? t0 + pos : 0, p, q, live, lc);
             const uint32_t vfull = group_mask<SPL>(lc.v, q), ffull = group_mask<SPL>(lc.f, q);
-            float* sc = S.score + pos * (kSlots * G + 1) + q * SPL * G;
+            // this lane's slots q * SPL + i of the first head: sc[i * 128]
+            const int swz = score_swz<G>(q);
+            float* sc = S.score + q * SPL * 128 + ((pos * G) ^ swz);
             if (G > 1 && live) {  // Eq.(11): summed over the group, into the first head's entry
 #pragma unroll
                 for (int i = 0; i < SPL; ++i) {
                     float x = 0.f;
 #pragma unroll
-                    for (int hh = 0; hh < G; ++hh) x += sc[i * G + hh];
-                    sc[i * G] = x;
+                    for (int hh = 0; hh < G; ++hh) x += S.score[(q * SPL + i) * 128 + ((pos * G + hh) ^ swz)];
+                    sc[i * 128] = x;
                 }
             }
-            const uint32_t keep = rank_keep<SPL>(sc, G, vfull, ffull, p.K, q);
+            const uint32_t keep = rank_keep<SPL>(sc, 128, vfull, ffull, p.K, q);
             __syncwarp();  // the group's lanes have read the kept nodes they expand
             if (live) write_kept<SPL>(S, pos, lc, keep, q);
         }
