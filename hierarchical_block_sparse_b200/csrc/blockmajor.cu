@@ -67,8 +67,10 @@ constexpr int kORowStride = kD * 4 + 16;  // staged fp32 output row: 16-byte pad
 // resume[unit] is 0 for a position it finished, else (resume level << 8 |
 // count) with the kept nodes in cand_out's row, which this kernel reads
 // before it overwrites the row with the level-1 candidates.
+// (below the tile walk, the group-of-4+ walker runs faster with the registers
+// of 3 CTAs per SM, no spills; the group-of-1-2 one with 4)
 template <int G, class W, bool RESUME = false>
-__global__ void __launch_bounds__(256, PISA_STAGE1_MINBLOCKS) stage1_kernel(const __nv_bfloat16* __restrict__ Q,
+__global__ void __launch_bounds__(256, (RESUME && G >= 4) ? 3 : PISA_STAGE1_MINBLOCKS) stage1_kernel(const __nv_bfloat16* __restrict__ Q,
                                                      const float* __restrict__ pyr, int32_t* __restrict__ cand_out,
                                                      int32_t* __restrict__ counts, int32_t* __restrict__ slots,
                                                      int64_t M1, int* __restrict__ err, SelectParams p,
