@@ -3,12 +3,19 @@
 selection -> sparse attention) on B200, one process per GPU.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl pisa|reference]
-                    [--workload mha8_n256k] [--no-decode] [--no-cpu-baseline]
+                    [--workload mha8_n256k] [--seq N] [--no-decode] [--no-cpu-baseline]
+                    [--no-bsa] [--no-sweep] [--no-per-config] [--no-backward]
+                    [--no-variants] [--no-per-query] [--decode-only]
 
-A step is one pisa_forward over the whole workload (B*N tokens, all heads)
-with inputs resident in HBM. Rank 0 prints one JSON line. Under torchrun
-every rank runs its own seeded copy of the workload (weak scaling, no
-data-path collective); the time is the max over ranks.
+A step is one pisa_forward_ws over the whole workload (B*N tokens, all
+heads) with inputs resident in HBM. Rank 0 prints one JSON line: the step,
+its phases and the dominant phase's roofline, the end-to-end figure through
+pisa_forward_host from pinned host buffers, the other prefill workloads,
+flat BSA selection beside PISA's (and a sweep of both to 1M tokens), the
+PISA-1 / PISA-2 scores, the backward with the selection fixed, the decode
+step and the oracle's CPU baseline. Under torchrun every rank runs its own
+seeded copy of the workload (weak scaling, no data-path collective); the
+time is the max over ranks.
 """
 from __future__ import annotations
 
