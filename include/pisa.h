@@ -167,14 +167,17 @@ int pisa_bsa_select_ws(const pisa_cfg *cfg, const void *Q, const float *pyr, int
                        size_t workspace_bytes, void *stream);
 
 /* ---- block-major tensor-core prefill (close reading §05 Algorithm 1, §5.1) ------
- * The pages' two-stage form: Stage 1 walks the internal levels per query;
- * Stage 2 groups the (query, candidate leaf) pairs by leaf so that each leaf's
+ * The pages' two-stage form: Stage 1 walks the internal levels (here the
+ * coarse ones for tiles of consecutive positions on the tensor cores, the fine
+ * ones per query); Stage 2 groups the (query, candidate leaf) pairs by leaf so that each leaf's
  * 64 keys are loaded once per tile of up to 128 query rows and scored with one
  * tcgen05 MMA (exact leaf LSE in the epilogue, Eq.(7)); a final Top-K per
  * query follows. Attention runs the same way: per (leaf, tile of queries that
  * kept it) S = Q K^T and O += softmax-weighted V on the tensor cores, using the
  * per-query normaliser taken from the leaf LSEs. Results equal pisa_select /
- * pisa_sparse_attn up to fp32 rounding.
+ * pisa_sparse_attn up to fp32 rounding (a row whose keep decision has a
+ * margin below about 1e-5 may differ: the tile walk takes the fp32 summaries
+ * as bf16 high and low parts).
  * Limits: dtype bf16, d = 128, C = 64, K <= 16, G in {1,2,4,8,16}, N < 2^27,
  * B * Hkv * N * 32 < 2^31, B * Hkv <= 65535. Other shapes return
  * PISA_E_UNSUPPORTED. The pyramid pointer must be 32-byte aligned (its rows are
