@@ -247,3 +247,24 @@ def test_select_noalloc_status_validates(lib):
     assert lib.pisa_select_noalloc_status(ctypes.byref(bad), None) == -2
     empty = pisa.make_cfg(B=1, Hq=2, Hkv=2, N=0, d=128, C=64, K=8)
     assert lib.pisa_select_noalloc_status(ctypes.byref(empty), None) == 0
+
+
+def test_bsa_select_ws_and_fma_probe_validate_before_launch(lib):
+    cfg = pisa.make_cfg(B=1, Hq=2, Hkv=2, N=1000, d=128, C=64, K=8)
+    need = pisa.pisa_workspace_bytes(cfg)
+    Q, pyr, idx = ctypes.c_void_p(4096), ctypes.c_void_p(8192), ctypes.c_void_p(12288)
+    ws = ctypes.c_void_p(1 << 20)
+    f = lib.pisa_bsa_select_ws
+    assert f(ctypes.byref(cfg), Q, pyr, idx, None, need, None) == -1                     # no workspace
+    assert f(ctypes.byref(cfg), Q, pyr, idx, ctypes.c_void_p((1 << 20) + 16), need, None) == -4  # misaligned
+    assert f(ctypes.byref(cfg), Q, pyr, idx, ws, need - 1, None) == -1                    # too small
+    assert f(ctypes.byref(cfg), None, pyr, idx, ws, need, None) == -1                     # no Q
+    assert f(ctypes.byref(cfg), ctypes.c_void_p(4096 + 8), pyr, idx, ws, need, None) == -4  # Q misaligned
+    bad = pisa.make_cfg(B=1, Hq=2, Hkv=2, N=1000, d=128, C=32, K=8)
+    assert f(ctypes.byref(bad), Q, pyr, idx, ws, need, None) == -2                        # C != 64
+    empty = pisa.make_cfg(B=1, Hq=2, Hkv=2, N=0, d=128, C=64, K=8)
+    assert f(ctypes.byref(empty), None, None, None, None, 0, None) == 0                   # nothing to do
+    p = lib.pisa_fma_probe
+    assert p(None, 148, 10, 0, None) == -1
+    assert p(ctypes.c_void_p(4096), 0, 10, 0, None) == -1
+    assert p(ctypes.c_void_p(4096), 148, 0, 1, None) == -1
